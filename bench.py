@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Throughput of the BERT-style encoder forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload KIND:BATCH[:SEQ]] [--no-cpu-baseline]
+
+A step is one enc_forward over one batch of the workload (every layer, every
+kernel of the path), inputs already in HBM; the L2 is flushed (256 MiB write)
+before every timed step.  value = sequences/s over all ranks (weak scaling:
+each rank runs its own batch; no collective on the data path).  e2e = the same
+metric through enc_forward_host (pinned host input, copies inside the timed
+region).  The per-kernel breakdown and the roofline come from CUDA events the
+library records between its kernels on the launching stream, during the timed
+steps.  --impl reference times the float64 CPU oracle on a bounded sample.
+Default workload: 12-layer BERT-Base shape (12x64, FFN 3072), seq 32, batch 512.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import encoder_inputs as EI  # noqa: E402
+
+METRIC = "BERT-Base FP16 encoder fwd sequences/s (seq 32/128); % tensor/HBM roofline"
+UNIT = "sequences/s"
+DEFAULT_WORKLOAD = "bert-base-s32:512"
+KERNEL_NAMES = ["qkv_gemm", "attention", "out_proj_gemm", "ln1", "ffn1_gemm", "ffn2_gemm", "ln2"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_workload(spec: str) -> EI.Workload:
+    parts = spec.split(":")
+    kind, batch = parts[0], int(parts[1])
+    seq = int(parts[2]) if len(parts) > 2 else None
+    return EI.named_workload(kind, batch, seq)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ algorithmic work per kernel
+def kernel_work(wl: EI.Workload):
+    """Per launch: (flops, algorithmic HBM bytes) of each kernel of one layer (FP16 storage)."""
+    sh = wl.shape
+    H, F, M, S = sh.hidden, sh.ffn_dim, wl.tokens, wl.seq
+    es = 2 if wl.dtype == "fp16" else 4
+    def gemm(n, k, extra_out=0):
+        return 2.0 * M * n * k, es * (M * k + k * n + M * n) + extra_out
+    return {
+        "qkv_gemm": gemm(3 * H, H),
+        "attention": (4.0 * M * S * H, es * 4.0 * M * H + 4 * wl.batch),
+        "out_proj_gemm": gemm(H, H),
+        "ln1": (0.0, es * 3.0 * M * H),
+        "ffn1_gemm": gemm(F, H),
+        "ffn2_gemm": gemm(H, F),
+        "ln2": (0.0, es * 3.0 * M * H),
+    }
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        self.index = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{local_rank}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [v.strip() for v in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx.append(float(p[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, p[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_rate(inp: EI.EncoderInputs, budget_s: float, chunk: int = 4, max_seqs=None, widened=None):
+    """Sequences/s of the float64 oracle on sequences 0, 1, ... until budget_s elapses
+    (the inputs are widened to float64 before the clock starts)."""
+    from oracle import encoder_oracle as O
+    wl = inp.workload
+    sh = wl.shape
+    x64, vl, layers = widened if widened is not None else inp.as_float64()
+    done, t0 = 0, time.perf_counter()
+    limit = wl.batch if max_seqs is None else min(wl.batch, max_seqs)
+    while done < limit:
+        idx = list(range(done, min(done + chunk, limit)))
+        O.encoder_forward(x64, vl, layers, sh.head_num, sh.size_per_head, seqs=idx)
+        done += len(idx)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def run_reference(args, wl: EI.Workload, rank: int, world: int):
+    if rank != 0:
+        return 0
+    inp = EI.make_inputs(wl)
+    sample = max(1, args.ref_sample)
+    widened = inp.as_float64()
+    times = []
+    for i in range(args.warmup + args.steps):
+        _, n, dt = oracle_rate(inp, budget_s=1e9, chunk=sample, max_seqs=sample, widened=widened)
+        if i >= args.warmup:
+            times.append(dt)
+    step_s = sum(times) / len(times)
+    value = sample / step_s
+    cores = blas_threads()
+    desc = f"float64 numpy oracle, first {sample} sequences of the workload per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, world, l2="n/a (CPU)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl: EI.Workload, world: int, l2: str):
+    sh = wl.shape
+    return {"workload": wl.name, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+            "seq_len": wl.seq, "layers": sh.num_layers, "heads": sh.head_num, "size_per_head": sh.size_per_head,
+            "ffn": sh.ffn_dim, "valid_len": f"U[{wl.valid_lo},{wl.valid_hi}]", "storage": wl.dtype,
+            "accumulate": "fp32", "parallelism": f"replicas x{world} (batch-sharded, no collective)",
+            "l2": l2, "seed": wl.seed}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from transformer_encoder_bert_b200 import Encoder
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = wl.with_(seed=wl.seed + rank)          # each replica has its own batch
+    inp = EI.make_inputs(wl)
+    sh = wl.shape
+    enc = Encoder(sh.head_num, sh.size_per_head, sh.ffn_dim, inp.layers, wl.dtype)
+    enc.reserve(wl.batch, wl.seq)
+    x = torch.from_numpy(inp.x).to(dev)
+    vl = torch.from_numpy(inp.valid_len).to(dev)
+    out = torch.empty_like(x)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        enc.forward(x, vl, out)
+    torch.cuda.synchronize()
+
+    nk = enc.kernels_per_forward()
+    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for evs in ev_sets:                                   # create the events before the timed region
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = enc.launch_count()
+    for i in range(args.steps):
+        flush.zero_()
+        enc.set_trace_events(ev_sets[i], prepare=False)
+        starts[i].record(stream)
+        enc.forward(x, vl, out)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = enc.launch_count() - launches0
+    clk = clocks.stop()
+    enc.set_trace_events(None)
+
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+    per_kernel = {k: [] for k in KERNEL_NAMES}
+    for evs in ev_sets:
+        for j in range(nk):
+            per_kernel[KERNEL_NAMES[j % 7]].append(evs[j].elapsed_time(evs[j + 1]))
+
+    # e2e through enc_forward_host: pinned host input, copies inside the timed region.
+    hx = torch.from_numpy(inp.x).pin_memory()
+    hvl = torch.from_numpy(inp.valid_len).pin_memory()
+    hout = torch.empty_like(hx).pin_memory()
+    for _ in range(2):
+        enc.forward_host_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), wl.batch, wl.seq)
+    e2e_ms = []
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        enc.forward_host_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), wl.batch, wl.seq)
+        e.record(stream)
+        e.synchronize()
+        e2e_ms.append(s.elapsed_time(e))
+    barrier()
+    e2e_step = sum(e2e_ms) / len(e2e_ms)
+    status = enc.device_status()
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_step = float(t[0]), float(t[1])
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    work = kernel_work(wl)
+    kernels = {}
+    total = sum(sum(v) for v in per_kernel.values())
+    for k in KERNEL_NAMES:
+        vals = per_kernel[k]
+        avg_ms = sum(vals) / len(vals)
+        flops, nbytes = work[k]
+        entry = {"avg_us": avg_ms * 1e3, "share": sum(vals) / total}
+        if flops and k.endswith("gemm"):
+            entry["tflops"] = flops / (avg_ms * 1e-3) / 1e12
+        entry["gbs"] = nbytes / (avg_ms * 1e-3) / 1e9
+        kernels[k] = entry
+    dominant = max(KERNEL_NAMES, key=lambda k: kernels[k]["share"])
+    d = kernels[dominant]
+    if dominant.endswith("gemm"):
+        peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        roof = {"bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
+                "frac": d["tflops"] / peak, "traffic": args.traffic,
+                "kernel": dominant, "per_launch_flops": work[dominant][0],
+                "peak_source": f"{peak_src} sustained bf16 matmul (FP16 dense rate = BF16 dense rate)"}
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": d["gbs"], "peak": peak, "unit": "GB/s", "frac": d["gbs"] / peak,
+                "traffic": args.traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
+                "peak_source": f"{peak_src} HBM copy bandwidth"}
+
+    value = wl.batch * world / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp16" if wl.dtype == "fp16" else "fp32", "data": "synthetic",
+        "config": workload_config(wl, world, l2="flushed before every timed step (256 MiB write)"),
+        "roofline": roof,
+        "e2e": {"value": wl.batch * world / (e2e_step * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(hx.numel() * hx.element_size() + hvl.numel() * 4),
+                "d2h_bytes_per_step": int(hout.numel() * hout.element_size())},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "kernels": kernels,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, n, dt = oracle_rate(inp, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"first {n} of the {wl.batch} sequences of this workload, "
+                                          f"float64 numpy oracle, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-sample", type=int, default=8, help="sequences per reference-arm step")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per launch of the dominant kernel, if captured for this build")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    wl = parse_workload(args.workload)
+
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,203 @@
+/*
+ * enc.h - C ABI of a B200 (sm_100a) library for the forward pass of a
+ * BERT-style post-LayerNorm Transformer encoder stack.
+ *
+ * Source page: "有钱任性：英伟达训练80亿参数量GPT-2，1475块V100 53分钟训练BERT"
+ * (机器之心; the Faster Transformer write-up), cited as [FT] with a section.
+ *
+ *  - [FT] "什么是 Faster Transformer": the encoder forward is the whole
+ *    product; the network structure is fixed by head_num and size_per_head,
+ *    and batch size and maximum sequence length are given per run; the
+ *    computation runs in FP32 or in FP16 (FP16 on tensor cores); the library
+ *    offers a C++ API.  Unlike the page's fixed lengths (32/64/128), any
+ *    sequence length >= 1 is accepted here.
+ *  - [FT] "Faster Transformer 优化原理": per layer, the matrix multiplies run
+ *    on tensor cores and every other operation is fused into as few kernels
+ *    as possible (add-bias/transposes, SoftMax, add-bias + residual +
+ *    LayerNorm, add-bias + GELU).
+ *
+ * Per layer (x: [batch, seq, H], H = head_num * size_per_head, F = ffn_dim):
+ *   QKV = x Wqkv + bqkv;  per head: ctx = softmax(Q K^T / sqrt(d), keys j < n) V
+ *   H1  = LN(x + ctx Wo + bo; ln1);   U = GELU(H1 W1 + b1)  (erf form)
+ *   out = LN(H1 + U W2 + b2; ln2)
+ * with n = clamp(valid_len[b], 0, seq); LN eps = 1e-12, biased variance.
+ * Query rows i >= n are computed (attending to the n valid keys) but are not
+ * meaningful to callers; n == 0 gives ctx = 0 for that sequence.
+ *
+ * Numerics: FP16 mode stores every tensor in IEEE half and accumulates every
+ * matmul, softmax and LayerNorm in FP32 (no half accumulation).  FP32 mode
+ * stores and computes in FP32 on CUDA cores (no TF32).
+ *
+ * Threading and streams: every call is asynchronous on the given stream
+ * unless stated.  A handle owns one workspace, so it must not be used by two
+ * streams at once.  Device-side faults surface at the caller's next
+ * synchronisation, as with any CUDA launch.
+ */
+#ifndef BERT_ENCODER_B200_ENC_H
+#define BERT_ENCODER_B200_ENC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ENC_API __attribute__((visibility("default")))
+#else
+#define ENC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream (a pointer to the driver's stream object); NULL = legacy default stream. */
+typedef struct CUstream_st* enc_stream_t;
+
+typedef struct enc_handle* enc_t;
+
+typedef enum {
+  ENC_OK = 0,
+  ENC_ERR_INVALID_ARG = 1,   /* a host-side argument check failed; nothing was enqueued */
+  ENC_ERR_UNSUPPORTED = 2,   /* valid but not supported (e.g. size_per_head not in {32,64,128}) */
+  ENC_ERR_OOM = 3,           /* a device allocation failed; the handle stays usable */
+  ENC_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed; see enc_last_error() */
+  ENC_ERR_DEVICE = 5         /* a kernel reported a failure through the handle's device status word */
+} enc_status;
+
+typedef enum { ENC_FP32 = 0, ENC_FP16 = 1 } enc_dtype;
+
+/* One layer's parameters.  Element type = the handle's dtype (float or IEEE half).
+ * Matrices are [in, out] row-major (y = x W + b).  Wqkv's columns are Q | K | V,
+ * and inside each block head h owns columns h*d .. h*d+d-1.  The pointers may be
+ * host or device memory (detected per pointer); they are only read during
+ * enc_create. */
+typedef struct {
+  const void* w_qkv; const void* b_qkv;   /* [H, 3H], [3H] */
+  const void* w_o;   const void* b_o;     /* [H, H],  [H]  */
+  const void* ln1_g; const void* ln1_b;   /* [H], [H] */
+  const void* w_ff1; const void* b_ff1;   /* [H, F],  [F]  */
+  const void* w_ff2; const void* b_ff2;   /* [F, H],  [H]  */
+  const void* ln2_g; const void* ln2_b;   /* [H], [H] */
+} enc_layer_weights;
+
+/* enc_create - build a handle on the current CUDA device.
+ * [FT] "什么是 Faster Transformer": head_num and size_per_head are the two
+ * structural parameters; ffn_dim and num_layers complete the stack.
+ *   head_num, ffn_dim, num_layers > 0; size_per_head in {32, 64, 128}
+ *   (else ENC_ERR_UNSUPPORTED); ffn_dim a multiple of 8.
+ *   weights: array of num_layers structs (see enc_layer_weights).
+ * The handle copies and repacks every parameter into its own device memory
+ * (FP16 weights are stored transposed, [out, in], for the tensor-core GEMMs;
+ * biases and LayerNorm parameters are widened to FP32), so the caller may free
+ * its buffers on return.  Synchronous.  On error *out is set to NULL. */
+ENC_API enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_layers,
+                      enc_dtype dtype, const enc_layer_weights* weights, enc_t* out);
+
+/* enc_forward - run the whole encoder stack on `stream`.
+ * [FT] "什么是 Faster Transformer" (batch size and sequence length per run)
+ * and "Faster Transformer 优化原理" (the fused per-layer kernels).
+ *   x:         device [batch, seq, H] in the handle's dtype, row-major.
+ *   valid_len: device int32 [batch]; values are clamped to [0, seq] on device.
+ *   out:       device [batch, seq, H]; must not overlap x.
+ *   1 <= batch <= 65535, seq >= 1.  x and out must be 16-byte aligned.
+ * The handle's workspace grows (cudaMalloc) when batch*seq exceeds what it
+ * holds; call enc_reserve first to keep allocation out of a timed or captured
+ * region.  No host synchronisation inside; errors in host checks are returned
+ * before anything is enqueued. */
+ENC_API enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* out,
+                       int batch, int seq, enc_stream_t stream);
+
+/* enc_forward_host - enc_forward on HOST buffers: copies x and valid_len to
+ * handle-owned device staging buffers, runs the stack and copies the result
+ * back into out, all on `stream`, then synchronises the stream.  Host buffers
+ * may be pageable or pinned (pinned gives asynchronous DMA).
+ *   x: host [batch, seq, H]; valid_len: host int32 [batch]; out: host [batch, seq, H]. */
+ENC_API enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, void* out,
+                            int batch, int seq, enc_stream_t stream);
+
+/* enc_reserve - grow the workspace to hold batch*seq tokens now (synchronous). */
+ENC_API enc_status enc_reserve(enc_t h, int batch, int seq);
+
+/* enc_workspace_bytes - device bytes enc_forward needs for a batch*seq-token run. */
+ENC_API size_t enc_workspace_bytes(enc_t h, int batch, int seq);
+
+/* enc_destroy - free every device buffer the handle owns (synchronises the device). NULL is a no-op. */
+ENC_API enc_status enc_destroy(enc_t h);
+
+/* enc_last_error - message for the last non-OK status on the calling thread ("" if none).
+ * The string is thread-local and valid until the next library call on this thread. */
+ENC_API const char* enc_last_error(void);
+
+/* enc_device_status - read and clear the handle's device status word (synchronises
+ * the device).  *code is 0 when no kernel has reported a failure since the last
+ * read; otherwise the code of the first failure (1 = a bounded wait inside a
+ * tensor-core GEMM gave up).  Returns ENC_ERR_DEVICE when *code != 0. */
+ENC_API enc_status enc_device_status(enc_t h, int32_t* code);
+
+/* enc_kernels_per_forward - kernel launches one enc_forward issues (7 per layer). */
+ENC_API int enc_kernels_per_forward(enc_t h);
+
+/* enc_launch_count - kernel launches this handle has issued since enc_create
+ * (forward passes and single steps), for checking what ran. */
+ENC_API uint64_t enc_launch_count(enc_t h);
+
+/* enc_set_trace_events - optional per-kernel timing of enc_forward.  events
+ * holds count CUDA events (cudaEvent_t, created by the caller); with count >=
+ * enc_kernels_per_forward(h) + 1, each enc_forward records events[k] on its
+ * stream just before its k-th kernel and events[kernels] after the last, so
+ * cudaEventElapsedTime(events[k], events[k+1]) is kernel k's duration.
+ * Kernel order per layer: QKV GEMM, attention, output GEMM, LayerNorm 1,
+ * FFN1 GEMM, FFN2 GEMM, LayerNorm 2.  events = NULL or count = 0 switches
+ * tracing off.  The handle keeps the pointers; the caller keeps the events
+ * alive while tracing is on. */
+ENC_API enc_status enc_set_trace_events(enc_t h, void* const* events, int count);
+
+/* ------------------------------------------------------------------------------
+ * Single steps of one layer, for checking each kernel alone.  Each runs exactly
+ * the kernel enc_forward runs for that step, with layer `layer`'s parameters,
+ * on caller-owned device buffers (same dtype as the handle, 16-byte aligned,
+ * non-overlapping).  M = batch * seq tokens.  Asynchronous on `stream`.
+ * ---------------------------------------------------------------------------- */
+
+/* Steps QKV projection + add-bias + head split ([FT] "Faster Transformer 优化原理":
+ * the Q/K/V matrix multiplies and the add-bias/transpose custom kernel, fused here
+ * into one GEMM epilogue):
+ *   qkv[t][b][h][s][c] = (x Wqkv + bqkv)[b*seq+s][t*H + h*d + c],
+ *   x: [M, H];  qkv: [3, batch, head_num, seq, d]. */
+ENC_API enc_status enc_op_qkv(enc_t h, int layer, const void* x, void* qkv, int batch, int seq,
+                      enc_stream_t stream);
+
+/* Steps scaled QK^T + padding mask, softmax, PV and head merge ([FT] "Faster
+ * Transformer 优化原理": the batched matrix multiplies around the SoftMax kernel
+ * and the transpose back to [tokens, hidden]), one fused kernel:
+ *   qkv: [3, batch, head_num, seq, d];  valid_len: device int32 [batch];
+ *   ctx: [M, H], ctx[b*seq+i][h*d + c]. */
+ENC_API enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, void* ctx,
+                            int batch, int seq, enc_stream_t stream);
+
+/* Step output projection without its bias (the bias is added by the next step):
+ *   a = ctx Wo,  ctx: [M, H], a: [M, H]. */
+ENC_API enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, void* a, int tokens,
+                           enc_stream_t stream);
+
+/* Step add-bias + residual + LayerNorm ([FT] "Faster Transformer 优化原理"):
+ *   which = 1: out = LN(resid + a + bo; ln1_g, ln1_b)
+ *   which = 2: out = LN(resid + a + b2; ln2_g, ln2_b)
+ *   a, resid, out: [tokens, H]. */
+ENC_API enc_status enc_op_bias_residual_layernorm(enc_t h, int layer, int which, const void* a,
+                                          const void* resid, void* out, int tokens,
+                                          enc_stream_t stream);
+
+/* Step FFN1 + add-bias + GELU (erf form) fused in the GEMM epilogue:
+ *   u = GELU(h1 W1 + b1),  h1: [tokens, H], u: [tokens, F]. */
+ENC_API enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens,
+                       enc_stream_t stream);
+
+/* Step FFN2 without its bias (added by the next step):  y = u W2,  u: [tokens, F], y: [tokens, H]. */
+ENC_API enc_status enc_op_ffn2(enc_t h, int layer, const void* u, void* y, int tokens,
+                       enc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BERT_ENCODER_B200_ENC_H */

@@ -1,0 +1,172 @@
+"""The whole encoder stack through the C ABI against the float64 oracle (GPU).
+
+Tolerances on valid tokens (query rows i < valid_len):
+  FP32 mode:                 relative L2 <= 1e-5 per layer
+  FP16 storage, FP32 accum.: relative L2 <= 5e-3 and max abs <= 3e-2 after one
+                             layer; relative L2 <= 2e-2 after 12 layers.
+The full-size workloads run in the same launch configuration the bench times;
+the oracle checks a seeded sample of their sequences (sequences never
+interact), always including the first, the last and a shortest one.
+"""
+import numpy as np
+import pytest
+
+import encoder_inputs as EI
+from oracle import encoder_oracle as O
+from parity_utils import (FP16_LAYER_MAX_ABS, FP16_LAYER_REL_L2, FP16_STACK_REL_L2, FP32_LAYER_REL_L2,
+                          encoder_from_inputs, max_abs, rel_l2, to_dev, to_host, valid_mask)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, enc=None):
+    enc = enc or encoder_from_inputs(inp)
+    out = enc.forward(to_dev(inp.x), to_dev(inp.valid_len))
+    return enc, to_host(out)
+
+
+def _oracle(inp, seqs=None):
+    x64, vl, layers = inp.as_float64()
+    sh = inp.workload.shape
+    return O.encoder_forward(x64, vl, layers, sh.head_num, sh.size_per_head, seqs=seqs)
+
+
+def _check(got, ref, vl, seq, rel_tol, abs_tol=None):
+    m = valid_mask(vl, seq)
+    r = rel_l2(got, ref, m)
+    assert r < rel_tol, f"relative L2 {r:.3e} >= {rel_tol:g}"
+    if abs_tol is not None:
+        a = max_abs(got, ref, m)
+        assert a < abs_tol, f"max abs {a:.3e} >= {abs_tol:g}"
+    return r
+
+
+def test_tiny_fp32_one_layer():
+    inp = EI.make_inputs(EI.named_workload("tiny-fp32", 1))
+    _, got = _run(inp)
+    _check(got, _oracle(inp), inp.valid_len, 32, FP32_LAYER_REL_L2)
+
+
+def test_fp32_two_layers_ragged():
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    inp = EI.make_inputs(EI.Workload("fp32-2L", sh, 3, 45, "fp32", 1, 45, ln_affine_random=True))
+    _, got = _run(inp)
+    _check(got, _oracle(inp), inp.valid_len, 45, 2 * FP32_LAYER_REL_L2)
+
+
+def test_bert_base_one_layer_fp16():
+    wl = EI.named_workload("bert-base-s32", 8)
+    inp = EI.make_inputs(wl.with_(shape=EI.EncoderShape(12, 64, 3072, 1)))
+    _, got = _run(inp)
+    _check(got, _oracle(inp), inp.valid_len, 32, FP16_LAYER_REL_L2, FP16_LAYER_MAX_ABS)
+
+
+def test_bert_base_twelve_layers_fp16():
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 8))
+    _, got = _run(inp)
+    _check(got, _oracle(inp), inp.valid_len, 32, FP16_STACK_REL_L2)
+
+
+@pytest.mark.parametrize("seq", [1, 7, 31, 32, 33, 96, 127, 128, 129, 512])
+@pytest.mark.parametrize("vl_kind", ["one", "full"])
+def test_edge_sequence_lengths_one_layer(seq, vl_kind):
+    sh = EI.EncoderShape(12, 64, 3072, 1)
+    batch = 3
+    lo = hi = 1 if vl_kind == "one" else seq
+    inp = EI.make_inputs(EI.Workload("edge", sh, batch, seq, "fp16", lo, hi, seed=seq))
+    _, got = _run(inp)
+    _check(got, _oracle(inp), inp.valid_len, seq, FP16_LAYER_REL_L2, FP16_LAYER_MAX_ABS)
+
+
+@pytest.mark.parametrize("nh,d,F", [(4, 32, 512), (12, 64, 3072), (16, 64, 4096), (8, 128, 2048), (2, 128, 256)])
+def test_head_structures_two_layers(nh, d, F):
+    sh = EI.EncoderShape(nh, d, F, 2)
+    inp = EI.make_inputs(EI.Workload("heads", sh, 5, 53, "fp16", 1, 53, seed=nh + d, ln_affine_random=True))
+    _, got = _run(inp)
+    _check(got, _oracle(inp), inp.valid_len, 53, 2 * FP16_LAYER_REL_L2)
+
+
+FULL_SIZE = [
+    ("bert-base-s32", 512, None, 4),
+    ("pruned-s32", 1024, None, 6),
+    ("bert-base", 256, 128, 3),
+    ("bert-base", 256, 96, 3),
+    ("bert-large", 256, 128, 3),
+    ("bert-large", 32, 512, 3),
+]
+
+
+@pytest.mark.parametrize("kind,batch,seq,nsample", FULL_SIZE, ids=lambda v: str(v))
+def test_full_size_workloads_sampled(kind, batch, seq, nsample):
+    wl = EI.named_workload(kind, batch, seq)
+    inp = EI.make_inputs(wl)
+    _, got = _run(inp)
+    assert np.all(np.isfinite(got[valid_mask(inp.valid_len, wl.seq)]))
+    seqs = EI.sample_sequences(wl.batch, nsample, inp.valid_len)
+    ref = _oracle(inp, seqs)
+    _check(got[seqs], ref, inp.valid_len[seqs], wl.seq, FP16_STACK_REL_L2)
+
+
+def test_padding_tokens_do_not_change_valid_outputs():
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    inp = EI.make_inputs(EI.Workload("pad", sh, 6, 70, "fp16", 5, 60, seed=4))
+    enc, got = _run(inp)
+    x2 = inp.x.copy()
+    rng = np.random.default_rng(0)
+    for b, n in enumerate(inp.valid_len):
+        x2[b, n:] = rng.normal(0, 3, x2[b, n:].shape).astype(np.float16)
+    got2 = to_host(enc.forward(to_dev(x2), to_dev(inp.valid_len)))
+    m = valid_mask(inp.valid_len, 70)
+    assert np.array_equal(got[m], got2[m])
+
+
+def test_permutation_equivariance_over_valid_tokens():
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    inp = EI.make_inputs(EI.Workload("perm", sh, 4, 48, "fp16", 20, 48, seed=9))
+    enc, got = _run(inp)
+    rng = np.random.default_rng(1)
+    x2 = inp.x.copy()
+    perms = []
+    for b, n in enumerate(inp.valid_len):
+        p = np.concatenate([rng.permutation(n), np.arange(n, 48)])
+        perms.append(p)
+        x2[b] = inp.x[b, p]
+    got2 = to_host(enc.forward(to_dev(x2), to_dev(inp.valid_len)))
+    for b, n in enumerate(inp.valid_len):
+        assert rel_l2(got2[b, :n], got[b, perms[b]][:n]) < 2 * FP16_LAYER_REL_L2
+
+
+def test_identical_tokens_give_identical_outputs():
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    inp = EI.make_inputs(EI.Workload("same", sh, 2, 33, "fp16", 33, 33, seed=2))
+    inp.x[:] = inp.x[:, :1]
+    _, got = _run(inp)
+    assert np.max(np.abs(got - got[:, :1])) < 1e-2
+
+
+def test_deterministic_and_host_entry_point_matches():
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 16))
+    enc, got = _run(inp)
+    again = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    assert np.array_equal(got, again)
+    host = enc.forward_host(inp.x, inp.valid_len)
+    assert np.array_equal(got, host)
+    assert enc.device_status() == 0
+
+
+def test_host_argument_checks():
+    import torch
+    from transformer_encoder_bert_b200 import EncError
+    inp = EI.make_inputs(EI.Workload("args", EI.EncoderShape(4, 32, 512, 1), 2, 8, "fp16", 1, 8))
+    enc = encoder_from_inputs(inp)
+    x = to_dev(inp.x)
+    vl = to_dev(inp.valid_len)
+    with pytest.raises(EncError) as e:
+        enc.forward(x, vl, out=x)                       # out overlaps x
+    assert e.value.status == 1
+    buf = torch.empty(x.numel() + 8, dtype=torch.float16, device="cuda")
+    with pytest.raises(EncError) as e:
+        enc.forward(x, vl, out=buf[1:1 + x.numel()].view_as(x))     # not 16-byte aligned
+    assert e.value.status == 1
+    with pytest.raises(EncError):
+        enc.op_ffn1(3, x, x, 16)                        # layer out of range

@@ -1,0 +1,172 @@
+"""Each kernel of the forward path alone against its oracle step (GPU).
+
+Inputs are seeded and in the storage dtype; the oracle step runs in float64
+on exactly those values.  Shapes span several GEMM tiles (128 rows) and
+ragged tails, every supported head size, and the structures of the
+workloads (4x32, 12x64, 16x64, 8x128).
+"""
+import numpy as np
+import pytest
+
+import encoder_inputs as EI
+from oracle import encoder_oracle as O
+from parity_utils import empty_dev, max_abs, rel_l2, to_dev, to_host, valid_mask
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(4, 32, 512), (12, 64, 3072), (16, 64, 4096), (8, 128, 2048)]
+BATCH_SEQ = [(1, 1), (3, 37), (2, 128), (5, 131)]
+
+# Single-GEMM outputs are the exact product rounded once to FP16 (half an ulp,
+# 2^-11 relative) plus FP32 accumulation error; attention also rounds P to FP16.
+GEMM_REL_L2 = 1e-3
+ATTN_REL_L2 = 2e-3
+LN_MAX_ABS = 4e-3            # |LN output| <= ~5, one FP16 ulp there is 2^-8
+FP32_REL_L2 = 1e-5
+
+
+def _setup(shape, batch, seq, dtype="fp16", seed=0):
+    nh, d, F = shape
+    sh = EI.EncoderShape(nh, d, F, 1)
+    wl = EI.Workload("ops", sh, batch, seq, dtype, 1, seq, seed=seed, ln_affine_random=True)
+    inp = EI.make_inputs(wl)
+    from parity_utils import encoder_from_inputs
+    enc = encoder_from_inputs(inp)
+    x64, vl, layers64 = inp.as_float64()
+    return wl, inp, enc, x64, vl, layers64[0]
+
+
+def _ulp_bound(ref):
+    return 2.0 ** -10 * max(1.0, float(np.max(np.abs(ref))))
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}_F{s[2]}")
+@pytest.mark.parametrize("batch,seq", BATCH_SEQ, ids=lambda v: str(v))
+def test_qkv_projection_and_head_split(shape, batch, seq):
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    nh, d = shape[0], shape[1]
+    H = nh * d
+    out = empty_dev((3, batch, nh, seq, d), "fp16")
+    enc.op_qkv(0, to_dev(inp.x), out, batch, seq)
+    got = to_host(out)
+    ref = O.head_split(O.qkv_projection(x64.reshape(-1, H), lw["w_qkv"], lw["b_qkv"]), batch, seq, nh, d)
+    assert rel_l2(got, ref) < GEMM_REL_L2
+    assert max_abs(got, ref) < _ulp_bound(ref)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}_F{s[2]}")
+@pytest.mark.parametrize("batch,seq", BATCH_SEQ + [(2, 512), (3, 200)], ids=lambda v: str(v))
+def test_attention(shape, batch, seq):
+    nh, d, _ = shape
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=7)
+    vlen = np.random.default_rng(3).integers(1, seq + 1, batch).astype(np.int32)
+    vlen[0] = seq
+    ctx = empty_dev((batch * seq, nh * d), "fp16")
+    enc.op_attention(to_dev(qkv), to_dev(vlen), ctx, batch, seq)
+    got = to_host(ctx).reshape(batch, seq, nh * d)
+    ref = O.attention(qkv.astype(np.float64), vlen)
+    assert rel_l2(got, ref) < ATTN_REL_L2
+    assert max_abs(got, ref) < 4 * _ulp_bound(ref)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}_F{s[2]}")
+@pytest.mark.parametrize("batch,seq", BATCH_SEQ, ids=lambda v: str(v))
+def test_out_proj_ffn1_ffn2(shape, batch, seq):
+    nh, d, F = shape
+    H = nh * d
+    M = batch * seq
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    ctx = EI.random_array((M, H), "fp16", seed=11)
+    a = empty_dev((M, H), "fp16")
+    enc.op_out_proj(0, to_dev(ctx), a, M)
+    ref = ctx.astype(np.float64) @ lw["w_o"]
+    got = to_host(a)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+
+    h1 = EI.random_array((M, H), "fp16", seed=12)
+    u = empty_dev((M, F), "fp16")
+    enc.op_ffn1(0, to_dev(h1), u, M)
+    ref = O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"])
+    got = to_host(u)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+
+    uu = EI.random_array((M, F), "fp16", seed=13, std=0.5)
+    y = empty_dev((M, H), "fp16")
+    enc.op_ffn2(0, to_dev(uu), y, M)
+    ref = uu.astype(np.float64) @ lw["w_ff2"]
+    got = to_host(y)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}_F{s[2]}")
+@pytest.mark.parametrize("which", [1, 2])
+def test_bias_residual_layernorm(shape, which):
+    nh, d, F = shape
+    H = nh * d
+    batch, seq = 5, 131
+    M = batch * seq
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    a = EI.random_array((M, H), "fp16", seed=21, std=0.7)
+    r = EI.random_array((M, H), "fp16", seed=22, mean=0.3)
+    out = empty_dev((M, H), "fp16")
+    enc.op_bias_residual_layernorm(0, which, to_dev(a), to_dev(r), out, M)
+    tag = "1" if which == 1 else "2"
+    bias = lw["b_o"] if which == 1 else lw["b_ff2"]
+    ref = O.bias_residual_layernorm(a.astype(np.float64), bias, r.astype(np.float64),
+                                    lw[f"ln{tag}_g"], lw[f"ln{tag}_b"])
+    got = to_host(out)
+    assert max_abs(got, ref) < LN_MAX_ABS
+    assert rel_l2(got, ref) < GEMM_REL_L2
+
+
+@pytest.mark.parametrize("shape", [(4, 32, 512), (12, 64, 3072)], ids=lambda s: f"{s[0]}x{s[1]}")
+def test_fp32_steps(shape):
+    nh, d, F = shape
+    H = nh * d
+    batch, seq = 3, 37
+    M = batch * seq
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq, dtype="fp32")
+    qkv = empty_dev((3, batch, nh, seq, d), "fp32")
+    enc.op_qkv(0, to_dev(inp.x), qkv, batch, seq)
+    ref_qkv = O.head_split(O.qkv_projection(x64.reshape(-1, H), lw["w_qkv"], lw["b_qkv"]), batch, seq, nh, d)
+    assert rel_l2(to_host(qkv), ref_qkv) < FP32_REL_L2
+    ctx = empty_dev((M, H), "fp32")
+    vlen = np.array([37, 1, 20], np.int32)
+    enc.op_attention(qkv, to_dev(vlen), ctx, batch, seq)
+    ref_ctx = O.attention(to_host(qkv).astype(np.float64), vlen).reshape(M, H)
+    assert rel_l2(to_host(ctx), ref_ctx) < FP32_REL_L2
+    h1 = EI.random_array((M, H), "fp32", seed=5)
+    u = empty_dev((M, F), "fp32")
+    enc.op_ffn1(0, to_dev(h1), u, M)
+    assert rel_l2(to_host(u), O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"])) < FP32_REL_L2
+    a = EI.random_array((M, H), "fp32", seed=6)
+    out = empty_dev((M, H), "fp32")
+    enc.op_bias_residual_layernorm(0, 1, to_dev(a), to_dev(h1), out, M)
+    ref = O.bias_residual_layernorm(a.astype(np.float64), lw["b_o"], h1.astype(np.float64), lw["ln1_g"], lw["ln1_b"])
+    assert rel_l2(to_host(out), ref) < FP32_REL_L2
+
+
+def test_attention_valid_len_clamping_and_empty():
+    shape = (12, 64, 3072)
+    nh, d, _ = shape
+    batch, seq = 4, 40
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=8)
+    vlen = np.array([seq + 7, 0, -3, 1], np.int32)      # clamp to [0, seq]
+    ctx = empty_dev((batch * seq, nh * d), "fp16")
+    enc.op_attention(to_dev(qkv), to_dev(vlen), ctx, batch, seq)
+    got = to_host(ctx).reshape(batch, seq, nh * d)
+    ref = O.attention(qkv.astype(np.float64), np.clip(vlen, 0, seq))
+    assert np.all(got[1] == 0) and np.all(got[2] == 0)   # n == 0: ctx = 0, no NaN
+    assert np.all(np.isfinite(got))
+    assert rel_l2(got, ref) < ATTN_REL_L2
+
+
+def test_gemm_bounded_waits_never_fired():
+    shape = (12, 64, 3072)
+    wl, inp, enc, x64, vl, lw = _setup(shape, 5, 131)
+    M = 5 * 131
+    y = empty_dev((M, 768), "fp16")
+    enc.op_ffn2(0, to_dev(EI.random_array((M, 3072), "fp16", seed=1)), y, M)
+    assert enc.device_status() == 0

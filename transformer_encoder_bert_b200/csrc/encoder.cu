@@ -1,0 +1,601 @@
+// C-ABI layer: handle, weight repacking, workspace, the per-layer step
+// sequence and the entry points declared in enc.h.
+//
+// Per layer, enc_forward launches (FP16 mode):
+//   1 tcgen05 GEMM  x Wqkv, epilogue + bqkv and Q/K/V head split
+//   2 attention     masked scaled softmax(QK^T) V, heads merged to [M, H]
+//   3 tcgen05 GEMM  ctx Wo
+//   4 LayerNorm     LN(x + a + bo)
+//   5 tcgen05 GEMM  h1 W1, epilogue + b1 and GELU
+//   6 tcgen05 GEMM  u W2
+//   7 LayerNorm     LN(h1 + y + b2)
+// i.e. 7 launches for the page's 14 ("Faster Transformer 优化原理": 8 cuBLAS
+// GEMMs + 6 custom kernels).  FP32 mode runs the same sequence with the
+// CUDA-core GEMM and attention kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <algorithm>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+enc_status fail(enc_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+enc_status ok() {
+  g_last_error.clear();
+  return ENC_OK;
+}
+
+enc_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(ENC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// [rows, cols] -> [cols, rows] for FP16 weights (tensor-core B operands are K-major).
+__global__ void transpose_f16_kernel(const __half* __restrict__ in, __half* __restrict__ out, int rows,
+                                     int cols) {
+  __shared__ __half tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < cols && r < rows) out[(size_t)c * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+template <typename T>
+__global__ void widen_to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = static_cast<float>(in[i]);
+}
+
+struct LayerDev {
+  void* w_qkv = nullptr;   // FP16: [3H, H]; FP32: [H, 3H]
+  void* w_o = nullptr;     // FP16: [H, H] transposed; FP32: [H, H]
+  void* w_ff1 = nullptr;   // FP16: [F, H]; FP32: [H, F]
+  void* w_ff2 = nullptr;   // FP16: [H, F]; FP32: [F, H]
+  float *b_qkv = nullptr, *b_o = nullptr, *b_ff1 = nullptr, *b_ff2 = nullptr;
+  float *ln1_g = nullptr, *ln1_b = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
+  CUtensorMap tm_qkv[2], tm_o[2], tm_ff1[2], tm_ff2[2];   // [0]: 128-row box, [1]: 256-row box
+};
+
+}  // namespace
+
+struct enc_handle {
+  int nh = 0, d = 0, H = 0, F = 0, L = 0;
+  enc_dtype dtype = ENC_FP16;
+  int device = 0;
+  int num_sms = 0;
+  size_t esize = 2;
+  std::vector<LayerDev> layers;
+  void* param_block = nullptr;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  void* stage = nullptr;            // enc_forward_host device staging
+  size_t stage_bytes = 0;
+  int* status = nullptr;
+  uint64_t launches = 0;            // kernels launched through this handle
+  std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
+};
+
+namespace {
+
+struct Workspace {
+  void *qkv, *ctx, *a, *h1, *u, *x0, *x1;
+};
+
+size_t workspace_bytes(const enc_handle* h, size_t tokens) {
+  const size_t es = h->esize;
+  const size_t mh = align_up(tokens * h->H * es, 256);
+  const size_t mf = align_up(tokens * h->F * es, 256);
+  return 3 * mh + mh + mh + mh + mf + 2 * mh;
+}
+
+Workspace carve(const enc_handle* h, size_t tokens) {
+  const size_t es = h->esize;
+  const size_t mh = align_up(tokens * h->H * es, 256);
+  const size_t mf = align_up(tokens * h->F * es, 256);
+  char* p = static_cast<char*>(h->ws);
+  Workspace w;
+  w.qkv = p; p += 3 * mh;
+  w.ctx = p; p += mh;
+  w.a = p; p += mh;
+  w.h1 = p; p += mh;
+  w.u = p; p += mf;
+  w.x0 = p; p += mh;
+  w.x1 = p;
+  return w;
+}
+
+enc_status ensure_workspace(enc_handle* h, size_t tokens) {
+  const size_t need = workspace_bytes(h, tokens);
+  if (need <= h->ws_bytes) return ENC_OK;
+  if (h->ws) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize before workspace growth");
+    cudaFree(h->ws);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+  }
+  void* p = nullptr;
+  if (cudaMalloc(&p, need) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ENC_ERR_OOM, "workspace allocation of %zu bytes failed", need);
+  }
+  h->ws = p;
+  h->ws_bytes = need;
+  return ENC_OK;
+}
+
+enc_status check_handle(const enc_handle* h) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device)
+    return fail(ENC_ERR_INVALID_ARG, "current device %d is not the handle's device %d", dev, h->device);
+  return ENC_OK;
+}
+
+int choose_bn(const enc_handle* h, int M, int N) {
+  if (N % 256 != 0) return 128;
+  const long tiles256 = (long)((M + 127) / 128) * (N / 256);
+  return tiles256 >= h->num_sms ? 256 : 128;
+}
+
+// One GEMM step: C = A * W (+ epilogue), dispatched on the handle's dtype.
+enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const CUtensorMap* wmaps, int N,
+                    enc::Epi epi, const float* bias, void* C, enc::SplitShape sp, cudaStream_t st) {
+  if (h->dtype == ENC_FP16) {
+    const int bn = choose_bn(h, M, N);
+    CUtensorMap ta;
+    if (!enc::encode_kmajor_fp16_map(&ta, A, (uint64_t)M, (uint64_t)K, 128))
+      return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation operand [%d, %d]", M, K);
+    enc::TcGemmArgs a;
+    a.tmap_a = &ta;
+    a.tmap_b = &wmaps[bn == 256 ? 1 : 0];
+    a.M = M; a.N = N; a.K = K; a.bn = bn; a.epi = epi; a.bias = bias;
+    a.c = static_cast<__half*>(C);
+    a.split = sp;
+    a.status = h->status;
+    a.num_sms = h->num_sms;
+    cudaError_t e = enc::launch_gemm_tc(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
+    ++h->launches;
+  } else {
+    cudaError_t e = enc::launch_gemm_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K,
+                                         epi, bias, static_cast<float*>(C), sp, st);
+    if (e != cudaSuccess) return cuda_fail(e, "FP32 GEMM launch");
+    ++h->launches;
+  }
+  return ENC_OK;
+}
+
+enc_status step_qkv(enc_handle* h, int l, const void* x, void* qkv, int batch, int seq, cudaStream_t st) {
+  LayerDev& L = h->layers[l];
+  enc::SplitShape sp{batch, seq, h->nh, h->d};
+  return run_gemm(h, x, batch * seq, h->H, L.w_qkv, L.tm_qkv, 3 * h->H, enc::Epi::kBiasQkvSplit, L.b_qkv, qkv,
+                  sp, st);
+}
+
+enc_status step_attention(enc_handle* h, const void* qkv, const int32_t* vl, void* ctx, int batch, int seq,
+                          cudaStream_t st) {
+  cudaError_t e;
+  if (h->dtype == ENC_FP16)
+    e = enc::launch_attention_f16(static_cast<const __half*>(qkv), vl, static_cast<__half*>(ctx), batch, seq,
+                                  h->nh, h->d, st);
+  else
+    e = enc::launch_attention_f32(static_cast<const float*>(qkv), vl, static_cast<float*>(ctx), batch, seq,
+                                  h->nh, h->d, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  ++h->launches;
+  return ENC_OK;
+}
+
+enc_status step_out_proj(enc_handle* h, int l, const void* ctx, void* a, int tokens, cudaStream_t st) {
+  LayerDev& L = h->layers[l];
+  return run_gemm(h, ctx, tokens, h->H, L.w_o, L.tm_o, h->H, enc::Epi::kStore, nullptr, a, {}, st);
+}
+
+enc_status step_ln(enc_handle* h, int l, int which, const void* a, const void* resid, void* out, int tokens,
+                   cudaStream_t st) {
+  LayerDev& L = h->layers[l];
+  const float* bias = which == 1 ? L.b_o : L.b_ff2;
+  const float* g = which == 1 ? L.ln1_g : L.ln2_g;
+  const float* b = which == 1 ? L.ln1_b : L.ln2_b;
+  cudaError_t e;
+  if (h->dtype == ENC_FP16)
+    e = enc::launch_bias_residual_ln_f16(static_cast<const __half*>(a), bias, static_cast<const __half*>(resid),
+                                         g, b, static_cast<__half*>(out), tokens, h->H, st);
+  else
+    e = enc::launch_bias_residual_ln_f32(static_cast<const float*>(a), bias, static_cast<const float*>(resid), g,
+                                         b, static_cast<float*>(out), tokens, h->H, st);
+  if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
+  ++h->launches;
+  return ENC_OK;
+}
+
+enc_status step_ffn1(enc_handle* h, int l, const void* h1, void* u, int tokens, cudaStream_t st) {
+  LayerDev& L = h->layers[l];
+  return run_gemm(h, h1, tokens, h->H, L.w_ff1, L.tm_ff1, h->F, enc::Epi::kBiasGelu, L.b_ff1, u, {}, st);
+}
+
+enc_status step_ffn2(enc_handle* h, int l, const void* u, void* y, int tokens, cudaStream_t st) {
+  LayerDev& L = h->layers[l];
+  return run_gemm(h, u, tokens, h->F, L.w_ff2, L.tm_ff2, h->H, enc::Epi::kStore, nullptr, y, {}, st);
+}
+
+enc_status check_tokens(int batch, int seq) {
+  if (batch <= 0 || seq <= 0) return fail(ENC_ERR_INVALID_ARG, "batch (%d) and seq (%d) must be >= 1", batch, seq);
+  if (batch > 65535) return fail(ENC_ERR_UNSUPPORTED, "batch %d exceeds 65535", batch);
+  if ((long long)batch * seq > (1LL << 30)) return fail(ENC_ERR_UNSUPPORTED, "batch*seq too large");
+  return ENC_OK;
+}
+
+enc_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return fail(ENC_ERR_INVALID_ARG, "null buffer pointer");
+    if (!aligned16(p)) return fail(ENC_ERR_INVALID_ARG, "buffer %p is not 16-byte aligned", p);
+  }
+  return ENC_OK;
+}
+
+void free_handle(enc_handle* h) {
+  if (!h) return;
+  if (h->param_block) cudaFree(h->param_block);
+  if (h->ws) cudaFree(h->ws);
+  if (h->stage) cudaFree(h->stage);
+  if (h->status) cudaFree(h->status);
+  delete h;
+}
+
+}  // namespace
+
+int enc::device_sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+extern "C" {
+
+const char* enc_last_error(void) { return g_last_error.c_str(); }
+
+enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_layers, enc_dtype dtype,
+                      const enc_layer_weights* weights, enc_t* out) {
+  if (!out) return fail(ENC_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  if (head_num <= 0 || size_per_head <= 0 || ffn_dim <= 0 || num_layers <= 0)
+    return fail(ENC_ERR_INVALID_ARG, "head_num, size_per_head, ffn_dim and num_layers must be > 0");
+  if (size_per_head != 32 && size_per_head != 64 && size_per_head != 128)
+    return fail(ENC_ERR_UNSUPPORTED, "size_per_head %d not in {32, 64, 128}", size_per_head);
+  if (dtype != ENC_FP16 && dtype != ENC_FP32) return fail(ENC_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (ffn_dim % 8 != 0) return fail(ENC_ERR_INVALID_ARG, "ffn_dim %d is not a multiple of 8", ffn_dim);
+  const int H = head_num * size_per_head;
+  const int max_h = dtype == ENC_FP16 ? 4096 : 2048;
+  if (H > max_h) return fail(ENC_ERR_UNSUPPORTED, "hidden size %d exceeds %d", H, max_h);
+  if (!weights) return fail(ENC_ERR_INVALID_ARG, "weights is null");
+  for (int l = 0; l < num_layers; ++l) {
+    const enc_layer_weights& w = weights[l];
+    const void* ps[] = {w.w_qkv, w.b_qkv, w.w_o, w.b_o, w.ln1_g, w.ln1_b,
+                        w.w_ff1, w.b_ff1, w.w_ff2, w.b_ff2, w.ln2_g, w.ln2_b};
+    for (const void* p : ps)
+      if (!p) return fail(ENC_ERR_INVALID_ARG, "layer %d has a null parameter pointer", l);
+  }
+
+  enc_handle* h = new enc_handle();
+  h->nh = head_num; h->d = size_per_head; h->H = H; h->F = ffn_dim; h->L = num_layers;
+  h->dtype = dtype;
+  h->esize = dtype == ENC_FP16 ? 2 : 4;
+  cudaGetDevice(&h->device);
+  h->num_sms = enc::device_sm_count();
+  if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
+  if (dtype == ENC_FP16) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, h->device) != cudaSuccess || prop.major != 10) {
+      free_handle(h);
+      return fail(ENC_ERR_UNSUPPORTED, "FP16 mode needs an sm_100 (B200-class) device");
+    }
+  }
+  if (cudaMalloc(&h->status, sizeof(int)) != cudaSuccess || cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    free_handle(h);
+    return fail(ENC_ERR_OOM, "status word allocation failed");
+  }
+
+  const size_t es = h->esize;
+  const size_t F = ffn_dim;
+  const size_t wsz[4] = {(size_t)H * 3 * H, (size_t)H * H, (size_t)H * F, F * H};
+  const size_t vsz[8] = {3 * (size_t)H, (size_t)H, F, (size_t)H, (size_t)H, (size_t)H, (size_t)H, (size_t)H};
+  size_t per_layer = 0;
+  for (size_t s : wsz) per_layer += align_up(s * es, 256);
+  for (size_t s : vsz) per_layer += align_up(s * 4, 256);
+  size_t staging = 0;
+  for (size_t s : wsz) staging = std::max(staging, align_up(s * es, 256));
+  if (cudaMalloc(&h->param_block, per_layer * num_layers + staging) != cudaSuccess) {
+    cudaGetLastError();
+    free_handle(h);
+    return fail(ENC_ERR_OOM, "parameter allocation of %zu bytes failed", per_layer * num_layers + staging);
+  }
+  char* p = static_cast<char*>(h->param_block);
+  char* stage = p + per_layer * num_layers;
+  h->layers.resize(num_layers);
+  cudaStream_t st = nullptr;
+  for (int l = 0; l < num_layers; ++l) {
+    const enc_layer_weights& w = weights[l];
+    LayerDev& L = h->layers[l];
+    const void* wsrc[4] = {w.w_qkv, w.w_o, w.w_ff1, w.w_ff2};
+    void** wdst[4] = {&L.w_qkv, &L.w_o, &L.w_ff1, &L.w_ff2};
+    const int rows[4] = {H, H, H, ffn_dim};           // "in" dimension of each [in, out] matrix
+    const int cols[4] = {3 * H, H, ffn_dim, H};
+    for (int i = 0; i < 4; ++i) {
+      *wdst[i] = p;
+      const size_t bytes = wsz[i] * es;
+      if (dtype == ENC_FP16) {
+        cudaError_t e = cudaMemcpy(stage, wsrc[i], bytes, cudaMemcpyDefault);
+        if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "weight upload"); }
+        const dim3 grid((cols[i] + 31) / 32, (rows[i] + 31) / 32);
+        transpose_f16_kernel<<<grid, dim3(32, 8), 0, st>>>(reinterpret_cast<const __half*>(stage),
+                                                          reinterpret_cast<__half*>(p), rows[i], cols[i]);
+        e = cudaDeviceSynchronize();
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "weight repack"); }
+      } else {
+        cudaError_t e = cudaMemcpy(p, wsrc[i], bytes, cudaMemcpyDefault);
+        if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "weight upload"); }
+      }
+      p += align_up(bytes, 256);
+    }
+    const void* vsrc[8] = {w.b_qkv, w.b_o, w.b_ff1, w.b_ff2, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b};
+    float** vdst[8] = {&L.b_qkv, &L.b_o, &L.b_ff1, &L.b_ff2, &L.ln1_g, &L.ln1_b, &L.ln2_g, &L.ln2_b};
+    for (int i = 0; i < 8; ++i) {
+      *vdst[i] = reinterpret_cast<float*>(p);
+      const size_t n = vsz[i];
+      cudaError_t e = cudaMemcpy(stage, vsrc[i], n * es, cudaMemcpyDefault);
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "parameter upload"); }
+      if (dtype == ENC_FP16)
+        widen_to_f32_kernel<__half><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            reinterpret_cast<const __half*>(stage), *vdst[i], (int)n);
+      else
+        widen_to_f32_kernel<float><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            reinterpret_cast<const float*>(stage), *vdst[i], (int)n);
+      e = cudaDeviceSynchronize();
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "parameter widen"); }
+      p += align_up(n * 4, 256);
+    }
+    if (dtype == ENC_FP16) {
+      // B operands [N, K]: Wqkv^T [3H, H], Wo^T [H, H], W1^T [F, H], W2^T [H, F].
+      struct { CUtensorMap* m; void* w; int n, k; } maps[4] = {
+          {L.tm_qkv, L.w_qkv, 3 * H, H}, {L.tm_o, L.w_o, H, H}, {L.tm_ff1, L.w_ff1, ffn_dim, H},
+          {L.tm_ff2, L.w_ff2, H, ffn_dim}};
+      for (auto& m : maps) {
+        if (!enc::encode_kmajor_fp16_map(&m.m[0], m.w, m.n, m.k, 128) ||
+            !enc::encode_kmajor_fp16_map(&m.m[1], m.w, m.n, m.k, 256)) {
+          free_handle(h);
+          return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight operand");
+        }
+      }
+    }
+  }
+  *out = h;
+  return ok();
+}
+
+size_t enc_workspace_bytes(enc_t h, int batch, int seq) {
+  if (!h || batch <= 0 || seq <= 0) return 0;
+  return workspace_bytes(h, (size_t)batch * seq);
+}
+
+enc_status enc_reserve(enc_t h, int batch, int seq) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if ((s = ensure_workspace(h, (size_t)batch * seq)) != ENC_OK) return s;
+  return ok();
+}
+
+enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                       enc_stream_t stream) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if ((s = check_ptrs({x, out})) != ENC_OK) return s;
+  if (!valid_len) return fail(ENC_ERR_INVALID_ARG, "valid_len is null");
+  const size_t M = (size_t)batch * seq;
+  const size_t bytes = M * h->H * h->esize;
+  const char* xb = static_cast<const char*>(x);
+  const char* ob = static_cast<const char*>(out);
+  if (xb < ob + bytes && ob < xb + bytes) return fail(ENC_ERR_INVALID_ARG, "out overlaps x");
+  if ((s = ensure_workspace(h, M)) != ENC_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Workspace w = carve(h, M);
+  const int tokens = (int)M;
+  const bool tracing = !h->trace.empty();
+  int k = 0;
+  auto mark = [&]() {
+    if (tracing) cudaEventRecord(h->trace[k++], st);
+  };
+  for (int l = 0; l < h->L; ++l) {
+    const void* xin = l == 0 ? x : (((l - 1) & 1) ? w.x1 : w.x0);
+    void* xout = l == h->L - 1 ? out : ((l & 1) ? w.x1 : w.x0);
+    mark();
+    if ((s = step_qkv(h, l, xin, w.qkv, batch, seq, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_attention(h, w.qkv, valid_len, w.ctx, batch, seq, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_out_proj(h, l, w.ctx, w.a, tokens, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_ln(h, l, 1, w.a, xin, w.h1, tokens, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_ffn1(h, l, w.h1, w.u, tokens, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_ffn2(h, l, w.u, w.a, tokens, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_ln(h, l, 2, w.a, w.h1, xout, tokens, st)) != ENC_OK) return s;
+  }
+  mark();
+  return ok();
+}
+
+enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                            enc_stream_t stream) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if (!x || !valid_len || !out) return fail(ENC_ERR_INVALID_ARG, "null host buffer");
+  const size_t act = (size_t)batch * seq * h->H * h->esize;
+  const size_t act_al = align_up(act, 256);
+  const size_t need = 2 * act_al + align_up((size_t)batch * 4, 256);
+  if (need > h->stage_bytes) {
+    if (h->stage) {
+      cudaDeviceSynchronize();
+      cudaFree(h->stage);
+      h->stage = nullptr;
+      h->stage_bytes = 0;
+    }
+    if (cudaMalloc(&h->stage, need) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ENC_ERR_OOM, "staging allocation of %zu bytes failed", need);
+    }
+    h->stage_bytes = need;
+  }
+  char* base = static_cast<char*>(h->stage);
+  void* dx = base;
+  void* dout = base + act_al;
+  int32_t* dvl = reinterpret_cast<int32_t*>(base + 2 * act_al);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(dx, x, act, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dvl, valid_len, (size_t)batch * 4, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  if ((s = enc_forward(h, dx, dvl, dout, batch, seq, stream)) != ENC_OK) return s;
+  e = cudaMemcpyAsync(out, dout, act, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return ok();
+}
+
+enc_status enc_destroy(enc_t h) {
+  if (!h) return ok();
+  cudaDeviceSynchronize();
+  free_handle(h);
+  return ok();
+}
+
+enc_status enc_device_status(enc_t h, int32_t* code) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if (!code) return fail(ENC_ERR_INVALID_ARG, "code is null");
+  int v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  *code = v;
+  if (v != 0) return fail(ENC_ERR_DEVICE, "a kernel reported device status %d", v);
+  return ok();
+}
+
+int enc_kernels_per_forward(enc_t h) { return h ? 7 * h->L : 0; }
+
+uint64_t enc_launch_count(enc_t h) { return h ? h->launches : 0; }
+
+enc_status enc_set_trace_events(enc_t h, void* const* events, int count) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  if (!events || count == 0) {
+    h->trace.clear();
+    return ok();
+  }
+  if (count < 7 * h->L + 1)
+    return fail(ENC_ERR_INVALID_ARG, "need %d trace events, got %d", 7 * h->L + 1, count);
+  h->trace.assign(reinterpret_cast<cudaEvent_t const*>(events), reinterpret_cast<cudaEvent_t const*>(events) + count);
+  return ok();
+}
+
+// ---------------------------------------------------------------- single steps
+
+static enc_status op_prologue(enc_t h, int layer, bool needs_layer, int tokens) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if (needs_layer && (layer < 0 || layer >= h->L)) return fail(ENC_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (tokens <= 0) return fail(ENC_ERR_INVALID_ARG, "token count must be >= 1");
+  return ENC_OK;
+}
+
+enc_status enc_op_qkv(enc_t h, int layer, const void* x, void* qkv, int batch, int seq, enc_stream_t stream) {
+  enc_status s = op_prologue(h, layer, true, batch > 0 && seq > 0 ? batch * seq : 0);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if ((s = check_ptrs({x, qkv})) != ENC_OK) return s;
+  if ((s = step_qkv(h, layer, x, qkv, batch, seq, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  return ok();
+}
+
+enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, void* ctx, int batch, int seq,
+                            enc_stream_t stream) {
+  enc_status s = op_prologue(h, 0, false, batch > 0 && seq > 0 ? batch * seq : 0);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if ((s = check_ptrs({qkv, ctx})) != ENC_OK) return s;
+  if (!valid_len) return fail(ENC_ERR_INVALID_ARG, "valid_len is null");
+  if ((s = step_attention(h, qkv, valid_len, ctx, batch, seq, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK)
+    return s;
+  return ok();
+}
+
+enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, void* a, int tokens, enc_stream_t stream) {
+  enc_status s = op_prologue(h, layer, true, tokens);
+  if (s != ENC_OK) return s;
+  if ((s = check_ptrs({ctx, a})) != ENC_OK) return s;
+  if ((s = step_out_proj(h, layer, ctx, a, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  return ok();
+}
+
+enc_status enc_op_bias_residual_layernorm(enc_t h, int layer, int which, const void* a, const void* resid,
+                                          void* out, int tokens, enc_stream_t stream) {
+  enc_status s = op_prologue(h, layer, true, tokens);
+  if (s != ENC_OK) return s;
+  if (which != 1 && which != 2) return fail(ENC_ERR_INVALID_ARG, "which must be 1 or 2");
+  if ((s = check_ptrs({a, resid, out})) != ENC_OK) return s;
+  if ((s = step_ln(h, layer, which, a, resid, out, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK)
+    return s;
+  return ok();
+}
+
+enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens, enc_stream_t stream) {
+  enc_status s = op_prologue(h, layer, true, tokens);
+  if (s != ENC_OK) return s;
+  if ((s = check_ptrs({h1, u})) != ENC_OK) return s;
+  if ((s = step_ffn1(h, layer, h1, u, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  return ok();
+}
+
+enc_status enc_op_ffn2(enc_t h, int layer, const void* u, void* y, int tokens, enc_stream_t stream) {
+  enc_status s = op_prologue(h, layer, true, tokens);
+  if (s != ENC_OK) return s;
+  if ((s = check_ptrs({u, y})) != ENC_OK) return s;
+  if ((s = step_ffn2(h, layer, u, y, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,74 @@
+// Internal declarations shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "enc.h"
+
+namespace enc {
+
+constexpr float kLnEps = 1e-12f;   // LayerNorm epsilon (the original BERT value; the source page gives none)
+
+// What a GEMM does with its FP32 accumulator tile before storing it.
+enum class Epi : int {
+  kStore = 0,        // C[m][n] = acc
+  kBiasGelu = 1,     // C[m][n] = GELU(acc + bias[n]), erf form
+  kBiasQkvSplit = 2  // Q/K/V head split: dst[t][b][h][s][c] = acc + bias[n]
+};
+
+// Addressing for the head-split epilogue (n = t*H + h*d + c, m = b*seq + s).
+struct SplitShape {
+  int batch, seq, head_num, size_per_head;
+};
+
+// Device status codes written by kernels (first failure wins).
+constexpr int kStatusWaitTimeout = 1;
+
+// ---- FP16 tensor-core GEMM (tcgen05 + TMEM + TMA), gemm_tc.cu ----
+// C = A[M,K] * B[N,K]^T; A and B are K-major FP16 in global memory.
+struct TcGemmArgs {
+  const CUtensorMap* tmap_a;   // dims {K, M}, box {64, 128}, 128B swizzle
+  const CUtensorMap* tmap_b;   // dims {K, N}, box {64, bn}, 128B swizzle
+  int M, N, K;
+  int bn;                      // 128 or 256
+  Epi epi;
+  const float* bias;           // [N] (kBiasGelu, kBiasQkvSplit)
+  __half* c;                   // [M, N] or the split destination
+  SplitShape split;
+  int* status;                 // device status word
+  int num_sms;
+};
+cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream);
+
+// Encode a 2-D K-major FP16 tensor map over [rows, cols=K] with a {64, box_rows} box.
+bool encode_kmajor_fp16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_rows);
+
+// ---- FP32 SIMT GEMM (FP32 mode, no TF32), gemm_f32.cu ----
+// C = A[M,K] * W[K,N] (W row-major [K,N]).
+cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K, Epi epi,
+                            const float* bias, float* C, SplitShape split, cudaStream_t stream);
+
+// ---- attention, attention.cu ----
+cudaError_t launch_attention_f16(const __half* qkv, const int32_t* valid_len, __half* ctx,
+                                 int batch, int seq, int head_num, int size_per_head,
+                                 cudaStream_t stream);
+cudaError_t launch_attention_f32(const float* qkv, const int32_t* valid_len, float* ctx,
+                                 int batch, int seq, int head_num, int size_per_head,
+                                 cudaStream_t stream);
+
+// ---- add-bias + residual + LayerNorm, layernorm.cu ----
+cudaError_t launch_bias_residual_ln_f16(const __half* a, const float* bias, const __half* resid,
+                                        const float* gamma, const float* beta, __half* out,
+                                        int rows, int hidden, cudaStream_t stream);
+cudaError_t launch_bias_residual_ln_f32(const float* a, const float* bias, const float* resid,
+                                        const float* gamma, const float* beta, float* out,
+                                        int rows, int hidden, cudaStream_t stream);
+
+// ---- weight repack, encoder.cu ----
+int device_sm_count();
+
+}  // namespace enc
