@@ -170,3 +170,45 @@ def test_gemm_bounded_waits_never_fired():
     y = empty_dev((M, 768), "fp16")
     enc.op_ffn2(0, to_dev(EI.random_array((M, 3072), "fp16", seed=1)), y, M)
     assert enc.device_status() == 0
+
+
+@pytest.mark.parametrize("hidden,batch,seq", [(128, 3, 37), (256, 4, 96)], ids=["one-cta", "cta-pair"])
+def test_gelu_epilogue_against_exact_erf(hidden, batch, seq):
+    """W1 = I, b1 = 0 turns FFN1 into GELU of its FP16 input; inputs span [-8, 8].
+    The result must be the exact erf-GELU rounded once to FP16."""
+    from transformer_encoder_bert_b200 import Encoder
+    nh, d = hidden // 32, 32
+    M = batch * seq
+    lw = {k: v for k, v in _setup((nh, d, hidden), 1, 8)[1].layers[0].items()}
+    lw["w_ff1"] = np.eye(hidden, dtype=np.float16)
+    lw["b_ff1"] = np.zeros(hidden, np.float16)
+    enc = Encoder(nh, d, hidden, [lw], "fp16")
+    h1 = np.linspace(-8, 8, M * hidden).astype(np.float16).reshape(M, hidden)
+    u = empty_dev((M, hidden), "fp16")
+    enc.op_ffn1(0, to_dev(h1), u, M)
+    got = to_host(u).astype(np.float64)
+    ref = O.gelu_erf(h1.astype(np.float64))
+    # one FP16 rounding of the exact value: |got - ref| <= half an ulp of |ref| (+ tiny slack)
+    ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 0.5 * ulp + 1e-6)
+
+
+@pytest.mark.parametrize("batch,seq", [(2, 128), (5, 131)], ids=str)
+def test_one_cta_tiles_when_pairs_disabled(monkeypatch, batch, seq):
+    """The one-CTA 128x256 tile path (used for small M) on shapes that normally take the pair path."""
+    monkeypatch.setenv("ENC_GEMM_NO_PAIR", "1")
+    shape = (12, 64, 3072)
+    nh, d, F = shape
+    H = nh * d
+    M = batch * seq
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    h1 = EI.random_array((M, H), "fp16", seed=12)
+    u = empty_dev((M, F), "fp16")
+    enc.op_ffn1(0, to_dev(h1), u, M)
+    ref = O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"])
+    got = to_host(u)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+    out = empty_dev((3, batch, nh, seq, d), "fp16")
+    enc.op_qkv(0, to_dev(inp.x), out, batch, seq)
+    ref = O.head_split(O.qkv_projection(x64.reshape(-1, H), lw["w_qkv"], lw["b_qkv"]), batch, seq, nh, d)
+    assert rel_l2(to_host(out), ref) < GEMM_REL_L2

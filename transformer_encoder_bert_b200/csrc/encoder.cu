@@ -15,6 +15,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -96,6 +97,7 @@ struct enc_handle {
   size_t stage_bytes = 0;
   int* status = nullptr;
   uint64_t launches = 0;            // kernels launched through this handle
+  bool no_pair = false;             // ENC_GEMM_NO_PAIR=1: one-CTA tiles only (comparison runs)
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -156,7 +158,10 @@ enc_status check_handle(const enc_handle* h) {
   return ENC_OK;
 }
 
+// Tile choice: a 2-CTA 256x256 tile when N is a multiple of 256 and there are
+// enough rows to fill the 256-row tile; otherwise one CTA per 128 x {256,128}.
 int choose_bn(const enc_handle* h, int M, int N) {
+  if (N % 256 == 0 && M >= 256 && !h->no_pair) return enc::kPairTile;
   if (N % 256 != 0) return 128;
   const long tiles256 = (long)((M + 127) / 128) * (N / 256);
   return tiles256 >= h->num_sms ? 256 : 128;
@@ -172,7 +177,7 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
       return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation operand [%d, %d]", M, K);
     enc::TcGemmArgs a;
     a.tmap_a = &ta;
-    a.tmap_b = &wmaps[bn == 256 ? 1 : 0];
+    a.tmap_b = &wmaps[bn == 256 ? 1 : 0];      // the pair tile loads 128-row halves of B
     a.M = M; a.N = N; a.K = K; a.bn = bn; a.epi = epi; a.bias = bias;
     a.c = static_cast<__half*>(C);
     a.split = sp;
@@ -309,6 +314,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   h->esize = dtype == ENC_FP16 ? 2 : 4;
   cudaGetDevice(&h->device);
   h->num_sms = enc::device_sm_count();
+  if (const char* e = getenv("ENC_GEMM_NO_PAIR")) h->no_pair = e[0] == '1';
   if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
   if (dtype == ENC_FP16) {
     cudaDeviceProp prop;

@@ -28,12 +28,15 @@ struct SplitShape {
 constexpr int kStatusWaitTimeout = 1;
 
 // ---- FP16 tensor-core GEMM (tcgen05 + TMEM + TMA), gemm_tc.cu ----
+// TcGemmArgs::bn selects the tile: 128 or 256 (one CTA, 128 x bn), or kPairTile
+// (a 2-CTA cluster per 256 x 256 tile; B map box of 128 rows; N % 256 == 0).
+constexpr int kPairTile = 2;
 // C = A[M,K] * B[N,K]^T; A and B are K-major FP16 in global memory.
 struct TcGemmArgs {
   const CUtensorMap* tmap_a;   // dims {K, M}, box {64, 128}, 128B swizzle
-  const CUtensorMap* tmap_b;   // dims {K, N}, box {64, bn}, 128B swizzle
+  const CUtensorMap* tmap_b;   // dims {K, N}, box {64, bn} (128 rows for kPairTile), 128B swizzle
   int M, N, K;
-  int bn;                      // 128 or 256
+  int bn;                      // 128, 256 or kPairTile
   Epi epi;
   const float* bias;           // [N] (kBiasGelu, kBiasQkvSplit)
   __half* c;                   // [M, N] or the split destination
