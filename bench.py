@@ -2,7 +2,7 @@
 """Throughput of the BERT-style encoder forward on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload KIND:BATCH[:SEQ]] [--no-cpu-baseline]
+                    [--workload KIND:BATCH[:SEQ]] [--graph] [--no-cpu-baseline]
 
 A step is one enc_forward over one batch of the workload (every layer, every
 kernel of the path), inputs already in HBM; the L2 is flushed (256 MiB write)
@@ -215,8 +215,10 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         if world > 1:
             dist.barrier()
 
+    graph = enc.record(x, vl, out) if args.graph else None
+    step = (lambda: graph.launch()) if graph is not None else (lambda: enc.forward(x, vl, out))
     for _ in range(args.warmup):
-        enc.forward(x, vl, out)
+        step()
     torch.cuda.synchronize()
 
     nk = enc.kernels_per_forward()
@@ -235,14 +237,23 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     launches0 = enc.launch_count()
     for i in range(args.steps):
         flush.zero_()
-        enc.set_trace_events(ev_sets[i], prepare=False)
+        if graph is None:
+            enc.set_trace_events(ev_sets[i], prepare=False)
         starts[i].record(stream)
-        enc.forward(x, vl, out)
+        step()
         ends[i].record(stream)
     torch.cuda.synchronize()
     barrier()
     launches = enc.launch_count() - launches0
     clk = clocks.stop()
+    if graph is not None:
+        # A recorded forward carries no per-kernel events: take the breakdown from
+        # the same number of traced (non-recorded) forwards after the timed region.
+        for i in range(args.steps):
+            flush.zero_()
+            enc.set_trace_events(ev_sets[i], prepare=False)
+            enc.forward(x, vl, out)
+        torch.cuda.synchronize()
     enc.set_trace_events(None)
 
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
@@ -271,6 +282,8 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     barrier()
     e2e_step = sum(e2e_ms) / len(e2e_ms)
     status = enc.device_status()
+    if graph is not None:
+        graph.close()
 
     if world > 1:
         t = torch.tensor([ms, e2e_step], dtype=torch.float64, device=dev)
@@ -311,7 +324,8 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16" if wl.dtype == "fp16" else "fp32", "data": "synthetic",
-        "config": workload_config(wl, world, l2="flushed before every timed step (256 MiB write)"),
+        "config": dict(workload_config(wl, world, l2="flushed before every timed step (256 MiB write)"),
+                       launch="one recorded CUDA graph per step" if args.graph else "enc_forward per step"),
         "roofline": roof,
         "e2e": {"value": wl.batch * world / (e2e_step * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": int(hx.numel() * hx.element_size() + hvl.numel() * 4),
@@ -338,6 +352,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of a recorded forward (enc_graph_launch) instead of enc_forward calls")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-sample", type=int, default=8, help="sequences per reference-arm step")
     ap.add_argument("--traffic", type=float, default=None,

@@ -53,6 +53,7 @@ extern "C" {
 typedef struct CUstream_st* enc_stream_t;
 
 typedef struct enc_handle* enc_t;
+typedef struct enc_graph_s* enc_graph_t;
 
 typedef enum {
   ENC_OK = 0,
@@ -64,6 +65,12 @@ typedef enum {
 } enc_status;
 
 typedef enum { ENC_FP32 = 0, ENC_FP16 = 1 } enc_dtype;
+
+/* FFN activation.  ENC_GELU_ERF: 0.5 t (1 + erf(t / sqrt 2)) (default).
+ * ENC_GELU_TANH: 0.5 t (1 + tanh(sqrt(2/pi) (t + 0.044715 t^3))), the form the
+ * source page implies when it replaces pow(x, 3) by x*x*x ([FT] "Faster
+ * Transformer 优化原理"). */
+typedef enum { ENC_GELU_ERF = 0, ENC_GELU_TANH = 1 } enc_gelu;
 
 /* One layer's parameters.  Element type = the handle's dtype (float or IEEE half).
  * Matrices are [in, out] row-major (y = x W + b).  Wqkv's columns are Q | K | V,
@@ -83,7 +90,10 @@ typedef struct {
  * [FT] "什么是 Faster Transformer": head_num and size_per_head are the two
  * structural parameters; ffn_dim and num_layers complete the stack.
  *   head_num, ffn_dim, num_layers > 0; size_per_head in {32, 64, 128}
- *   (else ENC_ERR_UNSUPPORTED); ffn_dim a multiple of 8.
+ *   (else ENC_ERR_UNSUPPORTED); ffn_dim a multiple of 8; hidden size
+ *   H = head_num * size_per_head at most 2048 in FP16 mode and 1024 in FP32
+ *   mode (else ENC_ERR_UNSUPPORTED: a LayerNorm row lives in one warp's
+ *   registers).
  *   weights: array of num_layers structs (see enc_layer_weights).
  * The handle copies and repacks every parameter into its own device memory
  * (FP16 weights are stored transposed, [out, in], for the tensor-core GEMMs;
@@ -91,6 +101,10 @@ typedef struct {
  * its buffers on return.  Synchronous.  On error *out is set to NULL. */
 ENC_API enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_layers,
                       enc_dtype dtype, const enc_layer_weights* weights, enc_t* out);
+
+/* enc_set_gelu - choose the FFN activation of every later call on this handle
+ * (host-side setting; takes effect at the next launch). */
+ENC_API enc_status enc_set_gelu(enc_t h, enc_gelu form);
 
 /* enc_forward - run the whole encoder stack on `stream`.
  * [FT] "什么是 Faster Transformer" (batch size and sequence length per run)
@@ -132,6 +146,23 @@ ENC_API const char* enc_last_error(void);
  * read; otherwise the code of the first failure (1 = a bounded wait inside a
  * tensor-core GEMM gave up).  Returns ENC_ERR_DEVICE when *code != 0. */
 ENC_API enc_status enc_device_status(enc_t h, int32_t* code);
+
+/* enc_graph_create - record one enc_forward (these exact buffers, batch and seq)
+ * as an instantiated CUDA graph, so that it replays with a single launch.
+ * [FT] "Faster Transformer 优化原理": at small batch the cost is kernel
+ * launches, not arithmetic.  The workspace is reserved first; while any graph
+ * of the handle exists the workspace is pinned, and an enc_forward that would
+ * need a larger one returns ENC_ERR_INVALID_ARG.  Synchronous.  The graph
+ * reads x and valid_len and writes out at replay time; the caller keeps those
+ * buffers alive until enc_graph_destroy. */
+ENC_API enc_status enc_graph_create(enc_t h, const void* x, const int32_t* valid_len, void* out,
+                                    int batch, int seq, enc_graph_t* graph);
+
+/* enc_graph_launch - replay a recorded forward on `stream` (asynchronous). */
+ENC_API enc_status enc_graph_launch(enc_graph_t graph, enc_stream_t stream);
+
+/* enc_graph_destroy - release a recorded forward (synchronises the device). NULL is a no-op. */
+ENC_API enc_status enc_graph_destroy(enc_graph_t graph);
 
 /* enc_kernels_per_forward - kernel launches one enc_forward issues (7 per layer). */
 ENC_API int enc_kernels_per_forward(enc_t h);

@@ -107,6 +107,22 @@ def test_full_size_workloads_sampled(kind, batch, seq, nsample):
     _check(got[seqs], ref, inp.valid_len[seqs], wl.seq, FP16_STACK_REL_L2)
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "fp32"])
+def test_tanh_gelu_variant(dtype):
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    inp = EI.make_inputs(EI.Workload("tanh", sh, 4, 40, dtype, 1, 40, seed=6, ln_affine_random=True))
+    enc = encoder_from_inputs(inp)
+    enc.set_gelu("tanh")
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    x64, vl, layers = inp.as_float64()
+    ref = O.encoder_forward(x64, vl, layers, 12, 64, gelu="tanh")
+    tol = 2 * (FP16_LAYER_REL_L2 if dtype == "fp16" else FP32_LAYER_REL_L2)
+    _check(got, ref, vl, 40, tol)
+    # and it differs measurably from the erf form (the switch takes effect)
+    ref_erf = O.encoder_forward(x64, vl, layers, 12, 64, gelu="erf")
+    assert rel_l2(ref, ref_erf, valid_mask(vl, 40)) > 1e-6
+
+
 def test_padding_tokens_do_not_change_valid_outputs():
     sh = EI.EncoderShape(12, 64, 3072, 2)
     inp = EI.make_inputs(EI.Workload("pad", sh, 6, 70, "fp16", 5, 60, seed=4))
@@ -170,3 +186,35 @@ def test_host_argument_checks():
     assert e.value.status == 1
     with pytest.raises(EncError):
         enc.op_ffn1(3, x, x, 16)                        # layer out of range
+
+
+def test_recorded_forward_replays_bit_exact():
+    import torch
+    from transformer_encoder_bert_b200 import EncError
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 8))
+    enc = encoder_from_inputs(inp)
+    x, vl = to_dev(inp.x), to_dev(inp.valid_len)
+    ref = to_host(enc.forward(x, vl))
+    out = torch.zeros_like(x)
+    g = enc.record(x, vl, out)
+    assert np.all(to_host(out) == 0)                  # recording runs nothing
+    n0 = enc.launch_count()
+    s = torch.cuda.Stream()
+    for _ in range(3):
+        g.launch(stream=s)
+    s.synchronize()
+    assert enc.launch_count() - n0 == 3 * enc.kernels_per_forward()
+    assert np.array_equal(to_host(out), ref)
+    # new input values in the same buffers are picked up at replay time
+    x2 = EI.make_inputs(EI.named_workload("bert-base-s32", 8).with_(seed=5)).x
+    x.copy_(to_dev(x2))
+    g.launch()
+    torch.cuda.synchronize()
+    assert np.array_equal(to_host(out), to_host(enc.forward(x, vl)))
+    # the workspace is pinned while the graph exists
+    big = torch.empty((64, 32, 768), dtype=torch.float16, device="cuda")
+    with pytest.raises(EncError):
+        enc.forward(big, to_dev(np.full(64, 32, np.int32)))
+    g.close()
+    enc.forward(big, to_dev(np.full(64, 32, np.int32)))
+    assert enc.device_status() == 0

@@ -172,10 +172,11 @@ def test_gemm_bounded_waits_never_fired():
     assert enc.device_status() == 0
 
 
+@pytest.mark.parametrize("form", ["erf", "tanh"])
 @pytest.mark.parametrize("hidden,batch,seq", [(128, 3, 37), (256, 4, 96)], ids=["one-cta", "cta-pair"])
-def test_gelu_epilogue_against_exact_erf(hidden, batch, seq):
+def test_gelu_epilogue_against_exact_erf(hidden, batch, seq, form):
     """W1 = I, b1 = 0 turns FFN1 into GELU of its FP16 input; inputs span [-8, 8].
-    The result must be the exact erf-GELU rounded once to FP16."""
+    The result must be the exact GELU (erf form, or the tanh form) rounded once to FP16."""
     from transformer_encoder_bert_b200 import Encoder
     nh, d = hidden // 32, 32
     M = batch * seq
@@ -183,20 +184,23 @@ def test_gelu_epilogue_against_exact_erf(hidden, batch, seq):
     lw["w_ff1"] = np.eye(hidden, dtype=np.float16)
     lw["b_ff1"] = np.zeros(hidden, np.float16)
     enc = Encoder(nh, d, hidden, [lw], "fp16")
+    enc.set_gelu(form)
     h1 = np.linspace(-8, 8, M * hidden).astype(np.float16).reshape(M, hidden)
     u = empty_dev((M, hidden), "fp16")
     enc.op_ffn1(0, to_dev(h1), u, M)
     got = to_host(u).astype(np.float64)
-    ref = O.gelu_erf(h1.astype(np.float64))
+    ref = O.GELU[form](h1.astype(np.float64))
     # one FP16 rounding of the exact value: |got - ref| <= half an ulp of |ref| (+ tiny slack)
     ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
     assert np.all(np.abs(got - ref) <= 0.5 * ulp + 1e-6)
 
 
+@pytest.mark.parametrize("env", ["ENC_GEMM_NO_PAIR", "ENC_GEMM_NO_TMA_STORE"])
 @pytest.mark.parametrize("batch,seq", [(2, 128), (5, 131)], ids=str)
-def test_one_cta_tiles_when_pairs_disabled(monkeypatch, batch, seq):
-    """The one-CTA 128x256 tile path (used for small M) on shapes that normally take the pair path."""
-    monkeypatch.setenv("ENC_GEMM_NO_PAIR", "1")
+def test_alternative_gemm_paths(monkeypatch, env, batch, seq):
+    """The one-CTA tile path (used for small M) and the direct-store epilogue (used when
+    the output map cannot be built) on shapes that normally take the pair / TMA-store path."""
+    monkeypatch.setenv(env, "1")
     shape = (12, 64, 3072)
     nh, d, F = shape
     H = nh * d

@@ -352,3 +352,27 @@ def test_planted_mistake_is_caught(monkeypatch, name):
     ref = torch_encoder(x, vl, layers, 2)
     worst = max(np.max(np.abs(got[b, :int(vl[b])] - ref[b, :int(vl[b])])) for b in range(wl.batch))
     assert worst > 1e-6, f"planted mistake {name} was not detected (diff {worst:g})"
+
+
+def test_gelu_tanh_form_matches_library_routine():
+    # torch.nn.functional.gelu(approximate="tanh") is the library form of the same approximation.
+    t = np.linspace(-9, 9, 4001)
+    ref = torch.nn.functional.gelu(torch.from_numpy(t), approximate="tanh").numpy()
+    assert np.max(np.abs(O.gelu_tanh(t) - ref)) < 1e-15
+    # GELU(t) - GELU(-t) = t holds for both forms (the inner function is odd)
+    assert np.max(np.abs(O.gelu_tanh(t) - O.gelu_tanh(-t) - t)) < 1e-14
+    assert np.max(np.abs(O.gelu_erf(t) - O.gelu_erf(-t) - t)) < 1e-14
+
+
+def test_tanh_gelu_encoder_matches_torch_tanh_gelu():
+    wl, inp = _tiny_workload(nh=2, d=8, F=32, L=1, B=3, S=7, lo=1, seed=31, std=0.1)
+    x, vl, layers = _f64(inp)
+    got = O.encoder_forward(x, vl, layers, 2, 8, gelu="tanh")
+    layer = _torch_layer(layers[0], 16, 2, 32)
+    layer.activation = lambda v: torch.nn.functional.gelu(v, approximate="tanh")
+    mask = torch.arange(7)[None, :] >= torch.from_numpy(np.asarray(vl, dtype=np.int64))[:, None]
+    with torch.no_grad():
+        ref = layer(torch.from_numpy(x), src_key_padding_mask=mask).numpy()
+    for b in range(3):
+        n = int(vl[b])
+        assert np.max(np.abs(got[b, :n] - ref[b, :n])) < 1e-10

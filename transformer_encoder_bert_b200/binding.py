@@ -35,6 +35,10 @@ SIGNATURES = {
     "enc_destroy": (_i, [_vp]),
     "enc_last_error": (ctypes.c_char_p, []),
     "enc_device_status": (_i, [_vp, ctypes.POINTER(ctypes.c_int32)]),
+    "enc_set_gelu": (_i, [_vp, _i]),
+    "enc_graph_create": (_i, [_vp, _vp, _vp, _vp, _i, _i, ctypes.POINTER(_vp)]),
+    "enc_graph_launch": (_i, [_vp, _vp]),
+    "enc_graph_destroy": (_i, [_vp]),
     "enc_kernels_per_forward": (_i, [_vp]),
     "enc_launch_count": (ctypes.c_uint64, [_vp]),
     "enc_set_trace_events": (_i, [_vp, _vp, _i]),
@@ -149,6 +153,10 @@ class Encoder:
         self.close()
 
     # -------------------------------------------------------------- whole stack
+    def set_gelu(self, form: str):
+        """"erf" (default) or "tanh"."""
+        _check(self.lib.enc_set_gelu(self.handle, {"erf": 0, "tanh": 1}[form]))
+
     def reserve(self, batch: int, seq: int):
         _check(self.lib.enc_reserve(self.handle, batch, seq))
 
@@ -181,6 +189,14 @@ class Encoder:
         """enc_forward_host on raw host pointers (e.g. pinned torch tensors)."""
         _check(self.lib.enc_forward_host(self.handle, x_ptr, vl_ptr, out_ptr, batch, seq,
                                          _current_stream(stream)))
+
+    def record(self, x, valid_len, out) -> "RecordedForward":
+        """Record one forward on these CUDA tensors as a CUDA graph (see enc_graph_create)."""
+        B, S, _ = x.shape
+        g = ctypes.c_void_p()
+        _check(self.lib.enc_graph_create(self.handle, _dptr(x), _dptr(valid_len), _dptr(out), B, S,
+                                         ctypes.byref(g)))
+        return RecordedForward(self, g, (x, valid_len, out))
 
     def kernels_per_forward(self) -> int:
         return int(self.lib.enc_kernels_per_forward(self.handle))
@@ -235,6 +251,27 @@ class Encoder:
 
     def op_ffn2(self, layer: int, u, y, tokens: int, stream=None):
         _check(self.lib.enc_op_ffn2(self.handle, layer, _dptr(u), _dptr(y), tokens, _current_stream(stream)))
+
+
+class RecordedForward:
+    """A forward recorded by Encoder.record; launch() replays it on a stream."""
+
+    def __init__(self, enc: Encoder, g: ctypes.c_void_p, keep):
+        self.enc, self.g, self._keep = enc, g, keep
+
+    def launch(self, stream=None):
+        _check(self.enc.lib.enc_graph_launch(self.g, _current_stream(stream)))
+
+    def close(self):
+        if self.g is not None and self.g.value:
+            _check(self.enc.lib.enc_graph_destroy(self.g))
+        self.g = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def declared_symbols(header: Optional[str] = None) -> List[str]:

@@ -6,7 +6,7 @@
 // shapes), with row sums by warp shuffle and FP32 sums for FP16 data, plus a
 // transpose kernel.  Here the score tile never leaves the chip: each warp
 // keeps 16 query rows' scores in registers, takes the row max and row sum
-// with quad shuffles in FP32, and streams keys in blocks of 64 with an online
+// with quad shuffles in FP32, and streams keys in blocks of 32 or 64 with an online
 // softmax, so short (one key block) and long sequences share one kernel.
 // Only key blocks that hold valid keys (j < n) are visited.
 //
@@ -19,7 +19,6 @@
 namespace enc {
 namespace {
 
-constexpr int kBKV = 64;                        // keys per block
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -59,25 +58,31 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// One CTA = NW warps = 16*NW query rows of one (sequence, head).
-template <int D, int NW>
+// One CTA = NW warps = 16*NW query rows of one (sequence, head); keys are
+// streamed in blocks of BKV (32 for sequences of at most 32 tokens, so that no
+// score MMA is spent on padding, else 64).
+// STAGES = 2 double-buffers the K/V blocks; STAGES = 1 when one block covers
+// every key (S <= BKV), which halves the shared memory and so raises the number
+// of resident CTAs.
+template <int D, int NW, int BKV, int STAGES>
 struct AttnCfg {
   static constexpr int kBQ = 16 * NW;
   static constexpr int kLd = D + 8;                         // padded row (halves): conflict-free ldmatrix
   static constexpr int kQElems = kBQ * kLd;
-  static constexpr int kKVElems = kBKV * kLd;
-  static constexpr int kSmem = (kQElems + 4 * kKVElems) * 2;  // Q + 2 stages x (K, V)
+  static constexpr int kKVElems = BKV * kLd;
+  static constexpr int kSmem = (kQElems + 2 * STAGES * kKVElems) * 2;  // Q + STAGES x (K, V)
 };
 
-template <int D, int NW>
+template <int D, int NW, int BKV, int STAGES>
 __global__ void __launch_bounds__(NW * 32)
     attention_f16_kernel(const __half* __restrict__ qkv, const int32_t* __restrict__ valid_len,
                          __half* __restrict__ ctx, int B, int S, int NH, float score_scale_log2) {
-  using C = AttnCfg<D, NW>;
+  using C = AttnCfg<D, NW, BKV, STAGES>;
+  constexpr int kBKV = BKV;
   extern __shared__ __align__(16) __half sm[];
   __half* Qs = sm;
-  __half* Ks = sm + C::kQElems;                 // [2][kBKV][kLd]
-  __half* Vs = Ks + 2 * C::kKVElems;            // [2][kBKV][kLd]
+  __half* Ks = sm + C::kQElems;                 // [STAGES][kBKV][kLd]
+  __half* Vs = Ks + STAGES * C::kKVElems;       // [STAGES][kBKV][kLd]
 
   const int b = blockIdx.z, h = blockIdx.y, q0 = blockIdx.x * C::kBQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(NW * 32)
   uint32_t qf[D / 16][4];
 
   for (int kb = 0; kb < num_kb; ++kb) {
-    if (kb + 1 < num_kb) load_kv(kb + 1, (kb + 1) & 1);
+    if (STAGES > 1 && kb + 1 < num_kb) load_kv(kb + 1, (kb + 1) % STAGES);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
@@ -134,10 +139,10 @@ __global__ void __launch_bounds__(NW * 32)
         ldsm_x4(smem_addr(Qs + r * C::kLd + c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
       }
     }
-    const __half* kbuf = Ks + (kb & 1) * C::kKVElems;
-    const __half* vbuf = Vs + (kb & 1) * C::kKVElems;
+    const __half* kbuf = Ks + (kb % STAGES) * C::kKVElems;
+    const __half* vbuf = Vs + (kb % STAGES) * C::kKVElems;
 
-    // Scores for this warp's 16 rows x 64 keys.
+    // Scores for this warp's 16 rows x kBKV keys.
     float s[kBKV / 8][4];
 #pragma unroll
     for (int i = 0; i < kBKV / 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
@@ -242,29 +247,221 @@ __global__ void __launch_bounds__(NW * 32)
   }
 }
 
-template <int D, int NW>
+template <int D, int NW, int BKV, int STAGES>
 cudaError_t launch_f16(const __half* qkv, const int32_t* vl, __half* ctx, int B, int S, int NH,
                        cudaStream_t stream) {
-  using C = AttnCfg<D, NW>;
+  using C = AttnCfg<D, NW, BKV, STAGES>;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(attention_f16_kernel<D, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    attr = cudaFuncSetAttribute(attention_f16_kernel<D, NW, BKV, STAGES>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   });
   if (attr != cudaSuccess) return attr;
   const dim3 grid((S + C::kBQ - 1) / C::kBQ, NH, B);
   const float scale_log2 = kLog2e / sqrtf((float)D);
-  attention_f16_kernel<D, NW><<<grid, NW * 32, C::kSmem, stream>>>(qkv, vl, ctx, B, S, NH, scale_log2);
+  attention_f16_kernel<D, NW, BKV, STAGES><<<grid, NW * 32, C::kSmem, stream>>>(qkv, vl, ctx, B, S, NH,
+                                                                                 scale_log2);
   return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------------------
+// Short sequences (S <= BKV, so one query block of 16*NW rows and one key
+// block cover a whole (sequence, head)): a persistent CTA walks (sequence,
+// head) items with two shared-memory buffers, so the next item's Q/K/V copies
+// are in flight while the current item is computed.  The single key block
+// needs no online rescaling: row max, exponentials, row sum, PV.
+// ---------------------------------------------------------------------------
+template <int D, int NW, int BKV>
+struct ShortCfg {
+  static constexpr int kBQ = 16 * NW;
+  static constexpr int kLd = D + 8;
+  static constexpr int kBufElems = (kBQ + 2 * BKV) * kLd;   // Q, K, V of one item
+  static constexpr int kSmem = 2 * kBufElems * 2;
+};
+
+template <int D, int NW, int BKV>
+__global__ void __launch_bounds__(NW * 32)
+    attention_f16_short_kernel(const __half* __restrict__ qkv, const int32_t* __restrict__ valid_len,
+                               __half* __restrict__ ctx, int B, int S, int NH, float score_scale_log2) {
+  using C = ShortCfg<D, NW, BKV>;
+  static_assert(C::kBQ <= BKV || C::kBQ == 16 * NW, "one query block");
+  extern __shared__ __align__(16) __half sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  constexpr int kChunks = D / 8;
+  const int items = B * NH;
+  const size_t head_elems = (size_t)S * D;
+  const int H = NH * D;
+
+  auto issue_loads = [&](int item, int buf) {
+    const int b = item / NH, h = item - b * NH;
+    const __half* Qg = qkv + (((size_t)0 * B + b) * NH + h) * head_elems;
+    const __half* Kg = qkv + (((size_t)1 * B + b) * NH + h) * head_elems;
+    const __half* Vg = qkv + (((size_t)2 * B + b) * NH + h) * head_elems;
+    __half* qs = sm + buf * C::kBufElems;
+    __half* ks = qs + C::kBQ * C::kLd;
+    __half* vs = ks + BKV * C::kLd;
+    for (int i = threadIdx.x; i < BKV * kChunks; i += NW * 32) {
+      const int r = i / kChunks, c = i % kChunks;
+      const bool v = r < S;
+      const size_t off = (size_t)(v ? r : 0) * D + c * 8;
+      if (r < C::kBQ) cp_async16(smem_addr(qs + r * C::kLd + c * 8), Qg + off, v);
+      cp_async16(smem_addr(ks + r * C::kLd + c * 8), Kg + off, v);
+      cp_async16(smem_addr(vs + r * C::kLd + c * 8), Vg + off, v);
+    }
+  };
+
+  int item = blockIdx.x;
+  if (item < items) issue_loads(item, 0);
+  cp_async_commit();
+  for (int it = 0; item < items; ++it, item += gridDim.x) {
+    const int buf = it & 1;
+    const int next = item + gridDim.x;
+    if (next < items) issue_loads(next, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+
+    const int b = item / NH, h = item - b * NH;
+    int n = valid_len[b];
+    n = n < 0 ? 0 : (n > S ? S : n);
+    __half* qs = sm + buf * C::kBufElems;
+    const __half* ks = qs + C::kBQ * C::kLd;
+    const __half* vs = ks + BKV * C::kLd;
+
+    uint32_t qf[D / 16][4];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = warp * 16 + (lane & 15);
+      const int c = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4(smem_addr(qs + r * C::kLd + c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+    }
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float l_run[2] = {0.f, 0.f};
+    if (n > 0) {
+      float s[BKV / 8][4];
+#pragma unroll
+      for (int i = 0; i < BKV / 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+        for (int np = 0; np < BKV / 16; ++np) {
+          const int key = np * 16 + (lane >> 4) * 8 + (lane & 7);
+          const int dim = kk * 16 + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(smem_addr(ks + key * C::kLd + dim), b0, b1, b2, b3);
+          mma16816(s[2 * np], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
+          mma16816(s[2 * np + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
+        }
+      }
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < BKV / 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = nt * 8 + 2 * t + (e & 1);
+          if (j >= n) s[nt][e] = -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        mx[r] *= score_scale_log2;
+      }
+#pragma unroll
+      for (int nt = 0; nt < BKV / 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p = exp2f(fmaf(s[nt][e], score_scale_log2, -mx[e >> 1]));
+          s[nt][e] = p;
+          l_run[e >> 1] += p;
+        }
+      }
+#pragma unroll
+      for (int kc = 0; kc < BKV / 16; ++kc) {
+        const uint32_t a0 = pack_h2(s[2 * kc][0], s[2 * kc][1]);
+        const uint32_t a1 = pack_h2(s[2 * kc][2], s[2 * kc][3]);
+        const uint32_t a2 = pack_h2(s[2 * kc + 1][0], s[2 * kc + 1][1]);
+        const uint32_t a3 = pack_h2(s[2 * kc + 1][2], s[2 * kc + 1][3]);
+#pragma unroll
+        for (int dp = 0; dp < D / 16; ++dp) {
+          const int key = kc * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          const int dim = dp * 16 + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(smem_addr(vs + key * C::kLd + dim), b0, b1, b2, b3);
+          mma16816(o[2 * dp], a0, a1, a2, a3, b0, b1);
+          mma16816(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+      l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+    }
+    const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;   // n == 0: ctx = 0
+    const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
+    // Stage this warp's 16 output rows over its own Q rows (already in registers).
+    __syncwarp();
+    __half* orow = qs + warp * 16 * C::kLd;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      *reinterpret_cast<uint32_t*>(orow + g * C::kLd + i * 8 + 2 * t) = pack_h2(o[i][0] * inv0, o[i][1] * inv0);
+      *reinterpret_cast<uint32_t*>(orow + (g + 8) * C::kLd + i * 8 + 2 * t) = pack_h2(o[i][2] * inv1, o[i][3] * inv1);
+    }
+    __syncwarp();
+    for (int i = lane; i < 16 * kChunks; i += 32) {
+      const int r = i / kChunks, c = i % kChunks;
+      const int row = warp * 16 + r;
+      if (row < S) {
+        *reinterpret_cast<uint4*>(ctx + ((size_t)b * S + row) * H + h * D + c * 8) =
+            *reinterpret_cast<const uint4*>(orow + r * C::kLd + c * 8);
+      }
+    }
+    __syncthreads();   // buffer `buf` is refilled by the prefetch two items ahead
+  }
+  cp_async_wait<0>();
+}
+
+template <int D, int NW, int BKV>
+cudaError_t launch_short(const __half* qkv, const int32_t* vl, __half* ctx, int B, int S, int NH,
+                         cudaStream_t stream) {
+  using C = ShortCfg<D, NW, BKV>;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  static int per_sm = 1;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(attention_f16_short_kernel<D, NW, BKV>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (attr == cudaSuccess)
+      attr = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_f16_short_kernel<D, NW, BKV>, NW * 32,
+                                                           C::kSmem);
+    if (per_sm < 1) per_sm = 1;
+  });
+  if (attr != cudaSuccess) return attr;
+  const int items = B * NH;
+  const int cap = per_sm * device_sm_count();
+  const float scale_log2 = kLog2e / sqrtf((float)D);
+  attention_f16_short_kernel<D, NW, BKV><<<items < cap ? items : cap, NW * 32, C::kSmem, stream>>>(
+      qkv, vl, ctx, B, S, NH, scale_log2);
+  return cudaGetLastError();
+}
+
+// Launch shape by sequence length ([FT] "Faster Transformer 优化原理" keeps
+// several SoftMax versions and picks grid/block sizes from the shape).
 template <int D>
 cudaError_t launch_f16_d(const __half* qkv, const int32_t* vl, __half* ctx, int B, int S, int NH,
                          cudaStream_t stream) {
-  if (S <= 16) return launch_f16<D, 1>(qkv, vl, ctx, B, S, NH, stream);
-  if (S <= 32) return launch_f16<D, 2>(qkv, vl, ctx, B, S, NH, stream);
-  if (S <= 64) return launch_f16<D, 4>(qkv, vl, ctx, B, S, NH, stream);
-  return launch_f16<D, 8>(qkv, vl, ctx, B, S, NH, stream);
+  if (S <= 16) return launch_short<D, 1, 32>(qkv, vl, ctx, B, S, NH, stream);
+  if (S <= 32) return launch_short<D, 2, 32>(qkv, vl, ctx, B, S, NH, stream);
+  if (S <= 64) return launch_short<D, 4, 64>(qkv, vl, ctx, B, S, NH, stream);
+  return launch_f16<D, 8, 64, 2>(qkv, vl, ctx, B, S, NH, stream);
 }
 
 // ---------------------------------------------------------------- FP32 (CUDA cores)

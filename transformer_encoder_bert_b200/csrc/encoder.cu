@@ -78,6 +78,10 @@ struct LayerDev {
   void* w_ff2 = nullptr;   // FP16: [H, F]; FP32: [F, H]
   float *b_qkv = nullptr, *b_o = nullptr, *b_ff1 = nullptr, *b_ff2 = nullptr;
   float *ln1_g = nullptr, *ln1_b = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
+  // FP16 copies (FP16 mode only; exact, the caller supplied halves) for the LayerNorm kernel:
+  // b_o, ln1_g, ln1_b, b_ff2, ln2_g, ln2_b.
+  __half *h_b_o = nullptr, *h_ln1_g = nullptr, *h_ln1_b = nullptr, *h_b_ff2 = nullptr, *h_ln2_g = nullptr,
+         *h_ln2_b = nullptr;
   CUtensorMap tm_qkv[2], tm_o[2], tm_ff1[2], tm_ff2[2];   // [0]: 128-row box, [1]: 256-row box
 };
 
@@ -97,7 +101,10 @@ struct enc_handle {
   size_t stage_bytes = 0;
   int* status = nullptr;
   uint64_t launches = 0;            // kernels launched through this handle
+  int graphs_alive = 0;             // recorded forwards that reference the workspace
+  enc_gelu gelu = ENC_GELU_ERF;
   bool no_pair = false;             // ENC_GEMM_NO_PAIR=1: one-CTA tiles only (comparison runs)
+  bool no_tma_store = false;        // ENC_GEMM_NO_TMA_STORE=1: epilogue stores without TMA
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -133,6 +140,9 @@ Workspace carve(const enc_handle* h, size_t tokens) {
 enc_status ensure_workspace(enc_handle* h, size_t tokens) {
   const size_t need = workspace_bytes(h, tokens);
   if (need <= h->ws_bytes) return ENC_OK;
+  if (h->graphs_alive > 0)
+    return fail(ENC_ERR_INVALID_ARG, "workspace of %zu bytes needed but %d recorded graph(s) pin the current one",
+                need, h->graphs_alive);
   if (h->ws) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize before workspace growth");
@@ -175,8 +185,19 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
     CUtensorMap ta;
     if (!enc::encode_kmajor_fp16_map(&ta, A, (uint64_t)M, (uint64_t)K, 128))
       return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation operand [%d, %d]", M, K);
+    // Output through TMA stores (32x32 boxes); the head split needs whole
+    // 32-token chunks per sequence, otherwise its epilogue stores directly.
+    CUtensorMap tc;
+    bool use_tc = !h->no_tma_store;
+    if (use_tc) {
+      if (epi == enc::Epi::kBiasQkvSplit)
+        use_tc = (sp.seq % 32 == 0) && enc::encode_output_map_split(&tc, C, sp);
+      else
+        use_tc = enc::encode_output_map_2d(&tc, C, (uint64_t)M, (uint64_t)N);
+    }
     enc::TcGemmArgs a;
     a.tmap_a = &ta;
+    a.tmap_c = use_tc ? &tc : nullptr;
     a.tmap_b = &wmaps[bn == 256 ? 1 : 0];      // the pair tile loads 128-row halves of B
     a.M = M; a.N = N; a.K = K; a.bn = bn; a.epi = epi; a.bias = bias;
     a.c = static_cast<__half*>(C);
@@ -228,6 +249,14 @@ enc_status step_ln(enc_handle* h, int l, int which, const void* a, const void* r
   const float* g = which == 1 ? L.ln1_g : L.ln2_g;
   const float* b = which == 1 ? L.ln1_b : L.ln2_b;
   cudaError_t e;
+#ifndef ENC_LN_SMEM
+  if (h->dtype == ENC_FP16 && h->H <= 1024)
+    e = enc::launch_bias_residual_ln_f16h(static_cast<const __half*>(a), which == 1 ? L.h_b_o : L.h_b_ff2,
+                                          static_cast<const __half*>(resid), which == 1 ? L.h_ln1_g : L.h_ln2_g,
+                                          which == 1 ? L.h_ln1_b : L.h_ln2_b, static_cast<__half*>(out), tokens,
+                                          h->H, st);
+  else
+#endif
   if (h->dtype == ENC_FP16)
     e = enc::launch_bias_residual_ln_f16(static_cast<const __half*>(a), bias, static_cast<const __half*>(resid),
                                          g, b, static_cast<__half*>(out), tokens, h->H, st);
@@ -241,7 +270,8 @@ enc_status step_ln(enc_handle* h, int l, int which, const void* a, const void* r
 
 enc_status step_ffn1(enc_handle* h, int l, const void* h1, void* u, int tokens, cudaStream_t st) {
   LayerDev& L = h->layers[l];
-  return run_gemm(h, h1, tokens, h->H, L.w_ff1, L.tm_ff1, h->F, enc::Epi::kBiasGelu, L.b_ff1, u, {}, st);
+  const enc::Epi epi = h->gelu == ENC_GELU_TANH ? enc::Epi::kBiasGeluTanh : enc::Epi::kBiasGelu;
+  return run_gemm(h, h1, tokens, h->H, L.w_ff1, L.tm_ff1, h->F, epi, L.b_ff1, u, {}, st);
 }
 
 enc_status step_ffn2(enc_handle* h, int l, const void* u, void* y, int tokens, cudaStream_t st) {
@@ -297,7 +327,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   if (dtype != ENC_FP16 && dtype != ENC_FP32) return fail(ENC_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   if (ffn_dim % 8 != 0) return fail(ENC_ERR_INVALID_ARG, "ffn_dim %d is not a multiple of 8", ffn_dim);
   const int H = head_num * size_per_head;
-  const int max_h = dtype == ENC_FP16 ? 4096 : 2048;
+  const int max_h = dtype == ENC_FP16 ? 2048 : 1024;
   if (H > max_h) return fail(ENC_ERR_UNSUPPORTED, "hidden size %d exceeds %d", H, max_h);
   if (!weights) return fail(ENC_ERR_INVALID_ARG, "weights is null");
   for (int l = 0; l < num_layers; ++l) {
@@ -315,6 +345,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   cudaGetDevice(&h->device);
   h->num_sms = enc::device_sm_count();
   if (const char* e = getenv("ENC_GEMM_NO_PAIR")) h->no_pair = e[0] == '1';
+  if (const char* e = getenv("ENC_GEMM_NO_TMA_STORE")) h->no_tma_store = e[0] == '1';
   if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
   if (dtype == ENC_FP16) {
     cudaDeviceProp prop;
@@ -336,6 +367,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   size_t per_layer = 0;
   for (size_t s : wsz) per_layer += align_up(s * es, 256);
   for (size_t s : vsz) per_layer += align_up(s * 4, 256);
+  if (dtype == ENC_FP16) per_layer += 6 * align_up((size_t)H * 2, 256);
   size_t staging = 0;
   for (size_t s : wsz) staging = std::max(staging, align_up(s * es, 256));
   if (cudaMalloc(&h->param_block, per_layer * num_layers + staging) != cudaSuccess) {
@@ -391,6 +423,16 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
       p += align_up(n * 4, 256);
     }
     if (dtype == ENC_FP16) {
+      const void* hsrc[6] = {w.b_o, w.ln1_g, w.ln1_b, w.b_ff2, w.ln2_g, w.ln2_b};
+      __half** hdst[6] = {&L.h_b_o, &L.h_ln1_g, &L.h_ln1_b, &L.h_b_ff2, &L.h_ln2_g, &L.h_ln2_b};
+      for (int i = 0; i < 6; ++i) {
+        *hdst[i] = reinterpret_cast<__half*>(p);
+        cudaError_t e = cudaMemcpy(p, hsrc[i], (size_t)H * 2, cudaMemcpyDefault);
+        if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "parameter upload"); }
+        p += align_up((size_t)H * 2, 256);
+      }
+    }
+    if (dtype == ENC_FP16) {
       // B operands [N, K]: Wqkv^T [3H, H], Wo^T [H, H], W1^T [F, H], W2^T [H, F].
       struct { CUtensorMap* m; void* w; int n, k; } maps[4] = {
           {L.tm_qkv, L.w_qkv, 3 * H, H}, {L.tm_o, L.w_o, H, H}, {L.tm_ff1, L.w_ff1, ffn_dim, H},
@@ -421,8 +463,13 @@ enc_status enc_reserve(enc_t h, int batch, int seq) {
   return ok();
 }
 
-enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
-                       enc_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks, workspace, and the per-layer launches of one forward on `st`.
+enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                        cudaStream_t st, bool tracing) {
   enc_status s = check_handle(h);
   if (s != ENC_OK) return s;
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
@@ -434,10 +481,9 @@ enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* o
   const char* ob = static_cast<const char*>(out);
   if (xb < ob + bytes && ob < xb + bytes) return fail(ENC_ERR_INVALID_ARG, "out overlaps x");
   if ((s = ensure_workspace(h, M)) != ENC_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Workspace w = carve(h, M);
   const int tokens = (int)M;
-  const bool tracing = !h->trace.empty();
+  tracing = tracing && !h->trace.empty();
   int k = 0;
   auto mark = [&]() {
     if (tracing) cudaEventRecord(h->trace[k++], st);
@@ -461,6 +507,82 @@ enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* o
     if ((s = step_ln(h, l, 2, w.a, w.h1, xout, tokens, st)) != ENC_OK) return s;
   }
   mark();
+  return ENC_OK;
+}
+
+}  // namespace
+
+struct enc_graph_s {
+  enc_handle* h = nullptr;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+
+extern "C" {
+
+enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                       enc_stream_t stream) {
+  enc_status s = forward_impl(h, x, valid_len, out, batch, seq, reinterpret_cast<cudaStream_t>(stream), true);
+  return s == ENC_OK ? ok() : s;
+}
+
+enc_status enc_graph_create(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                            enc_graph_t* graph) {
+  if (!graph) return fail(ENC_ERR_INVALID_ARG, "graph is null");
+  *graph = nullptr;
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if ((s = ensure_workspace(h, (size_t)batch * seq)) != ENC_OK) return s;   // no allocation while recording
+  cudaStream_t st = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
+  const uint64_t launches_before = h->launches;
+  e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(st);
+    return cuda_fail(e, "cudaStreamBeginCapture");
+  }
+  s = forward_impl(h, x, valid_len, out, batch, seq, st, false);
+  cudaGraph_t g = nullptr;
+  e = cudaStreamEndCapture(st, &g);
+  cudaStreamDestroy(st);
+  h->launches = launches_before;            // recording launches nothing
+  if (s != ENC_OK) {
+    if (g) cudaGraphDestroy(g);
+    return s;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamEndCapture");
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, g, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return cuda_fail(e, "cudaGraphInstantiate");
+  }
+  enc_graph_s* out_g = new enc_graph_s();
+  out_g->h = h;
+  out_g->graph = g;
+  out_g->exec = exec;
+  ++h->graphs_alive;
+  *graph = out_g;
+  return ok();
+}
+
+enc_status enc_graph_launch(enc_graph_t graph, enc_stream_t stream) {
+  if (!graph) return fail(ENC_ERR_INVALID_ARG, "null graph");
+  cudaError_t e = cudaGraphLaunch(graph->exec, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGraphLaunch");
+  graph->h->launches += 7 * graph->h->L;
+  return ok();
+}
+
+enc_status enc_graph_destroy(enc_graph_t graph) {
+  if (!graph) return ok();
+  cudaDeviceSynchronize();
+  if (graph->exec) cudaGraphExecDestroy(graph->exec);
+  if (graph->graph) cudaGraphDestroy(graph->graph);
+  if (graph->h) --graph->h->graphs_alive;
+  delete graph;
   return ok();
 }
 
@@ -523,6 +645,13 @@ enc_status enc_device_status(enc_t h, int32_t* code) {
 }
 
 int enc_kernels_per_forward(enc_t h) { return h ? 7 * h->L : 0; }
+
+enc_status enc_set_gelu(enc_t h, enc_gelu form) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  if (form != ENC_GELU_ERF && form != ENC_GELU_TANH) return fail(ENC_ERR_INVALID_ARG, "unknown GELU form %d", (int)form);
+  h->gelu = form;
+  return ok();
+}
 
 uint64_t enc_launch_count(enc_t h) { return h ? h->launches : 0; }
 

@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
       float v = acc[i][j];
       if constexpr (EPI != Epi::kStore) v += bias[n];
       if constexpr (EPI == Epi::kBiasGelu) v = 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+      if constexpr (EPI == Epi::kBiasGeluTanh)
+        v = 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)));
       if constexpr (EPI == Epi::kBiasQkvSplit) {
         const int H = sp.head_num * sp.size_per_head;
         const int t = n / H, rem = n - t * H;
@@ -91,6 +93,9 @@ cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K,
       break;
     case Epi::kBiasQkvSplit:
       gemm_f32_kernel<Epi::kBiasQkvSplit><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
+      break;
+    case Epi::kBiasGeluTanh:
+      gemm_f32_kernel<Epi::kBiasGeluTanh><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
       break;
   }
   return cudaGetLastError();

@@ -15,7 +15,7 @@
 //               four per 64-wide k-block) into one of two TMEM accumulators.
 //   warps 2..9  epilogue: two warps per TMEM lane quadrant (32 rows), each
 //               taking half of the tile's columns: tcgen05.ld, bias / GELU /
-//               head split, 16-byte stores to global memory.
+//               head split, TMA stores from a shared staging buffer.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i+1.  Every mbarrier wait is bounded (kWaitLimitNs); a wait that gives up
 // records kStatusWaitTimeout in the status word and the CTA drains its copies
@@ -37,38 +37,68 @@ using namespace sm100;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kEpiWarps = 8;
+// Epilogue warps: 8 (two per TMEM lane quadrant) measured faster than 16 on
+// every GEMM of the encoder (16 warps cap the registers at 96 per thread).
+#ifndef ENC_EPI_WARPS
+#define ENC_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = ENC_EPI_WARPS;     // 8 or 16: 2 or 4 warps per TMEM lane quadrant
+constexpr int kEpiSlices = kEpiWarps / 4;    // column slices of a tile
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 template <int BN>
 struct Cfg {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = BN == 256 ? 3 : 5;
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kBiasOffset = (kStages * kStageBytes + kNumBars * 8 + 16 + 15) / 16 * 16;
-  static constexpr int kSmem = 1024 + kBiasOffset + kEpiWarps * (BN / 2) * 4;
+  static constexpr int kStoreOffset = (kBiasOffset + kEpiWarps * (BN / kEpiSlices) * 4 + 1023) / 1024 * 1024;
+  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * (32 * 32 * 2);
 };
 
-// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), with erf from the rational
-// approximation of Hastings (Abramowitz & Stegun, Handbook of Mathematical
-// Functions, formula 7.1.26): for z >= 0,
-//   erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),  t = 1/(1 + p z),
-// |error| <= 1.5e-7, and erf(-z) = -erf(z).  One reciprocal and one exponential
-// per element keep the epilogue of the FFN1 GEMM off the critical path; the
-// error is far below the FP16 rounding of the stored result.
+// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), with erf from the
+// rational approximation of Abramowitz & Stegun, Handbook of Mathematical
+// Functions, formula 7.1.28: for z >= 0,
+//   erf(z) = 1 - 1 / (1 + a1 z + a2 z^2 + a3 z^3 + a4 z^4 + a5 z^5 + a6 z^6)^16,
+// |error| <= 3e-7, and erf(-z) = -erf(z).  The 16th power is four squarings, so
+// an element costs one reciprocal (special-function unit) and a dozen FMA-pipe
+// operations, which keeps the FFN1 epilogue behind its MMAs.  For large z the
+// power overflows to +inf and the reciprocal gives 0, i.e. erf = 1.  The error
+// is far below the FP16 rounding of the stored result.
 __device__ __forceinline__ float gelu_erf(float v) {
   const float z = fabsf(v) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-  float poly = fmaf(t, 1.061405429f, -1.453152027f);
-  poly = fmaf(t, poly, 1.421413741f);
-  poly = fmaf(t, poly, -0.284496736f);
-  poly = fmaf(t, poly, 0.254829592f);
-  poly *= t;
-  const float erf_abs = fmaf(-poly, __expf(-z * z), 1.0f);
-  return 0.5f * v * (1.0f + copysignf(erf_abs, v));
+  float q = fmaf(z, 0.0000430638f, 0.0002765672f);
+  q = fmaf(z, q, 0.0001520143f);
+  q = fmaf(z, q, 0.0092705272f);
+  q = fmaf(z, q, 0.0422820123f);
+  q = fmaf(z, q, 0.0705230784f);
+  q = fmaf(z, q, 1.0f);
+  q *= q;            // ^2
+  q *= q;            // ^4
+  q *= q;            // ^8
+  q *= q;            // ^16
+  float rq;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rq) : "f"(q));
+  const float erf_abs = 1.0f - rq;
+  const float hv = 0.5f * v;
+  return fmaf(hv, copysignf(erf_abs, v), hv);
+}
+
+// tanh form of GELU: 0.5 v (1 + tanh(u)), u = sqrt(2/pi) (v + 0.044715 v^3), with
+// tanh(u) = 1 - 2 / (exp(2u) + 1) (one exponential and one reciprocal on the
+// special-function unit; exp overflowing to +inf gives tanh = 1, underflowing
+// to 0 gives -1).
+__device__ __forceinline__ float gelu_tanh(float v) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(u * 2.8853900817779268f));   // exp(2u) = 2^(2u log2 e)
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(e + 1.0f));
+  const float th = fmaf(-2.0f, r, 1.0f);
+  const float hv = 0.5f * v;
+  return fmaf(hv, th, hv);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -105,12 +135,11 @@ __device__ __forceinline__ size_t col_offset(int col0, const SplitShape& sp) {
   }
 }
 
-// Epilogue for one thread: 32 accumulator columns of one row.  `bias_s` holds
-// the bias of these 32 columns (shared memory, read as a broadcast).
+// Epilogue math for one thread: 32 accumulator columns of one row -> 16 packed
+// half2 words.  `bias_s` holds the bias of these 32 columns (shared memory,
+// read as a broadcast).
 template <Epi EPI>
-__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], bool row_ok, int col0, int N,
-                                            const float* bias_s, __half* __restrict__ dst) {
-  if (!row_ok) return;
+__device__ __forceinline__ void epilogue_math(const uint32_t (&r)[32], const float* bias_s, uint32_t (&p)[16]) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -125,63 +154,117 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], bool row_ok
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
   }
+  if constexpr (EPI == Epi::kBiasGeluTanh) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    if (col0 + 8 * j < N) {
-      uint4 w;
-      w.x = pack_half2(v[8 * j + 0], v[8 * j + 1]);
-      w.y = pack_half2(v[8 * j + 2], v[8 * j + 3]);
-      w.z = pack_half2(v[8 * j + 4], v[8 * j + 5]);
-      w.w = pack_half2(v[8 * j + 6], v[8 * j + 7]);
-      *reinterpret_cast<uint4*>(dst + 8 * j) = w;
-    }
+    for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
   }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) p[i] = pack_half2(v[2 * i], v[2 * i + 1]);
 }
+
+// Bytes of one warp's staging buffer: a 32x32 FP16 chunk.
+constexpr int kStageChunkBytes = 32 * 32 * 2;
 
 // One epilogue warp's share of a tile: rows [32*quad, 32*quad+32) of the
 // accumulator (one row per lane), global columns [col_begin, col_begin +
 // 32*CHUNKS), whose first column sits at TMEM address t_cols (lane field
-// included).
+// included); `row0` is the global row of lane 0.
 // The bias of those columns is staged in the warp's shared-memory slot before
 // the accumulator is awaited; the TMEM load of chunk j+1 is in flight while
 // chunk j is converted and stored.  `release` runs once the last TMEM load of
 // the tile has completed (it frees the accumulator for the next tile).
+// Stores: with an output map (tm_c != nullptr) each 32x32 chunk is written to
+// the warp's staging buffer in the map's 64-byte swizzle and stored by a TMA
+// bulk copy (full lines, no per-lane stores); the buffer is reused once the
+// previous copy has read it.  Otherwise each lane stores its row with 16-byte
+// stores.
 template <Epi EPI, int CHUNKS, typename WaitFull, typename Release>
-__device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row, int col_begin, int M, int N,
+__device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, int col_begin, int M, int N,
                                                    const float* __restrict__ bias, float* bias_s,
                                                    __half* __restrict__ C, const SplitShape& sp,
+                                                   const CUtensorMap* tm_c, uint8_t* stage, uint32_t& store_seq,
                                                    WaitFull wait_full, Release release) {
   const int lane = threadIdx.x & 31;
   if constexpr (EPI != Epi::kStore) {
-    for (int i = lane * 4; i < 32 * CHUNKS; i += 128) {
+    for (int i = lane * 4; i < 32 * CHUNKS; i += 128) {   // CHUNKS <= 4
       float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
       if (col_begin + i < N) b = *reinterpret_cast<const float4*>(bias + col_begin + i);
       *reinterpret_cast<float4*>(bias_s + i) = b;
     }
   }
+  const int row = row0 + lane;
   const bool row_ok = row < M;
   const size_t roff = row_ok ? row_offset<EPI>(row, N, sp) : 0;
+  // Token coordinates of the chunk's first row for the head-split store map.
+  const int b0 = EPI == Epi::kBiasQkvSplit ? row0 / sp.seq : 0;
+  const int s0 = EPI == Epi::kBiasQkvSplit ? row0 - b0 * sp.seq : 0;
   int got = 0;
   if (lane == 0) got = wait_full() ? 1 : 0;
   got = __shfl_sync(0xffffffffu, got, 0);     // also orders the bias staging before its use
   if (!got) return false;
   sm100::tc_fence_after();
-  uint32_t ra[32], rb[32];
-  sm100::tmem_ld_32x32b_x32_async(t_cols, ra);
+  // With more than two chunks per warp the next chunk's TMEM load is issued
+  // before the current one is processed; with one or two, other warps hide it.
+  constexpr bool kPrefetch = CHUNKS > 2;
+  uint32_t ra[32], rb[kPrefetch ? 32 : 1];
+  if constexpr (kPrefetch) sm100::tmem_ld_32x32b_x32_async(t_cols, ra);
 #pragma unroll
   for (int j = 0; j < CHUNKS; ++j) {
-    uint32_t(&cur)[32] = (j & 1) ? rb : ra;
-    uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
-    sm100::tmem_wait_ld(cur);
-    if (j + 1 < CHUNKS) {
-      sm100::tmem_ld_32x32b_x32_async(t_cols + 32 * (j + 1), nxt);
+    uint32_t* cur_p;
+    if constexpr (kPrefetch) {
+      uint32_t(&cur)[32] = (j & 1) ? *reinterpret_cast<uint32_t(*)[32]>(rb) : ra;
+      uint32_t(&nxt)[32] = (j & 1) ? ra : *reinterpret_cast<uint32_t(*)[32]>(rb);
+      sm100::tmem_wait_ld(cur);
+      if (j + 1 < CHUNKS) sm100::tmem_ld_32x32b_x32_async(t_cols + 32 * (j + 1), nxt);
+      cur_p = cur;
     } else {
+      sm100::tmem_ld_32x32b_x32(t_cols + 32 * j, ra);
+      cur_p = ra;
+    }
+    if (j + 1 == CHUNKS) {
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) release();
     }
+    uint32_t(&cur)[32] = *reinterpret_cast<uint32_t(*)[32]>(cur_p);
     const int col0 = col_begin + 32 * j;
-    if (col0 < N) store_chunk<EPI>(cur, row_ok, col0, N, bias_s + 32 * j, C + roff + col_offset<EPI>(col0, sp));
+    if (col0 >= N) continue;
+    uint32_t p[16];
+    epilogue_math<EPI>(cur, bias_s + 32 * j, p);
+    if (tm_c != nullptr) {
+      uint8_t* buf = stage;
+      ++store_seq;
+      if (lane == 0) sm100::bulk_wait_group_read<0>();   // the previous store has read the buffer
+      __syncwarp();
+      // 64-byte swizzle: 16-byte unit u of row r sits at unit u ^ ((r >> 1) & 3).
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        *reinterpret_cast<uint4*>(buf + lane * 64 + 16 * (u ^ ((lane >> 1) & 3))) =
+            make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
+      }
+      sm100::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (EPI == Epi::kBiasQkvSplit) {
+          const int H = sp.head_num * sp.size_per_head;
+          const int t = col0 / H;
+          const int rem = col0 - t * H;
+          const int h = rem / sp.size_per_head;
+          const int c = rem - h * sp.size_per_head;
+          if (b0 < sp.batch) sm100::tma_store_5d(tm_c, sm100::smem_u32(buf), c, s0, h, b0, t);
+        } else {
+          sm100::tma_store_2d(tm_c, sm100::smem_u32(buf), col0, row0);
+        }
+        sm100::bulk_commit_group();
+      }
+    } else if (row_ok) {
+      __half* dst = C + roff + col_offset<EPI>(col0, sp);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (col0 + 8 * u < N)
+          *reinterpret_cast<uint4*>(dst + 8 * u) = make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
+      }
+    }
   }
   return true;
 }
@@ -189,8 +272,8 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row, int
 template <int BN, Epi EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   int M, int N, int K, const float* __restrict__ bias, __half* __restrict__ C,
-                   SplitShape sp, int* __restrict__ status) {
+                   const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M, int N, int K,
+                   const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp, int* __restrict__ status) {
   using G = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -199,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + G::kStages * G::kBBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::kNumBars);
   float* bias_smem = reinterpret_cast<float*>(smem + G::kBiasOffset);
+  uint8_t* store_smem = smem + G::kStoreOffset;
 
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -293,23 +377,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
-    const int half = (warp - 2) >> 2;          // which half of the tile's columns
-    constexpr int kChunks = BN / 64;           // 32-column chunks per warp
-    float* bias_s = bias_smem + (warp - 2) * (BN / 2);
+    const int slice = (warp - 2) >> 2;         // which column slice of the tile
+    constexpr int kCols = BN / kEpiSlices;
+    constexpr int kChunks = kCols / 32;        // 32-column chunks per warp
+    float* bias_s = bias_smem + (warp - 2) * kCols;
+    uint8_t* stage = store_smem + (warp - 2) * kStageChunkBytes;
+    const CUtensorMap* tmc = use_tma_store ? &tm_c : nullptr;
+    uint32_t store_seq = 0;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int m_blk = tile / num_n;
       const int n_blk = tile - m_blk * num_n;
       const uint32_t acc = local & 1u;
       const uint32_t aph = (local >> 1) & 1u;
-      const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + half * (BN / 2);
-      const int row = m_blk * kBM + quad * 32 + lane;
+      const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + slice * kCols;
+      const int row0 = m_blk * kBM + quad * 32;
       const bool got = epilogue_warp_tile<EPI, kChunks>(
-          t_cols, row, n_blk * BN + half * (BN / 2), M, N, bias, bias_s, C, sp,
+          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, stage, store_seq,
           [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); },
           [&] { mbar_arrive(tempty_bar(acc)); });
       if (!got) { ok = false; break; }
     }
+    if (lane == 0) bulk_wait_group_all();      // every TMA store of this warp has completed
+    __syncwarp();
   }
 
   if (!ok) atomicCAS(status, 0, kStatusWaitTimeout);
@@ -339,21 +429,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 //     accumulator-empty barrier (count 2 x kEpiWarps).
 // ---------------------------------------------------------------------------
 struct PairCfg {
-  static constexpr int kStages = 6;
+  static constexpr int kStages = 5;
   static constexpr int kABytes = 128 * kBK * 2;
   static constexpr int kBBytes = 128 * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;             // two 256-column accumulators
   static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kBiasOffset = (kStages * kStageBytes + kNumBars * 8 + 16 + 15) / 16 * 16;
-  static constexpr int kSmem = 1024 + kBiasOffset + kEpiWarps * 128 * 4;
+  static constexpr int kStoreOffset = (kBiasOffset + kEpiWarps * (256 / kEpiSlices) * 4 + 1023) / 1024 * 1024;
+  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * (32 * 32 * 2);
 };
 
 template <Epi EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        int M, int N, int K, const float* __restrict__ bias, __half* __restrict__ C,
-                        SplitShape sp, int* __restrict__ status) {
+                        const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M, int N, int K,
+                        const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp,
+                        int* __restrict__ status) {
   using G = PairCfg;
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -363,6 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + G::kStages * G::kBBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::kNumBars);
   float* bias_smem = reinterpret_cast<float*>(smem + G::kBiasOffset);
+  uint8_t* store_smem = smem + G::kStoreOffset;
 
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -466,9 +559,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
-    constexpr int kChunks = BN / 64;
-    float* bias_s = bias_smem + (warp - 2) * (BN / 2);
+    const int slice = (warp - 2) >> 2;
+    constexpr int kCols = BN / kEpiSlices;
+    constexpr int kChunks = kCols / 32;
+    float* bias_s = bias_smem + (warp - 2) * kCols;
+    uint8_t* stage = store_smem + (warp - 2) * kStageChunkBytes;
+    const CUtensorMap* tmc = use_tma_store ? &tm_c : nullptr;
+    uint32_t store_seq = 0;
     const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
     const uint32_t leader_tempty1 = mapa_shared(tempty_bar(1), 0);
     uint32_t local = 0;
@@ -477,14 +574,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int n_blk = tile - m_blk * num_n;
       const uint32_t acc = local & 1u;
       const uint32_t aph = (local >> 1) & 1u;
-      const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + half * (BN / 2);
-      const int row = m_blk * 256 + (int)rank * 128 + quad * 32 + lane;
+      const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + slice * kCols;
+      const int row0 = m_blk * 256 + (int)rank * 128 + quad * 32;
       const bool got = epilogue_warp_tile<EPI, kChunks>(
-          t_cols, row, n_blk * BN + half * (BN / 2), M, N, bias, bias_s, C, sp,
+          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, stage, store_seq,
           [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); },
           [&] { mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0); });
       if (!got) { ok = false; break; }
     }
+    if (lane == 0) bulk_wait_group_all();      // every TMA store of this warp has completed
+    __syncwarp();
   }
 
   if (!ok) atomicCAS(status, 0, kStatusWaitTimeout);
@@ -527,8 +626,9 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   if (max_clusters <= 0) return cudaErrorInvalidConfiguration;
   const int tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
-  gemm_tc_pair_kernel<EPI><<<2 * pairs, kThreads, G::kSmem, stream>>>(*a.tmap_a, *a.tmap_b, a.M, a.N, a.K,
-                                                                      a.bias, a.c, a.split, a.status);
+  gemm_tc_pair_kernel<EPI><<<2 * pairs, kThreads, G::kSmem, stream>>>(
+      *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c, a.split,
+      a.status);
   return cudaGetLastError();
 }
 
@@ -544,8 +644,9 @@ cudaError_t launch_impl(const TcGemmArgs& a, cudaStream_t stream) {
   if (attr_err != cudaSuccess) return attr_err;
   const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + BN - 1) / BN);
   const int grid = tiles < a.num_sms ? tiles : a.num_sms;
-  gemm_tc_kernel<BN, EPI><<<grid, kThreads, G::kSmem, stream>>>(*a.tmap_a, *a.tmap_b, a.M, a.N, a.K,
-                                                               a.bias, a.c, a.split, a.status);
+  gemm_tc_kernel<BN, EPI><<<grid, kThreads, G::kSmem, stream>>>(
+      *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c, a.split,
+      a.status);
   return cudaGetLastError();
 }
 
@@ -555,6 +656,7 @@ cudaError_t launch_bn(const TcGemmArgs& a, cudaStream_t stream) {
     case Epi::kStore: return launch_impl<BN, Epi::kStore>(a, stream);
     case Epi::kBiasGelu: return launch_impl<BN, Epi::kBiasGelu>(a, stream);
     case Epi::kBiasQkvSplit: return launch_impl<BN, Epi::kBiasQkvSplit>(a, stream);
+    case Epi::kBiasGeluTanh: return launch_impl<BN, Epi::kBiasGeluTanh>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -589,15 +691,43 @@ bool encode_kmajor_fp16_map(CUtensorMap* map, const void* base, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
+bool encode_output_map_2d(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool encode_output_map_split(CUtensorMap* map, void* base, const SplitShape& sp) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const uint64_t d = sp.size_per_head, S = sp.seq, nh = sp.head_num, B = sp.batch;
+  const cuuint64_t dims[5] = {d, S, nh, B, 3};
+  const cuuint64_t strides[4] = {d * 2, S * d * 2, nh * S * d * 2, B * nh * S * d * 2};
+  const cuuint32_t box[5] = {32, 32, 1, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0 || (a.N % 8) != 0 || (a.K % 8) != 0) return cudaErrorInvalidValue;
   if (a.epi == Epi::kBiasQkvSplit && (a.split.size_per_head % 32) != 0) return cudaErrorInvalidValue;
+  // The head-split store map needs every 32-row chunk inside one sequence.
+  if (a.epi == Epi::kBiasQkvSplit && a.tmap_c && (a.split.seq % 32) != 0) return cudaErrorInvalidValue;
   if (a.bn == kPairTile) {
     if ((a.N % 256) != 0) return cudaErrorInvalidValue;
     switch (a.epi) {
       case Epi::kStore: return launch_pair<Epi::kStore>(a, stream);
       case Epi::kBiasGelu: return launch_pair<Epi::kBiasGelu>(a, stream);
       case Epi::kBiasQkvSplit: return launch_pair<Epi::kBiasQkvSplit>(a, stream);
+      case Epi::kBiasGeluTanh: return launch_pair<Epi::kBiasGeluTanh>(a, stream);
     }
     return cudaErrorInvalidValue;
   }

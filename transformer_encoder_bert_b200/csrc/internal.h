@@ -16,7 +16,8 @@ constexpr float kLnEps = 1e-12f;   // LayerNorm epsilon (the original BERT value
 enum class Epi : int {
   kStore = 0,        // C[m][n] = acc
   kBiasGelu = 1,     // C[m][n] = GELU(acc + bias[n]), erf form
-  kBiasQkvSplit = 2  // Q/K/V head split: dst[t][b][h][s][c] = acc + bias[n]
+  kBiasQkvSplit = 2, // Q/K/V head split: dst[t][b][h][s][c] = acc + bias[n]
+  kBiasGeluTanh = 3  // C[m][n] = GELU_tanh(acc + bias[n])
 };
 
 // Addressing for the head-split epilogue (n = t*H + h*d + c, m = b*seq + s).
@@ -35,6 +36,8 @@ constexpr int kPairTile = 2;
 struct TcGemmArgs {
   const CUtensorMap* tmap_a;   // dims {K, M}, box {64, 128}, 128B swizzle
   const CUtensorMap* tmap_b;   // dims {K, N}, box {64, bn} (128 rows for kPairTile), 128B swizzle
+  const CUtensorMap* tmap_c;   // output map with a 32x32 box, 64B swizzle, or nullptr (direct stores):
+                               // C [M, N] as dims {N, M}; the head split as dims {d, seq, heads, batch, 3}
   int M, N, K;
   int bn;                      // 128, 256 or kPairTile
   Epi epi;
@@ -49,6 +52,9 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream);
 // Encode a 2-D K-major FP16 tensor map over [rows, cols=K] with a {64, box_rows} box.
 bool encode_kmajor_fp16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                             uint32_t box_rows);
+// Output maps for the GEMM epilogue's TMA stores (32x32 boxes, 64-byte swizzle).
+bool encode_output_map_2d(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols);
+bool encode_output_map_split(CUtensorMap* map, void* base, const SplitShape& sp);
 
 // ---- FP32 SIMT GEMM (FP32 mode, no TF32), gemm_f32.cu ----
 // C = A[M,K] * W[K,N] (W row-major [K,N]).
@@ -67,6 +73,10 @@ cudaError_t launch_attention_f32(const float* qkv, const int32_t* valid_len, flo
 cudaError_t launch_bias_residual_ln_f16(const __half* a, const float* bias, const __half* resid,
                                         const float* gamma, const float* beta, __half* out,
                                         int rows, int hidden, cudaStream_t stream);
+// FP16 rows with FP16 parameters (hidden <= 1024): one row per warp.
+cudaError_t launch_bias_residual_ln_f16h(const __half* a, const __half* bias, const __half* resid,
+                                         const __half* gamma, const __half* beta, __half* out,
+                                         int rows, int hidden, cudaStream_t stream);
 cudaError_t launch_bias_residual_ln_f32(const float* a, const float* bias, const float* resid,
                                         const float* gamma, const float* beta, float* out,
                                         int rows, int hidden, cudaStream_t stream);
