@@ -65,10 +65,14 @@ def blas_threads() -> int:
 
 
 # ------------------------------------------------------------------ algorithmic work per kernel
-def kernel_work(wl: EI.Workload):
-    """Per launch: (flops, algorithmic HBM bytes) of each kernel of one layer (FP16 storage)."""
+def kernel_work(wl: EI.Workload, attn_seq=None, attn_tokens=None):
+    """Per launch: (flops, algorithmic HBM bytes) of each kernel of one layer (FP16 storage).
+    Attention flops are 4*S*H per token over the padded length (dense mode) or per
+    valid token (attn_seq, attn_tokens for the packed mode, an upper bound)."""
     sh = wl.shape
     H, F, M, S = sh.hidden, sh.ffn_dim, wl.tokens, wl.seq
+    if attn_seq is not None:
+        S = attn_seq
     es = 2 if wl.dtype == "fp16" else 4
     def gemm(n, k, extra_out=0):
         return 2.0 * M * n * k, es * (M * k + k * n + M * n) + extra_out
@@ -183,6 +187,29 @@ def run_reference(args, wl: EI.Workload, rank: int, world: int):
     return 0
 
 
+# ------------------------------------------------------------------ replicas (N > 1)
+def replica_workload(wl: EI.Workload, rank: int) -> EI.Workload:
+    """Each rank runs its own batch of the same workload (weak scaling): seed + rank."""
+    return wl.with_(seed=wl.seed + rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks of the default process
+    group (identity without one).  The job's time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(batch_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Sequences per second of the whole job: every rank's batch in the slowest rank's time."""
+    return batch_per_rank * world / (ms_per_step * 1e-3)
+
+
 def workload_config(wl: EI.Workload, world: int, l2: str):
     sh = wl.shape
     return {"workload": wl.name, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
@@ -200,10 +227,12 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = wl.with_(seed=wl.seed + rank)          # each replica has its own batch
+    wl = replica_workload(wl, rank)             # each replica has its own batch
     inp = EI.make_inputs(wl)
     sh = wl.shape
     enc = Encoder(sh.head_num, sh.size_per_head, sh.ffn_dim, inp.layers, wl.dtype)
+    if args.packed:
+        enc.set_packing(True)
     enc.reserve(wl.batch, wl.seq)
     x = torch.from_numpy(inp.x).to(dev)
     vl = torch.from_numpy(inp.valid_len).to(dev)
@@ -258,10 +287,12 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
 
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
-    per_kernel = {k: [] for k in KERNEL_NAMES}
+    names = (["offsets", "pack"] + KERNEL_NAMES * sh.num_layers + ["unpack"]) if args.packed \
+        else KERNEL_NAMES * sh.num_layers
+    per_kernel = {k: [] for k in names}
     for evs in ev_sets:
         for j in range(nk):
-            per_kernel[KERNEL_NAMES[j % 7]].append(evs[j].elapsed_time(evs[j + 1]))
+            per_kernel[names[j]].append(evs[j].elapsed_time(evs[j + 1]))
 
     # e2e through enc_forward_host: pinned host input, copies inside the timed region.
     hx = torch.from_numpy(inp.x).pin_memory()
@@ -285,18 +316,21 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     if graph is not None:
         graph.close()
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_step = float(t[0]), float(t[1])
+    ms, e2e_step = max_over_ranks([ms, e2e_step], device=dev)
     if rank != 0:
         return 0
 
     peaks, peak_src = load_peaks()
     work = kernel_work(wl)
+    if args.packed:
+        # valid tokens only: the algorithmic work of the packed path
+        t_valid = int(np.clip(inp.valid_len, 0, wl.seq).sum())
+        work = kernel_work(wl.with_(batch=1, seq=t_valid), attn_seq=wl.seq, attn_tokens=t_valid)
+        work.update({"offsets": (0.0, 8.0 * wl.batch), "pack": (0.0, 4.0 * t_valid * sh.hidden),
+                     "unpack": (0.0, 4.0 * t_valid * sh.hidden)})
     kernels = {}
     total = sum(sum(v) for v in per_kernel.values())
-    for k in KERNEL_NAMES:
+    for k in per_kernel:
         vals = per_kernel[k]
         avg_ms = sum(vals) / len(vals)
         flops, nbytes = work[k]
@@ -305,7 +339,7 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
             entry["tflops"] = flops / (avg_ms * 1e-3) / 1e12
         entry["gbs"] = nbytes / (avg_ms * 1e-3) / 1e9
         kernels[k] = entry
-    dominant = max(KERNEL_NAMES, key=lambda k: kernels[k]["share"])
+    dominant = max(kernels, key=lambda k: kernels[k]["share"])
     d = kernels[dominant]
     if dominant.endswith("gemm"):
         peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -319,15 +353,17 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
                 "traffic": args.traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
                 "peak_source": f"{peak_src} HBM copy bandwidth"}
 
-    value = wl.batch * world / (ms * 1e-3)
+    value = job_throughput(wl.batch, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16" if wl.dtype == "fp16" else "fp32", "data": "synthetic",
         "config": dict(workload_config(wl, world, l2="flushed before every timed step (256 MiB write)"),
-                       launch="one recorded CUDA graph per step" if args.graph else "enc_forward per step"),
+                       launch="one recorded CUDA graph per step" if args.graph else "enc_forward per step",
+                       padding="removed (valid tokens only; padded outputs zero)" if args.packed
+                       else "computed (fixed length)"),
         "roofline": roof,
-        "e2e": {"value": wl.batch * world / (e2e_step * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_throughput(wl.batch, world, e2e_step), "unit": UNIT,
                 "h2d_bytes_per_step": int(hx.numel() * hx.element_size() + hvl.numel() * 4),
                 "d2h_bytes_per_step": int(hout.numel() * hout.element_size())},
         "gpu_launches": int(launches),
@@ -352,6 +388,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--packed", action="store_true",
+                    help="padding removal (enc_set_packing): compute the valid tokens only")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of a recorded forward (enc_graph_launch) instead of enc_forward calls")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")

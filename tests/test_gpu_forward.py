@@ -218,3 +218,65 @@ def test_recorded_forward_replays_bit_exact():
     g.close()
     enc.forward(big, to_dev(np.full(64, 32, np.int32)))
     assert enc.device_status() == 0
+
+
+def test_host_entry_point_chunked_pipeline_matches_device_forward():
+    # 256 x 32 tokens: enc_forward_host cuts the batch into 4 chunks with overlapped copies.
+    import torch
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 256))
+    enc = encoder_from_inputs(inp)
+    dev = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    hx = torch.from_numpy(inp.x).pin_memory()
+    hvl = torch.from_numpy(inp.valid_len).pin_memory()
+    hout = torch.empty_like(hx).pin_memory()
+    enc.forward_host_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), 256, 32)
+    assert np.array_equal(hout.numpy(), dev)
+    pageable = enc.forward_host(inp.x, inp.valid_len)
+    assert np.array_equal(pageable, dev)
+
+
+# ---------------------------------------------------------------- padding removal
+
+@pytest.mark.parametrize("seq,lo,hi,L", [(32, 1, 32, 12), (37, 0, 37, 2), (96, 64, 96, 2), (128, 64, 128, 2),
+                                         (512, 256, 512, 1)])
+def test_packed_forward_matches_oracle_and_zeroes_padding(seq, lo, hi, L):
+    sh = EI.EncoderShape(12, 64, 3072, L)
+    inp = EI.make_inputs(EI.Workload("packed", sh, 6, seq, "fp16", lo, hi, seed=seq + L))
+    if lo == 0:
+        inp.valid_len[1] = 0                      # an empty sequence in the middle of the batch
+    enc = encoder_from_inputs(inp)
+    dense = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    enc.set_packing(True)
+    assert enc.kernels_per_forward() == 7 * L + 3
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    m = valid_mask(inp.valid_len, seq)
+    assert np.all(got[~m] == 0)
+    tol = FP16_STACK_REL_L2 if L > 2 else L * FP16_LAYER_REL_L2
+    _check(got, _oracle(inp), inp.valid_len, seq, tol)
+    assert rel_l2(got, dense, m) < tol
+    assert enc.device_status() == 0
+
+
+def test_packed_mode_replays_and_host_entry_point():
+    import torch
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 128))
+    enc = encoder_from_inputs(inp)
+    enc.set_packing(True)
+    x, vl = to_dev(inp.x), to_dev(inp.valid_len)
+    ref = to_host(enc.forward(x, vl))
+    out = torch.empty_like(x)
+    g = enc.record(x, vl, out)
+    g.launch()
+    torch.cuda.synchronize()
+    assert np.array_equal(to_host(out), ref)
+    g.close()
+    assert np.array_equal(enc.forward_host(inp.x, inp.valid_len), ref)
+
+
+def test_packed_mode_needs_fp16():
+    from transformer_encoder_bert_b200 import EncError
+    inp = EI.make_inputs(EI.named_workload("tiny-fp32", 1))
+    enc = encoder_from_inputs(inp)
+    with pytest.raises(EncError) as e:
+        enc.set_packing(True)
+    assert e.value.status == 2

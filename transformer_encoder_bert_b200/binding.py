@@ -36,6 +36,8 @@ SIGNATURES = {
     "enc_last_error": (ctypes.c_char_p, []),
     "enc_device_status": (_i, [_vp, ctypes.POINTER(ctypes.c_int32)]),
     "enc_set_gelu": (_i, [_vp, _i]),
+    "enc_set_packing": (_i, [_vp, _i]),
+    "enc_set_host_chunks": (_i, [_vp, _i]),
     "enc_graph_create": (_i, [_vp, _vp, _vp, _vp, _i, _i, ctypes.POINTER(_vp)]),
     "enc_graph_launch": (_i, [_vp, _vp]),
     "enc_graph_destroy": (_i, [_vp]),
@@ -156,6 +158,13 @@ class Encoder:
     def set_gelu(self, form: str):
         """"erf" (default) or "tanh"."""
         _check(self.lib.enc_set_gelu(self.handle, {"erf": 0, "tanh": 1}[form]))
+
+    def set_packing(self, enable: bool):
+        """Padding removal: compute valid tokens only; padded output rows become zeros."""
+        _check(self.lib.enc_set_packing(self.handle, 1 if enable else 0))
+
+    def set_host_chunks(self, chunks: int):
+        _check(self.lib.enc_set_host_chunks(self.handle, chunks))
 
     def reserve(self, batch: int, seq: int):
         _check(self.lib.enc_reserve(self.handle, batch, seq))

@@ -99,10 +99,16 @@ struct enc_handle {
   size_t ws_bytes = 0;
   void* stage = nullptr;            // enc_forward_host device staging
   size_t stage_bytes = 0;
+  cudaStream_t copy_in = nullptr;   // enc_forward_host: host-to-device copies
+  cudaStream_t copy_out = nullptr;  // enc_forward_host: device-to-host copies
+  static constexpr int kMaxChunks = 4;
+  cudaEvent_t ev_in[kMaxChunks] = {}, ev_done[kMaxChunks] = {}, ev_out = nullptr, ev_start = nullptr;
   int* status = nullptr;
   uint64_t launches = 0;            // kernels launched through this handle
   int graphs_alive = 0;             // recorded forwards that reference the workspace
   enc_gelu gelu = ENC_GELU_ERF;
+  bool packed = false;              // padding removal (enc_set_packing)
+  int host_chunks = 1;              // enc_forward_host: most chunks the batch is cut into (see enc.h)
   bool no_pair = false;             // ENC_GEMM_NO_PAIR=1: one-CTA tiles only (comparison runs)
   bool no_tma_store = false;        // ENC_GEMM_NO_TMA_STORE=1: epilogue stores without TMA
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
@@ -112,13 +118,14 @@ namespace {
 
 struct Workspace {
   void *qkv, *ctx, *a, *h1, *u, *x0, *x1;
+  int32_t* offsets;   // packed mode: [batch + 1] token offsets of the sequences
 };
 
 size_t workspace_bytes(const enc_handle* h, size_t tokens) {
   const size_t es = h->esize;
   const size_t mh = align_up(tokens * h->H * es, 256);
   const size_t mf = align_up(tokens * h->F * es, 256);
-  return 3 * mh + mh + mh + mh + mf + 2 * mh;
+  return 3 * mh + mh + mh + mh + mf + 2 * mh + align_up((tokens + 1) * 4, 256);
 }
 
 Workspace carve(const enc_handle* h, size_t tokens) {
@@ -133,7 +140,8 @@ Workspace carve(const enc_handle* h, size_t tokens) {
   w.h1 = p; p += mh;
   w.u = p; p += mf;
   w.x0 = p; p += mh;
-  w.x1 = p;
+  w.x1 = p; p += mh;
+  w.offsets = reinterpret_cast<int32_t*>(p);
   return w;
 }
 
@@ -179,7 +187,8 @@ int choose_bn(const enc_handle* h, int M, int N) {
 
 // One GEMM step: C = A * W (+ epilogue), dispatched on the handle's dtype.
 enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const CUtensorMap* wmaps, int N,
-                    enc::Epi epi, const float* bias, void* C, enc::SplitShape sp, cudaStream_t st) {
+                    enc::Epi epi, const float* bias, void* C, enc::SplitShape sp, cudaStream_t st,
+                    const int* m_dev = nullptr) {
   if (h->dtype == ENC_FP16) {
     const int bn = choose_bn(h, M, N);
     CUtensorMap ta;
@@ -204,6 +213,7 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
     a.split = sp;
     a.status = h->status;
     a.num_sms = h->num_sms;
+    a.m_dev = m_dev;
     cudaError_t e = enc::launch_gemm_tc(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
     ++h->launches;
@@ -296,6 +306,14 @@ enc_status check_ptrs(std::initializer_list<const void*> ps) {
 
 void free_handle(enc_handle* h) {
   if (!h) return;
+  for (int i = 0; i < enc_handle::kMaxChunks; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_done[i]) cudaEventDestroy(h->ev_done[i]);
+  }
+  if (h->ev_out) cudaEventDestroy(h->ev_out);
+  if (h->ev_start) cudaEventDestroy(h->ev_start);
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
   if (h->param_block) cudaFree(h->param_block);
   if (h->ws) cudaFree(h->ws);
   if (h->stage) cudaFree(h->stage);
@@ -467,6 +485,72 @@ enc_status enc_reserve(enc_t h, int batch, int seq) {
 
 namespace {
 
+// Padding removal: offsets <- prefix sum of the valid lengths (T = offsets[batch]
+// on the device); the valid tokens are packed into [T, H]; every layer runs on
+// T rows (GEMMs and LayerNorms read T from the device, attention walks each
+// sequence through its offset); the last layer's rows are scattered back into
+// out, with zeros in the padded positions.  Kernels: 2 + 7 per layer + 1.
+template <typename Mark>
+enc_status forward_packed(enc_handle* h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                          cudaStream_t st, const Workspace& w, Mark& mark) {
+  const int M = batch * seq;                 // most rows any step can hold
+  const int H = h->H;
+  const int* T = w.offsets + batch;
+  cudaError_t e;
+  mark();
+  e = enc::launch_valid_offsets(valid_len, batch, seq, w.offsets, st);
+  if (e != cudaSuccess) return cuda_fail(e, "offsets launch");
+  ++h->launches;
+  mark();
+  e = enc::launch_pack_rows(static_cast<const __half*>(x), valid_len, w.offsets, static_cast<__half*>(w.x1), batch,
+                            seq, H, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  ++h->launches;
+  enc_status s;
+  void* last = nullptr;
+  for (int l = 0; l < h->L; ++l) {
+    LayerDev& L = h->layers[l];
+    void* xin = l == 0 ? w.x1 : (((l - 1) & 1) ? w.x1 : w.x0);
+    void* xout = (l & 1) ? w.x1 : w.x0;
+    mark();
+    if ((s = run_gemm(h, xin, M, H, L.w_qkv, L.tm_qkv, 3 * H, enc::Epi::kBiasStore, L.b_qkv, w.qkv, {}, st, T)) !=
+        ENC_OK)
+      return s;
+    mark();
+    e = enc::launch_attention_f16_packed(static_cast<const __half*>(w.qkv), valid_len, w.offsets,
+                                         static_cast<__half*>(w.ctx), batch, seq, h->nh, h->d, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    ++h->launches;
+    mark();
+    if ((s = run_gemm(h, w.ctx, M, H, L.w_o, L.tm_o, H, enc::Epi::kStore, nullptr, w.a, {}, st, T)) != ENC_OK)
+      return s;
+    mark();
+    e = enc::launch_bias_residual_ln_f16h(static_cast<const __half*>(w.a), L.h_b_o, static_cast<const __half*>(xin),
+                                          L.h_ln1_g, L.h_ln1_b, static_cast<__half*>(w.h1), M, H, st, T);
+    if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
+    ++h->launches;
+    mark();
+    const enc::Epi gelu = h->gelu == ENC_GELU_TANH ? enc::Epi::kBiasGeluTanh : enc::Epi::kBiasGelu;
+    if ((s = run_gemm(h, w.h1, M, H, L.w_ff1, L.tm_ff1, h->F, gelu, L.b_ff1, w.u, {}, st, T)) != ENC_OK) return s;
+    mark();
+    if ((s = run_gemm(h, w.u, M, h->F, L.w_ff2, L.tm_ff2, H, enc::Epi::kStore, nullptr, w.a, {}, st, T)) != ENC_OK)
+      return s;
+    mark();
+    e = enc::launch_bias_residual_ln_f16h(static_cast<const __half*>(w.a), L.h_b_ff2, static_cast<const __half*>(w.h1),
+                                          L.h_ln2_g, L.h_ln2_b, static_cast<__half*>(xout), M, H, st, T);
+    if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
+    ++h->launches;
+    last = xout;
+  }
+  mark();
+  e = enc::launch_unpack_rows(static_cast<const __half*>(last), valid_len, w.offsets, static_cast<__half*>(out), batch,
+                              seq, H, st);
+  if (e != cudaSuccess) return cuda_fail(e, "unpack launch");
+  ++h->launches;
+  mark();
+  return ENC_OK;
+}
+
 // Checks, workspace, and the per-layer launches of one forward on `st`.
 enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
                         cudaStream_t st, bool tracing) {
@@ -488,6 +572,7 @@ enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, 
   auto mark = [&]() {
     if (tracing) cudaEventRecord(h->trace[k++], st);
   };
+  if (h->packed) return forward_packed(h, x, valid_len, out, batch, seq, st, w, mark);
   for (int l = 0; l < h->L; ++l) {
     const void* xin = l == 0 ? x : (((l - 1) & 1) ? w.x1 : w.x0);
     void* xout = l == h->L - 1 ? out : ((l & 1) ? w.x1 : w.x0);
@@ -572,7 +657,7 @@ enc_status enc_graph_launch(enc_graph_t graph, enc_stream_t stream) {
   if (!graph) return fail(ENC_ERR_INVALID_ARG, "null graph");
   cudaError_t e = cudaGraphLaunch(graph->exec, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaGraphLaunch");
-  graph->h->launches += 7 * graph->h->L;
+  graph->h->launches += enc_kernels_per_forward(graph->h);
   return ok();
 }
 
@@ -592,7 +677,8 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
   if (s != ENC_OK) return s;
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if (!x || !valid_len || !out) return fail(ENC_ERR_INVALID_ARG, "null host buffer");
-  const size_t act = (size_t)batch * seq * h->H * h->esize;
+  const size_t seq_bytes = (size_t)seq * h->H * h->esize;
+  const size_t act = (size_t)batch * seq_bytes;
   const size_t act_al = align_up(act, 256);
   const size_t need = 2 * act_al + align_up((size_t)batch * 4, 256);
   if (need > h->stage_bytes) {
@@ -608,16 +694,53 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
     }
     h->stage_bytes = need;
   }
+  if (!h->copy_in) {
+    cudaError_t e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
+    for (int i = 0; i < enc_handle::kMaxChunks && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "copy stream setup");
+  }
+  // Sequences are independent, so the batch is cut into up to kMaxChunks chunks
+  // of at least 2048 tokens: chunk i+1 is copied in and chunk i-1 copied out
+  // while chunk i runs, so the copies hide behind the encoder.
+  const long tokens = (long)batch * seq;
+  int chunks = (int)std::min<long>(h->host_chunks, std::max<long>(1, tokens / 2048));
+  chunks = std::min(chunks, batch);
   char* base = static_cast<char*>(h->stage);
-  void* dx = base;
-  void* dout = base + act_al;
+  char* dx = base;
+  char* dout = base + act_al;
   int32_t* dvl = reinterpret_cast<int32_t*>(base + 2 * act_al);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemcpyAsync(dx, x, act, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dvl, valid_len, (size_t)batch * 4, cudaMemcpyHostToDevice, st);
+  const char* hx = static_cast<const char*>(x);
+  char* hout = static_cast<char*>(out);
+  // Copies start after the caller's earlier work on `st` (the staging buffers may be in use).
+  cudaError_t e = cudaEventRecord(h->ev_start, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_in, h->ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_start, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dvl, valid_len, (size_t)batch * 4, cudaMemcpyHostToDevice, h->copy_in);
   if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-  if ((s = enc_forward(h, dx, dvl, dout, batch, seq, stream)) != ENC_OK) return s;
-  e = cudaMemcpyAsync(out, dout, act, cudaMemcpyDeviceToHost, st);
+  int b0 = 0;
+  for (int c = 0; c < chunks; ++c) {
+    const int nb = batch / chunks + (c < batch % chunks ? 1 : 0);
+    const size_t off = (size_t)b0 * seq_bytes, bytes = (size_t)nb * seq_bytes;
+    e = cudaMemcpyAsync(dx + off, hx + off, bytes, cudaMemcpyHostToDevice, h->copy_in);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_in[c], h->copy_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->ev_in[c], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    if ((s = forward_impl(h, dx + off, dvl + b0, dout + off, nb, seq, st, false)) != ENC_OK) return s;
+    e = cudaEventRecord(h->ev_done[c], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_done[c], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(hout + off, dout + off, bytes, cudaMemcpyDeviceToHost, h->copy_out);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    b0 += nb;
+  }
+  e = cudaEventRecord(h->ev_out, h->copy_out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->ev_out, 0);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
   return ok();
@@ -644,7 +767,23 @@ enc_status enc_device_status(enc_t h, int32_t* code) {
   return ok();
 }
 
-int enc_kernels_per_forward(enc_t h) { return h ? 7 * h->L : 0; }
+int enc_kernels_per_forward(enc_t h) { return h ? 7 * h->L + (h->packed ? 3 : 0) : 0; }
+
+enc_status enc_set_packing(enc_t h, int enable) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  if (enable && (h->dtype != ENC_FP16 || h->H > 1024))
+    return fail(ENC_ERR_UNSUPPORTED, "padding removal needs FP16 mode and hidden size <= 1024");
+  h->packed = enable != 0;
+  return ok();
+}
+
+enc_status enc_set_host_chunks(enc_t h, int chunks) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  if (chunks < 1 || chunks > enc_handle::kMaxChunks)
+    return fail(ENC_ERR_INVALID_ARG, "chunks must be in [1, %d]", enc_handle::kMaxChunks);
+  h->host_chunks = chunks;
+  return ok();
+}
 
 enc_status enc_set_gelu(enc_t h, enc_gelu form) {
   if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");

@@ -97,6 +97,9 @@ cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K,
     case Epi::kBiasGeluTanh:
       gemm_f32_kernel<Epi::kBiasGeluTanh><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
       break;
+    case Epi::kBiasStore:
+      gemm_f32_kernel<Epi::kBiasStore><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
+      break;
   }
   return cudaGetLastError();
 }

@@ -68,23 +68,53 @@ struct Cfg {
 // operations, which keeps the FFN1 epilogue behind its MMAs.  For large z the
 // power overflows to +inf and the reciprocal gives 0, i.e. erf = 1.  The error
 // is far below the FP16 rounding of the stored result.
-__device__ __forceinline__ float gelu_erf(float v) {
-  const float z = fabsf(v) * 0.70710678118654752f;
-  float q = fmaf(z, 0.0000430638f, 0.0002765672f);
-  q = fmaf(z, q, 0.0001520143f);
-  q = fmaf(z, q, 0.0092705272f);
-  q = fmaf(z, q, 0.0422820123f);
-  q = fmaf(z, q, 0.0705230784f);
-  q = fmaf(z, q, 1.0f);
-  q *= q;            // ^2
-  q *= q;            // ^4
-  q *= q;            // ^8
-  q *= q;            // ^16
-  float rq;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rq) : "f"(q));
-  const float erf_abs = 1.0f - rq;
-  const float hv = 0.5f * v;
-  return fmaf(hv, copysignf(erf_abs, v), hv);
+// Two elements are evaluated at once with the packed FP32 instructions of
+// sm_100 (fma/mul .f32x2): the polynomial, the squarings and the final
+// scaling cost one instruction per pair; the reciprocal and the sign stay per
+// element.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ void gelu_erf_pair(float& v0, float& v1) {
+  const uint64_t v = f2_pack(v0, v1);
+  const uint64_t z = f2_mul(f2_pack(fabsf(v0), fabsf(v1)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
+  uint64_t q = f2_fma(z, f2_pack(0.0000430638f, 0.0000430638f), f2_pack(0.0002765672f, 0.0002765672f));
+  q = f2_fma(z, q, f2_pack(0.0001520143f, 0.0001520143f));
+  q = f2_fma(z, q, f2_pack(0.0092705272f, 0.0092705272f));
+  q = f2_fma(z, q, f2_pack(0.0422820123f, 0.0422820123f));
+  q = f2_fma(z, q, f2_pack(0.0705230784f, 0.0705230784f));
+  q = f2_fma(z, q, f2_pack(1.0f, 1.0f));
+  q = f2_mul(q, q);
+  q = f2_mul(q, q);
+  q = f2_mul(q, q);
+  q = f2_mul(q, q);
+  float q0, q1, r0, r1;
+  f2_unpack(q, q0, q1);
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(q0));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(q1));
+  // erf(|z|) = 1 - r >= 0; give it the sign of v
+  const uint64_t e = f2_fma(f2_pack(r0, r1), f2_pack(-1.0f, -1.0f), f2_pack(1.0f, 1.0f));
+  float e0, e1;
+  f2_unpack(e, e0, e1);
+  e0 = copysignf(e0, v0);
+  e1 = copysignf(e1, v1);
+  const uint64_t hv = f2_mul(v, f2_pack(0.5f, 0.5f));
+  f2_unpack(f2_fma(hv, f2_pack(e0, e1), hv), v0, v1);
 }
 
 // tanh form of GELU: 0.5 v (1 + tanh(u)), u = sqrt(2/pi) (v + 0.044715 v^3), with
@@ -152,7 +182,7 @@ __device__ __forceinline__ void epilogue_math(const uint32_t (&r)[32], const flo
   }
   if constexpr (EPI == Epi::kBiasGelu) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+    for (int i = 0; i < 32; i += 2) gelu_erf_pair(v[i], v[i + 1]);
   }
   if constexpr (EPI == Epi::kBiasGeluTanh) {
 #pragma unroll
@@ -272,8 +302,10 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
 template <int BN, Epi EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M, int N, int K,
-                   const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp, int* __restrict__ status) {
+                   const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M_max, int N, int K,
+                   const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp, int* __restrict__ status,
+                   const int* __restrict__ m_dev) {
+  const int M = m_dev ? min(*m_dev, M_max) : M_max;
   using G = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -443,9 +475,10 @@ struct PairCfg {
 template <Epi EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M, int N, int K,
+                        const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M_max, int N, int K,
                         const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp,
-                        int* __restrict__ status) {
+                        int* __restrict__ status, const int* __restrict__ m_dev) {
+  const int M = m_dev ? min(*m_dev, M_max) : M_max;
   using G = PairCfg;
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -628,7 +661,7 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
   gemm_tc_pair_kernel<EPI><<<2 * pairs, kThreads, G::kSmem, stream>>>(
       *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c, a.split,
-      a.status);
+      a.status, a.m_dev);
   return cudaGetLastError();
 }
 
@@ -646,7 +679,7 @@ cudaError_t launch_impl(const TcGemmArgs& a, cudaStream_t stream) {
   const int grid = tiles < a.num_sms ? tiles : a.num_sms;
   gemm_tc_kernel<BN, EPI><<<grid, kThreads, G::kSmem, stream>>>(
       *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c, a.split,
-      a.status);
+      a.status, a.m_dev);
   return cudaGetLastError();
 }
 
@@ -657,6 +690,7 @@ cudaError_t launch_bn(const TcGemmArgs& a, cudaStream_t stream) {
     case Epi::kBiasGelu: return launch_impl<BN, Epi::kBiasGelu>(a, stream);
     case Epi::kBiasQkvSplit: return launch_impl<BN, Epi::kBiasQkvSplit>(a, stream);
     case Epi::kBiasGeluTanh: return launch_impl<BN, Epi::kBiasGeluTanh>(a, stream);
+    case Epi::kBiasStore: return launch_impl<BN, Epi::kBiasStore>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -728,6 +762,7 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
       case Epi::kBiasGelu: return launch_pair<Epi::kBiasGelu>(a, stream);
       case Epi::kBiasQkvSplit: return launch_pair<Epi::kBiasQkvSplit>(a, stream);
       case Epi::kBiasGeluTanh: return launch_pair<Epi::kBiasGeluTanh>(a, stream);
+      case Epi::kBiasStore: return launch_pair<Epi::kBiasStore>(a, stream);
     }
     return cudaErrorInvalidValue;
   }

@@ -17,7 +17,8 @@ enum class Epi : int {
   kStore = 0,        // C[m][n] = acc
   kBiasGelu = 1,     // C[m][n] = GELU(acc + bias[n]), erf form
   kBiasQkvSplit = 2, // Q/K/V head split: dst[t][b][h][s][c] = acc + bias[n]
-  kBiasGeluTanh = 3  // C[m][n] = GELU_tanh(acc + bias[n])
+  kBiasGeluTanh = 3, // C[m][n] = GELU_tanh(acc + bias[n])
+  kBiasStore = 4     // C[m][n] = acc + bias[n]
 };
 
 // Addressing for the head-split epilogue (n = t*H + h*d + c, m = b*seq + s).
@@ -46,6 +47,7 @@ struct TcGemmArgs {
   SplitShape split;
   int* status;                 // device status word
   int num_sms;
+  const int* m_dev = nullptr;  // optional device row count (<= M): rows past it are neither computed nor stored
 };
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream);
 
@@ -56,6 +58,17 @@ bool encode_kmajor_fp16_map(CUtensorMap* map, const void* base, uint64_t rows, u
 bool encode_output_map_2d(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols);
 bool encode_output_map_split(CUtensorMap* map, void* base, const SplitShape& sp);
 
+// ---- padding removal, pack.cu ----
+// offsets[b] = sum_{b' < b} clamp(valid_len[b'], 0, seq); offsets[batch] = total valid tokens.
+cudaError_t launch_valid_offsets(const int32_t* valid_len, int batch, int seq, int32_t* offsets,
+                                 cudaStream_t stream);
+// xp[offsets[b] + s] = x[b][s] for s < n_b (rows of `hidden` halves).
+cudaError_t launch_pack_rows(const __half* x, const int32_t* valid_len, const int32_t* offsets, __half* xp,
+                             int batch, int seq, int hidden, cudaStream_t stream);
+// out[b][s] = yp[offsets[b] + s] for s < n_b, 0 otherwise.
+cudaError_t launch_unpack_rows(const __half* yp, const int32_t* valid_len, const int32_t* offsets, __half* out,
+                               int batch, int seq, int hidden, cudaStream_t stream);
+
 // ---- FP32 SIMT GEMM (FP32 mode, no TF32), gemm_f32.cu ----
 // C = A[M,K] * W[K,N] (W row-major [K,N]).
 cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K, Epi epi,
@@ -65,6 +78,11 @@ cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K,
 cudaError_t launch_attention_f16(const __half* qkv, const int32_t* valid_len, __half* ctx,
                                  int batch, int seq, int head_num, int size_per_head,
                                  cudaStream_t stream);
+// Packed tokens: qkv is [T, 3H] (Q | K | V per token), sequence b occupies rows
+// offsets[b] .. offsets[b] + n_b - 1; ctx is [T, H].
+cudaError_t launch_attention_f16_packed(const __half* qkv, const int32_t* valid_len, const int32_t* offsets,
+                                        __half* ctx, int batch, int seq, int head_num, int size_per_head,
+                                        cudaStream_t stream);
 cudaError_t launch_attention_f32(const float* qkv, const int32_t* valid_len, float* ctx,
                                  int batch, int seq, int head_num, int size_per_head,
                                  cudaStream_t stream);
@@ -76,7 +94,8 @@ cudaError_t launch_bias_residual_ln_f16(const __half* a, const float* bias, cons
 // FP16 rows with FP16 parameters (hidden <= 1024): one row per warp.
 cudaError_t launch_bias_residual_ln_f16h(const __half* a, const __half* bias, const __half* resid,
                                          const __half* gamma, const __half* beta, __half* out,
-                                         int rows, int hidden, cudaStream_t stream);
+                                         int rows, int hidden, cudaStream_t stream,
+                                         const int* rows_dev = nullptr);
 cudaError_t launch_bias_residual_ln_f32(const float* a, const float* bias, const float* resid,
                                         const float* gamma, const float* beta, float* out,
                                         int rows, int hidden, cudaStream_t stream);

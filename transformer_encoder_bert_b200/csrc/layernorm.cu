@@ -195,10 +195,12 @@ template <int VPT>
 __global__ void __launch_bounds__(128)
     bias_residual_ln_rowwarp_kernel(const __half* __restrict__ a, const __half* __restrict__ bias,
                                     const __half* __restrict__ resid, const __half* __restrict__ gamma,
-                                    const __half* __restrict__ beta, __half* __restrict__ out, int rows, int H) {
+                                    const __half* __restrict__ beta, __half* __restrict__ out, int rows, int H,
+                                    const int* __restrict__ rows_dev) {
   constexpr int E = 8;
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (rows_dev) rows = min(rows, *rows_dev);   // packed tokens: the row count lives on the device
   if (row >= rows) return;
   const int nvec = H / E;
   uint4 xa[VPT], ya[VPT];
@@ -287,13 +289,14 @@ cudaError_t launch_ln(const T* a, const float* bias, const T* resid, const float
 
 cudaError_t launch_bias_residual_ln_f16h(const __half* a, const __half* bias, const __half* resid,
                                          const __half* gamma, const __half* beta, __half* out, int rows,
-                                         int hidden, cudaStream_t stream) {
+                                         int hidden, cudaStream_t stream, const int* rows_dev) {
   if (rows <= 0 || hidden <= 0 || hidden % 8 != 0) return cudaErrorInvalidValue;
   const int vpt = (hidden / 8 + 31) / 32;
   const dim3 grid((rows + 3) / 4);
 #define ENC_LN_ROW_CASE(V)                                                                                  \
   if (vpt <= V) {                                                                                           \
-    bias_residual_ln_rowwarp_kernel<V><<<grid, 128, 0, stream>>>(a, bias, resid, gamma, beta, out, rows, hidden); \
+    bias_residual_ln_rowwarp_kernel<V><<<grid, 128, 0, stream>>>(a, bias, resid, gamma, beta, out, rows, hidden, \
+                                                                 rows_dev);                                  \
     return cudaGetLastError();                                                                              \
   }
   ENC_LN_ROW_CASE(1)
