@@ -220,12 +220,16 @@ def test_recorded_forward_replays_bit_exact():
     assert enc.device_status() == 0
 
 
-def test_host_entry_point_chunked_pipeline_matches_device_forward():
-    # 256 x 32 tokens: enc_forward_host cuts the batch into 4 chunks with overlapped copies.
+@pytest.mark.parametrize("chunks,layers", [(2, 12), (4, 12), (4, 2), (3, 3)])
+def test_host_entry_point_chunked_pipeline_matches_device_forward(chunks, layers):
+    # 256 x 32 tokens: the first and last layers run chunk by chunk while the
+    # copies of the other chunks are in flight; results are bit-identical.
     import torch
-    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 256))
+    wl = EI.named_workload("bert-base-s32", 256)
+    inp = EI.make_inputs(wl.with_(shape=EI.EncoderShape(12, 64, 3072, layers)))
     enc = encoder_from_inputs(inp)
     dev = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    enc.set_host_chunks(chunks)
     hx = torch.from_numpy(inp.x).pin_memory()
     hvl = torch.from_numpy(inp.valid_len).pin_memory()
     hout = torch.empty_like(hx).pin_memory()

@@ -551,6 +551,29 @@ enc_status forward_packed(enc_handle* h, const void* x, const int32_t* valid_len
   return ENC_OK;
 }
 
+// The 7 launches of one dense layer: xin [batch*seq, H] -> xout, with the
+// intermediate buffers of `w` (carved for at least batch*seq tokens).
+template <typename Mark>
+enc_status run_layer(enc_handle* h, int l, const void* xin, void* xout, const int32_t* valid_len, int batch, int seq,
+                     const Workspace& w, cudaStream_t st, Mark& mark) {
+  const int tokens = batch * seq;
+  enc_status s;
+  mark();
+  if ((s = step_qkv(h, l, xin, w.qkv, batch, seq, st)) != ENC_OK) return s;
+  mark();
+  if ((s = step_attention(h, w.qkv, valid_len, w.ctx, batch, seq, st)) != ENC_OK) return s;
+  mark();
+  if ((s = step_out_proj(h, l, w.ctx, w.a, tokens, st)) != ENC_OK) return s;
+  mark();
+  if ((s = step_ln(h, l, 1, w.a, xin, w.h1, tokens, st)) != ENC_OK) return s;
+  mark();
+  if ((s = step_ffn1(h, l, w.h1, w.u, tokens, st)) != ENC_OK) return s;
+  mark();
+  if ((s = step_ffn2(h, l, w.u, w.a, tokens, st)) != ENC_OK) return s;
+  mark();
+  return step_ln(h, l, 2, w.a, w.h1, xout, tokens, st);
+}
+
 // Checks, workspace, and the per-layer launches of one forward on `st`.
 enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
                         cudaStream_t st, bool tracing) {
@@ -573,23 +596,11 @@ enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, 
     if (tracing) cudaEventRecord(h->trace[k++], st);
   };
   if (h->packed) return forward_packed(h, x, valid_len, out, batch, seq, st, w, mark);
+  (void)tokens;
   for (int l = 0; l < h->L; ++l) {
     const void* xin = l == 0 ? x : (((l - 1) & 1) ? w.x1 : w.x0);
     void* xout = l == h->L - 1 ? out : ((l & 1) ? w.x1 : w.x0);
-    mark();
-    if ((s = step_qkv(h, l, xin, w.qkv, batch, seq, st)) != ENC_OK) return s;
-    mark();
-    if ((s = step_attention(h, w.qkv, valid_len, w.ctx, batch, seq, st)) != ENC_OK) return s;
-    mark();
-    if ((s = step_out_proj(h, l, w.ctx, w.a, tokens, st)) != ENC_OK) return s;
-    mark();
-    if ((s = step_ln(h, l, 1, w.a, xin, w.h1, tokens, st)) != ENC_OK) return s;
-    mark();
-    if ((s = step_ffn1(h, l, w.h1, w.u, tokens, st)) != ENC_OK) return s;
-    mark();
-    if ((s = step_ffn2(h, l, w.u, w.a, tokens, st)) != ENC_OK) return s;
-    mark();
-    if ((s = step_ln(h, l, 2, w.a, w.h1, xout, tokens, st)) != ENC_OK) return s;
+    if ((s = run_layer(h, l, xin, xout, valid_len, batch, seq, w, st, mark)) != ENC_OK) return s;
   }
   mark();
   return ENC_OK;
@@ -705,12 +716,16 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_fail(e, "copy stream setup");
   }
-  // Sequences are independent, so the batch is cut into up to kMaxChunks chunks
-  // of at least 2048 tokens: chunk i+1 is copied in and chunk i-1 copied out
-  // while chunk i runs, so the copies hide behind the encoder.
+  // Sequences are independent, so the batch can be cut into chunks: the first
+  // layer runs chunk by chunk as each chunk's input lands, the middle layers
+  // run on the whole batch, and the last layer runs chunk by chunk so that each
+  // chunk's output is copied out while the next one is computed.  Only the
+  // first and last layers pay the smaller GEMMs.  One chunk, a packed forward,
+  // or fewer than 2 layers: copy in, run, copy out.
   const long tokens = (long)batch * seq;
   int chunks = (int)std::min<long>(h->host_chunks, std::max<long>(1, tokens / 2048));
   chunks = std::min(chunks, batch);
+  if (h->packed || h->L < 2) chunks = 1;
   char* base = static_cast<char*>(h->stage);
   char* dx = base;
   char* dout = base + act_al;
@@ -724,20 +739,54 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
   if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_start, 0);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dvl, valid_len, (size_t)batch * 4, cudaMemcpyHostToDevice, h->copy_in);
   if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-  int b0 = 0;
+  int cb[enc_handle::kMaxChunks + 1];
+  cb[0] = 0;
+  for (int c = 0; c < chunks; ++c) cb[c + 1] = cb[c] + batch / chunks + (c < batch % chunks ? 1 : 0);
   for (int c = 0; c < chunks; ++c) {
-    const int nb = batch / chunks + (c < batch % chunks ? 1 : 0);
-    const size_t off = (size_t)b0 * seq_bytes, bytes = (size_t)nb * seq_bytes;
+    const size_t off = (size_t)cb[c] * seq_bytes, bytes = (size_t)(cb[c + 1] - cb[c]) * seq_bytes;
     e = cudaMemcpyAsync(dx + off, hx + off, bytes, cudaMemcpyHostToDevice, h->copy_in);
     if (e == cudaSuccess) e = cudaEventRecord(h->ev_in[c], h->copy_in);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->ev_in[c], 0);
     if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-    if ((s = forward_impl(h, dx + off, dvl + b0, dout + off, nb, seq, st, false)) != ENC_OK) return s;
-    e = cudaEventRecord(h->ev_done[c], st);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_done[c], 0);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(hout + off, dout + off, bytes, cudaMemcpyDeviceToHost, h->copy_out);
-    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
-    b0 += nb;
+  }
+  auto copy_out_chunk = [&](int c) -> enc_status {
+    const size_t off = (size_t)cb[c] * seq_bytes, bytes = (size_t)(cb[c + 1] - cb[c]) * seq_bytes;
+    cudaError_t ce = cudaEventRecord(h->ev_done[c], st);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(h->copy_out, h->ev_done[c], 0);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(hout + off, dout + off, bytes, cudaMemcpyDeviceToHost, h->copy_out);
+    return ce == cudaSuccess ? ENC_OK : cuda_fail(ce, "device-to-host copy");
+  };
+  if (chunks == 1) {
+    e = cudaStreamWaitEvent(st, h->ev_in[0], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "stream wait");
+    if ((s = forward_impl(h, dx, dvl, dout, batch, seq, st, false)) != ENC_OK) return s;
+    if ((s = copy_out_chunk(0)) != ENC_OK) return s;
+  } else {
+    if ((s = check_handle(h)) != ENC_OK) return s;
+    if ((s = ensure_workspace(h, (size_t)tokens)) != ENC_OK) return s;
+    const Workspace w = carve(h, (size_t)tokens);
+    auto no_mark = [] {};
+    const int L = h->L;
+    for (int c = 0; c < chunks; ++c) {          // layer 0, chunk by chunk
+      const size_t off = (size_t)cb[c] * seq_bytes;
+      e = cudaStreamWaitEvent(st, h->ev_in[c], 0);
+      if (e != cudaSuccess) return cuda_fail(e, "stream wait");
+      if ((s = run_layer(h, 0, dx + off, static_cast<char*>(w.x0) + off, dvl + cb[c], cb[c + 1] - cb[c], seq, w, st,
+                         no_mark)) != ENC_OK)
+        return s;
+    }
+    for (int l = 1; l < L - 1; ++l) {            // middle layers, whole batch
+      const void* xin = ((l - 1) & 1) ? w.x1 : w.x0;
+      void* xo = (l & 1) ? w.x1 : w.x0;
+      if ((s = run_layer(h, l, xin, xo, dvl, batch, seq, w, st, no_mark)) != ENC_OK) return s;
+    }
+    const char* xlast = static_cast<const char*>(((L - 2) & 1) ? w.x1 : w.x0);
+    for (int c = 0; c < chunks; ++c) {          // last layer, chunk by chunk, each copied out at once
+      const size_t off = (size_t)cb[c] * seq_bytes;
+      if ((s = run_layer(h, L - 1, xlast + off, dout + off, dvl + cb[c], cb[c + 1] - cb[c], seq, w, st, no_mark)) !=
+          ENC_OK)
+        return s;
+      if ((s = copy_out_chunk(c)) != ENC_OK) return s;
+    }
   }
   e = cudaEventRecord(h->ev_out, h->copy_out);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->ev_out, 0);
