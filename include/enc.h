@@ -166,7 +166,8 @@ ENC_API const char* enc_last_error(void);
 /* enc_device_status - read and clear the handle's device status word (synchronises
  * the device).  *code is 0 when no kernel has reported a failure since the last
  * read; otherwise the code of the first failure (1 = a bounded wait inside a
- * tensor-core GEMM gave up).  Returns ENC_ERR_DEVICE when *code != 0. */
+ * tensor-core GEMM or attention kernel gave up).  Returns ENC_ERR_DEVICE when
+ * *code != 0. */
 ENC_API enc_status enc_device_status(enc_t h, int32_t* code);
 
 /* enc_graph_create - record one enc_forward (these exact buffers, batch and seq)

@@ -55,7 +55,7 @@ def test_qkv_projection_and_head_split(shape, batch, seq):
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}_F{s[2]}")
-@pytest.mark.parametrize("batch,seq", BATCH_SEQ + [(2, 512), (3, 200)], ids=lambda v: str(v))
+@pytest.mark.parametrize("batch,seq", BATCH_SEQ + [(2, 512), (3, 200), (4, 96), (3, 65)], ids=lambda v: str(v))
 def test_attention(shape, batch, seq):
     nh, d, _ = shape
     wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
@@ -147,10 +147,13 @@ def test_fp32_steps(shape):
     assert rel_l2(to_host(out), ref) < FP32_REL_L2
 
 
-def test_attention_valid_len_clamping_and_empty():
+@pytest.mark.parametrize("seq", [40, 100], ids=str)
+def test_attention_valid_len_clamping_and_empty(seq):
+    """Lengths outside [0, seq] are clamped; n == 0 gives ctx = 0 (seq 40 runs the
+    mma.sync kernel, seq 100 the tensor-core one)."""
     shape = (12, 64, 3072)
     nh, d, _ = shape
-    batch, seq = 4, 40
+    batch = 4
     wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
     qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=8)
     vlen = np.array([seq + 7, 0, -3, 1], np.int32)      # clamp to [0, seq]
@@ -216,3 +219,21 @@ def test_alternative_gemm_paths(monkeypatch, env, batch, seq):
     enc.op_qkv(0, to_dev(inp.x), out, batch, seq)
     ref = O.head_split(O.qkv_projection(x64.reshape(-1, H), lw["w_qkv"], lw["b_qkv"]), batch, seq, nh, d)
     assert rel_l2(to_host(out), ref) < GEMM_REL_L2
+
+
+@pytest.mark.parametrize("batch,seq", [(3, 128), (4, 96), (3, 65)], ids=str)
+def test_attention_mma_sync_path_for_long_sequences(monkeypatch, batch, seq):
+    """Size-64 heads on sequences of 65..128 run on the tensor-core (tcgen05) kernel;
+    the mma.sync kernel for the same shapes stays checked through ENC_ATTN_NO_TC."""
+    monkeypatch.setenv("ENC_ATTN_NO_TC", "1")
+    shape = (12, 64, 3072)
+    nh, d, _ = shape
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=17)
+    vlen = np.array([seq] + [max(1, seq // (i + 2)) for i in range(batch - 1)], np.int32)
+    ctx = empty_dev((batch * seq, nh * d), "fp16")
+    enc.op_attention(to_dev(qkv), to_dev(vlen), ctx, batch, seq)
+    got = to_host(ctx).reshape(batch, seq, nh * d)
+    ref = O.attention(qkv.astype(np.float64), vlen)
+    assert rel_l2(got, ref) < ATTN_REL_L2
+

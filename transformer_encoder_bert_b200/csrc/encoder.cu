@@ -111,6 +111,7 @@ struct enc_handle {
   int host_chunks = 1;              // enc_forward_host: most chunks the batch is cut into (see enc.h)
   bool no_pair = false;             // ENC_GEMM_NO_PAIR=1: one-CTA tiles only (comparison runs)
   bool no_tma_store = false;        // ENC_GEMM_NO_TMA_STORE=1: epilogue stores without TMA
+  bool no_tc_attn = false;          // ENC_ATTN_NO_TC=1: mma.sync attention for every length
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -233,10 +234,20 @@ enc_status step_qkv(enc_handle* h, int l, const void* x, void* qkv, int batch, i
                   sp, st);
 }
 
+// Attention kernel choice: the tensor-core kernel for size_per_head 64 when one
+// 128-key block covers a sequence longer than the short kernel's 64-row tiles;
+// mma.sync otherwise (and for every length under ENC_ATTN_NO_TC=1).
+bool use_tc_attention(const enc_handle* h, int seq) {
+  return enc::attention_tc_supported(h->d, seq) && !h->no_tc_attn;
+}
+
 enc_status step_attention(enc_handle* h, const void* qkv, const int32_t* vl, void* ctx, int batch, int seq,
                           cudaStream_t st) {
   cudaError_t e;
-  if (h->dtype == ENC_FP16)
+  if (h->dtype == ENC_FP16 && use_tc_attention(h, seq))
+    e = enc::launch_attention_tc(static_cast<const __half*>(qkv), vl, nullptr, static_cast<__half*>(ctx), batch, seq,
+                                 h->nh, h->status, st);
+  else if (h->dtype == ENC_FP16)
     e = enc::launch_attention_f16(static_cast<const __half*>(qkv), vl, static_cast<__half*>(ctx), batch, seq,
                                   h->nh, h->d, st);
   else
@@ -364,6 +375,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   h->num_sms = enc::device_sm_count();
   if (const char* e = getenv("ENC_GEMM_NO_PAIR")) h->no_pair = e[0] == '1';
   if (const char* e = getenv("ENC_GEMM_NO_TMA_STORE")) h->no_tma_store = e[0] == '1';
+  if (const char* e = getenv("ENC_ATTN_NO_TC")) h->no_tc_attn = e[0] == '1';
   if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
   if (dtype == ENC_FP16) {
     cudaDeviceProp prop;
@@ -517,8 +529,12 @@ enc_status forward_packed(enc_handle* h, const void* x, const int32_t* valid_len
         ENC_OK)
       return s;
     mark();
-    e = enc::launch_attention_f16_packed(static_cast<const __half*>(w.qkv), valid_len, w.offsets,
-                                         static_cast<__half*>(w.ctx), batch, seq, h->nh, h->d, st);
+    if (use_tc_attention(h, seq))
+      e = enc::launch_attention_tc(static_cast<const __half*>(w.qkv), valid_len, w.offsets,
+                                   static_cast<__half*>(w.ctx), batch, seq, h->nh, h->status, st);
+    else
+      e = enc::launch_attention_f16_packed(static_cast<const __half*>(w.qkv), valid_len, w.offsets,
+                                           static_cast<__half*>(w.ctx), batch, seq, h->nh, h->d, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     ++h->launches;
     mark();

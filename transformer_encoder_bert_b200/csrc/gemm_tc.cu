@@ -72,24 +72,6 @@ struct Cfg {
 // sm_100 (fma/mul .f32x2): the polynomial, the squarings and the final
 // scaling cost one instruction per pair; the reciprocal and the sign stay per
 // element.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ void gelu_erf_pair(float& v0, float& v1) {
   const uint64_t v = f2_pack(v0, v1);
   const uint64_t z = f2_mul(f2_pack(fabsf(v0), fabsf(v1)), f2_pack(0.70710678118654752f, 0.70710678118654752f));

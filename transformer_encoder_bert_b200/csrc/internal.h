@@ -87,6 +87,13 @@ cudaError_t launch_attention_f32(const float* qkv, const int32_t* valid_len, flo
                                  int batch, int seq, int head_num, int size_per_head,
                                  cudaStream_t stream);
 
+// Tensor-core attention (attention_tc.cu): size_per_head 64 and 64 < seq <= 128
+// (attention_tc_supported); offsets == nullptr reads the split layout
+// [3, B, nh, S, 64], else the packed [T, 3H] layout.
+bool attention_tc_supported(int size_per_head, int seq);
+cudaError_t launch_attention_tc(const __half* qkv, const int32_t* valid_len, const int32_t* offsets, __half* ctx,
+                                int batch, int seq, int head_num, int* status, cudaStream_t stream);
+
 // ---- add-bias + residual + LayerNorm, layernorm.cu ----
 cudaError_t launch_bias_residual_ln_f16(const __half* a, const float* bias, const __half* resid,
                                         const float* gamma, const float* beta, __half* out,
