@@ -237,3 +237,54 @@ def test_attention_mma_sync_path_for_long_sequences(monkeypatch, batch, seq):
     ref = O.attention(qkv.astype(np.float64), vlen)
     assert rel_l2(got, ref) < ATTN_REL_L2
 
+
+@pytest.mark.parametrize("batch,seq", [(1, 32), (8, 32), (1, 7), (3, 37)], ids=str)
+def test_split_k_gemms(monkeypatch, batch, seq):
+    """At small M the GEMMs run split-K: a cluster of CTAs shares each 128x128 tile,
+    each CTA one range of the k-blocks, and the partial tiles are summed in rank
+    order through distributed shared memory.  Every epilogue (head split, plain,
+    erf-GELU, tanh-GELU) against its oracle step; a repeated call is bit-identical
+    (the sum's order does not depend on timing); the unsplit kernel
+    (ENC_GEMM_NO_SPLITK=1) agrees within the GEMM bound."""
+    shape = (12, 64, 3072)
+    nh, d, F = shape
+    H = nh * d
+    M = batch * seq
+    ctx = EI.random_array((M, H), "fp16", seed=31)
+    h1 = EI.random_array((M, H), "fp16", seed=32)
+    uu = EI.random_array((M, F), "fp16", seed=33, std=0.5)
+
+    def run(enc):
+        qkv = empty_dev((3, batch, nh, seq, d), "fp16")
+        enc.op_qkv(0, to_dev(inp.x), qkv, batch, seq)
+        a = empty_dev((M, H), "fp16")
+        enc.op_out_proj(0, to_dev(ctx), a, M)
+        u = empty_dev((M, F), "fp16")
+        enc.op_ffn1(0, to_dev(h1), u, M)
+        enc.set_gelu("tanh")
+        ut = empty_dev((M, F), "fp16")
+        enc.op_ffn1(0, to_dev(h1), ut, M)
+        enc.set_gelu("erf")
+        y = empty_dev((M, H), "fp16")
+        enc.op_ffn2(0, to_dev(uu), y, M)
+        return [to_host(t) for t in (qkv, a, u, ut, y)]
+
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    got = run(enc)
+    refs = [
+        O.head_split(O.qkv_projection(x64.reshape(-1, H), lw["w_qkv"], lw["b_qkv"]), batch, seq, nh, d),
+        ctx.astype(np.float64) @ lw["w_o"],
+        O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"]),
+        O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"], gelu="tanh"),
+        uu.astype(np.float64) @ lw["w_ff2"],
+    ]
+    for g, r in zip(got, refs):
+        assert rel_l2(g, r) < GEMM_REL_L2 and max_abs(g, r) < _ulp_bound(r)
+    again = run(enc)
+    for g, a in zip(got, again):
+        assert np.array_equal(g, a)
+    assert enc.device_status() == 0
+    monkeypatch.setenv("ENC_GEMM_NO_SPLITK", "1")
+    wl, inp, enc1, x64, vl, lw = _setup(shape, batch, seq)
+    for g, r in zip(got, run(enc1)):
+        assert rel_l2(g, r) < GEMM_REL_L2

@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(NW * 32)
   using C = AttnCfg<D, NW, BKV, STAGES, MT>;
   constexpr int kBKV = BKV;
   extern __shared__ __align__(16) __half sm[];
+  pdl_wait();                                   // Q/K/V (and offsets) of the previous kernels are visible
+  pdl_trigger();
   __half* Qs = sm;
   __half* Ks = sm + C::kQElems;                 // [STAGES][kBKV][kLd]
   __half* Vs = Ks + STAGES * C::kKVElems;       // [STAGES][kBKV][kLd]
@@ -329,9 +331,8 @@ cudaError_t launch_f16(const __half* qkv, const int32_t* vl, const int32_t* offs
   if (attr != cudaSuccess) return attr;
   const dim3 grid((S + C::kBQ - 1) / C::kBQ, NH, B);
   const float scale_log2 = kLog2e / sqrtf((float)D);
-  attention_f16_kernel<D, NW, BKV, STAGES, MT, PACKED><<<grid, NW * 32, C::kSmem, stream>>>(
-      qkv, vl, offsets, ctx, B, S, NH, scale_log2);
-  return cudaGetLastError();
+  return launch_kernel(attention_f16_kernel<D, NW, BKV, STAGES, MT, PACKED>, grid, dim3(NW * 32), C::kSmem, stream,
+                       nullptr, 0, qkv, vl, offsets, ctx, B, S, NH, scale_log2);
 }
 
 
@@ -358,6 +359,8 @@ __global__ void __launch_bounds__(NW * 32)
   using C = ShortCfg<D, NW, BKV>;
   static_assert(C::kBQ <= BKV || C::kBQ == 16 * NW, "one query block");
   extern __shared__ __align__(16) __half sm[];
+  pdl_wait();                                   // Q/K/V (and offsets) of the previous kernels are visible
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   constexpr int kChunks = D / 8;
@@ -517,9 +520,8 @@ cudaError_t launch_short(const __half* qkv, const int32_t* vl, const int32_t* of
   const int items = B * NH;
   const int cap = per_sm * device_sm_count();
   const float scale_log2 = kLog2e / sqrtf((float)D);
-  attention_f16_short_kernel<D, NW, BKV, PACKED><<<items < cap ? items : cap, NW * 32, C::kSmem, stream>>>(
-      qkv, vl, offsets, ctx, B, S, NH, scale_log2);
-  return cudaGetLastError();
+  return launch_kernel(attention_f16_short_kernel<D, NW, BKV, PACKED>, dim3(items < cap ? items : cap), dim3(NW * 32),
+                       C::kSmem, stream, nullptr, 0, qkv, vl, offsets, ctx, B, S, NH, scale_log2);
 }
 
 
@@ -547,6 +549,8 @@ __global__ void __launch_bounds__(128)
     attention_f32_kernel(const float* __restrict__ qkv, const int32_t* __restrict__ valid_len,
                          float* __restrict__ ctx, int B, int S, int NH) {
   constexpr int kPer = D / 32;
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.z, h = blockIdx.y;
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -616,12 +620,17 @@ cudaError_t launch_attention_f32(const float* qkv, const int32_t* valid_len, flo
   if (batch <= 0 || seq <= 0 || head_num <= 0 || head_num > 65535 || batch > 65535) return cudaErrorInvalidValue;
   const dim3 grid((seq + 3) / 4, head_num, batch);
   switch (size_per_head) {
-    case 32: attention_f32_kernel<32><<<grid, 128, 0, stream>>>(qkv, valid_len, ctx, batch, seq, head_num); break;
-    case 64: attention_f32_kernel<64><<<grid, 128, 0, stream>>>(qkv, valid_len, ctx, batch, seq, head_num); break;
-    case 128: attention_f32_kernel<128><<<grid, 128, 0, stream>>>(qkv, valid_len, ctx, batch, seq, head_num); break;
-    default: return cudaErrorInvalidValue;
+    case 32:
+      return launch_kernel(attention_f32_kernel<32>, grid, dim3(128), 0, stream, nullptr, 0, qkv, valid_len, ctx,
+                           batch, seq, head_num);
+    case 64:
+      return launch_kernel(attention_f32_kernel<64>, grid, dim3(128), 0, stream, nullptr, 0, qkv, valid_len, ctx,
+                           batch, seq, head_num);
+    case 128:
+      return launch_kernel(attention_f32_kernel<128>, grid, dim3(128), 0, stream, nullptr, 0, qkv, valid_len, ctx,
+                           batch, seq, head_num);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace enc

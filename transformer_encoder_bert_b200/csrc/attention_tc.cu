@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
+  pdl_wait();                                          // Q/K/V (and offsets) of the previous kernels are visible
   int n = valid_len[b];
   n = n < 0 ? 0 : (n > S ? S : n);
   if (PACKED && n == 0) return;                        // the sequence has no rows (uniform per CTA)
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;                    // S in columns [0, 128); O in [0, 64) after softmax
+  pdl_trigger();                                       // after taking TMEM
 
   bool ok = true;
   if (warp == kSoftmaxWarps) {
@@ -207,45 +209,58 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
   } else {
     const int r = warp * 32 + lane;                    // query row = TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int full_chunks = n >> 5;                    // chunks of 32 keys, all valid
-    const int lim = n & 31;                            // valid keys of the partial chunk (0: none)
+    const int nchunks = (n + 31) >> 5;                 // 32-key chunks holding valid keys
     uint8_t* prow = smem + kP + r * 128;
-    uint32_t sv[32];
+    uint32_t sa[32], sb[32];                           // two chunks: one in use, one loading
     uint64_t sum2 = 0;                                 // two partial row sums (0.0f, 0.0f)
     if (n > 0) {
       ok = warp_wait(s_full, 0);
       if (ok) {
         tc_fence_after();
-        // Pass 1: row max over the valid keys.
+        // Pass 1: row max over the valid keys.  The next chunk's TMEM load is
+        // in flight while the current one is scanned.
         float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < full_chunks; ++c) {
-          tmem_ld_32x32b_x32(t_row + 32 * c, sv);
+        tmem_ld_32x32b_x32_async(t_row, sa);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-        }
-        if (lim) {
-          tmem_ld_32x32b_x32(t_row + 32 * full_chunks, sv);
+        for (int c = 0; c < kRows / 32; ++c) {
+          if (c < nchunks) {
+            uint32_t(&cur)[32] = (c & 1) ? sb : sa;
+            uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
+            tmem_wait_ld(cur);
+            if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_row + 32 * (c + 1), nxt);
+            const int lim = n - 32 * c;
+            if (lim >= 32) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < lim) mx = fmaxf(mx, __uint_as_float(sv[i]));
+              for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(cur[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (i < lim) mx = fmaxf(mx, __uint_as_float(cur[i]));
+            }
+          }
         }
         const uint64_t scale2 = f2_pack(score_scale_log2, score_scale_log2);
         const uint64_t neg_m2 = f2_pack(-mx * score_scale_log2, -mx * score_scale_log2);
-        // Pass 2: P, its row sum, FP16 P into the swizzled tile (over Q and K).
-#pragma unroll 1
-        for (int c = 0; c < full_chunks; ++c) {
-          tmem_ld_32x32b_x32(t_row + 32 * c, sv);
-          p_chunk<false>(sv, 32, scale2, neg_m2, sum2, prow, c, r);
+        // Pass 2: P, its row sum, FP16 P into the swizzled tile (over Q and K);
+        // chunks past n get P = 0.
+        tmem_ld_32x32b_x32_async(t_row, sa);
+#pragma unroll
+        for (int c = 0; c < kRows / 32; ++c) {
+          if (c < nchunks) {
+            uint32_t(&cur)[32] = (c & 1) ? sb : sa;
+            uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
+            tmem_wait_ld(cur);
+            if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_row + 32 * (c + 1), nxt);
+            const int lim = n - 32 * c;
+            if (lim >= 32)
+              p_chunk<false>(cur, 32, scale2, neg_m2, sum2, prow, c, r);
+            else
+              p_chunk<true>(cur, lim, scale2, neg_m2, sum2, prow, c, r);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) store_p_unit(prow, 4 * c + u, r, make_uint4(0, 0, 0, 0));
+          }
         }
-        int c = full_chunks;
-        if (lim) {
-          tmem_ld_32x32b_x32(t_row + 32 * c, sv);
-          p_chunk<true>(sv, lim, scale2, neg_m2, sum2, prow, c, r);
-          ++c;
-        }
-        for (; c < kRows / 32; ++c)                    // chunks past n: P = 0
-          for (int u = 0; u < 4; ++u) store_p_unit(prow, 4 * c + u, r, make_uint4(0, 0, 0, 0));
         // V rows of keys >= n: their P is 0, but a row the TMA box brought in
         // from outside the sequence may hold non-finite data (0 * NaN = NaN in
         // the MMA), so zero them.  Row r of the tile is key r.
@@ -274,14 +289,18 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
       const float inv = l > 0.f ? 1.f / l : 0.f;       // n == 0: ctx = 0
       const uint64_t inv2 = f2_pack(inv, inv);
       uint8_t* orow = smem + kV + r * 128;
-#pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
-        if (n > 0) {
-          tmem_ld_32x32b_x32(t_row + 32 * c, sv);
-        } else {
+      if (n > 0) {
+        tmem_ld_32x32b_x32_async(t_row, sa);
+        tmem_ld_32x32b_x32_async(t_row + 32, sb);
+        tmem_wait_ld(sa);
+        tmem_wait_ld(sb);
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[i] = 0u;
-        }
+        for (int i = 0; i < 32; ++i) sa[i] = sb[i] = 0u;
+      }
+#pragma unroll
+      for (int c = 0; c < kD / 32; ++c) {
+        const uint32_t(&sv)[32] = c ? sb : sa;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint32_t w[4];
@@ -366,9 +385,8 @@ cudaError_t launch_tc(const __half* qkv, const int32_t* vl, const int32_t* offse
     return cudaErrorInvalidValue;
   const dim3 grid(NH, B);
   const float scale_log2 = kLog2e / sqrtf((float)kD);
-  attention_tc_kernel<PACKED><<<grid, kThreads, kSmemTotal, stream>>>(map, vl, offsets, ctx, B, S, NH, scale_log2,
-                                                                       status);
-  return cudaGetLastError();
+  return launch_kernel(attention_tc_kernel<PACKED>, grid, dim3(kThreads), kSmemTotal, stream, nullptr, 0, map, vl,
+                       offsets, ctx, B, S, NH, scale_log2, status);
 }
 
 }  // namespace

@@ -112,6 +112,7 @@ struct enc_handle {
   bool no_pair = false;             // ENC_GEMM_NO_PAIR=1: one-CTA tiles only (comparison runs)
   bool no_tma_store = false;        // ENC_GEMM_NO_TMA_STORE=1: epilogue stores without TMA
   bool no_tc_attn = false;          // ENC_ATTN_NO_TC=1: mma.sync attention for every length
+  bool no_splitk = false;           // ENC_GEMM_NO_SPLITK=1: no split-K for small GEMMs (comparison runs)
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -177,13 +178,27 @@ enc_status check_handle(const enc_handle* h) {
   return ENC_OK;
 }
 
-// Tile choice: a 2-CTA 256x256 tile when N is a multiple of 256 and there are
-// enough rows to fill the 256-row tile; otherwise one CTA per 128 x {256,128}.
+// GEMM tiling.  The 2-CTA 256x256 tile when it still gives at least a quarter
+// of the SMs a cluster each; else 128x256 one-CTA tiles when they fill the
+// GPU; else 128x128.
 int choose_bn(const enc_handle* h, int M, int N) {
-  if (N % 256 == 0 && M >= 256 && !h->no_pair) return enc::kPairTile;
+  if (N % 256 == 0 && M >= 256 && !h->no_pair) {
+    const long pair_tiles = (long)((M + 255) / 256) * (N / 256);
+    if (4 * pair_tiles >= h->num_sms) return enc::kPairTile;
+  }
   if (N % 256 != 0) return 128;
   const long tiles256 = (long)((M + 127) / 128) * (N / 256);
   return tiles256 >= h->num_sms ? 256 : 128;
+}
+
+// Split-K for GEMMs whose 128x128 tiles would leave more than half the SMs
+// idle (small batches): the k-blocks of a tile are shared by a cluster of CTAs,
+// so that the weights are streamed by most SMs instead of a few.
+int choose_splits(const enc_handle* h, int M, int N, int K, int bn) {
+  if (bn != 128 || h->no_splitk) return 1;
+  const long tiles = (long)((M + 127) / 128) * ((N + 127) / 128);
+  if (2 * tiles > h->num_sms) return 1;
+  return enc::choose_gemm_splits((int)tiles, (K + 63) / 64, h->num_sms);
 }
 
 // One GEMM step: C = A * W (+ epilogue), dispatched on the handle's dtype.
@@ -215,6 +230,7 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
     a.status = h->status;
     a.num_sms = h->num_sms;
     a.m_dev = m_dev;
+    a.splits = choose_splits(h, M, N, K, bn);
     cudaError_t e = enc::launch_gemm_tc(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
     ++h->launches;
@@ -334,6 +350,14 @@ void free_handle(enc_handle* h) {
 
 }  // namespace
 
+bool enc::pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("ENC_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
 int enc::device_sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -376,6 +400,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   if (const char* e = getenv("ENC_GEMM_NO_PAIR")) h->no_pair = e[0] == '1';
   if (const char* e = getenv("ENC_GEMM_NO_TMA_STORE")) h->no_tma_store = e[0] == '1';
   if (const char* e = getenv("ENC_ATTN_NO_TC")) h->no_tc_attn = e[0] == '1';
+  if (const char* e = getenv("ENC_GEMM_NO_SPLITK")) h->no_splitk = e[0] == '1';
   if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
   if (dtype == ENC_FP16) {
     cudaDeviceProp prop;

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        float* __restrict__ C, SplitShape sp) {
   __shared__ float As[TK][TM + 4];
   __shared__ float Ws[TK][TN + 4];
+  pdl_wait();
+  pdl_trigger();
   const int tx = threadIdx.x & 15;   // column group
   const int ty = threadIdx.x >> 4;   // row group
   const int m0 = blockIdx.y * TM;
@@ -86,22 +88,22 @@ cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K,
   const dim3 grid((N + TN - 1) / TN, (M + TM - 1) / TM);
   switch (epi) {
     case Epi::kStore:
-      gemm_f32_kernel<Epi::kStore><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
-      break;
+      return launch_kernel(gemm_f32_kernel<Epi::kStore>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
+                           C, split);
     case Epi::kBiasGelu:
-      gemm_f32_kernel<Epi::kBiasGelu><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
-      break;
+      return launch_kernel(gemm_f32_kernel<Epi::kBiasGelu>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
+                           C, split);
     case Epi::kBiasQkvSplit:
-      gemm_f32_kernel<Epi::kBiasQkvSplit><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
-      break;
+      return launch_kernel(gemm_f32_kernel<Epi::kBiasQkvSplit>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
+                           C, split);
     case Epi::kBiasGeluTanh:
-      gemm_f32_kernel<Epi::kBiasGeluTanh><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
-      break;
+      return launch_kernel(gemm_f32_kernel<Epi::kBiasGeluTanh>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
+                           C, split);
     case Epi::kBiasStore:
-      gemm_f32_kernel<Epi::kBiasStore><<<grid, 256, 0, stream>>>(A, W, M, N, K, bias, C, split);
-      break;
+      return launch_kernel(gemm_f32_kernel<Epi::kBiasStore>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
+                           C, split);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace enc

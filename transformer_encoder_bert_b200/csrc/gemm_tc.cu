@@ -20,6 +20,7 @@
 // i+1.  Every mbarrier wait is bounded (kWaitLimitNs); a wait that gives up
 // records kStatusWaitTimeout in the status word and the CTA drains its copies
 // and MMAs, frees TMEM and exits.
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <mutex>
@@ -287,7 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M_max, int N, int K,
                    const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp, int* __restrict__ status,
                    const int* __restrict__ m_dev) {
-  const int M = m_dev ? min(*m_dev, M_max) : M_max;
   using G = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -307,10 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_m = (M + kBM - 1) / kBM;
-  const int num_n = (N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
-  const int num_kb = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G::kStages; ++s) {
@@ -336,6 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();                                  // the previous kernel's writes (A, m_dev) are visible
+  pdl_trigger();
+  const int M = m_dev ? min(*m_dev, M_max) : M_max;
+  const int num_m = (M + kBM - 1) / kBM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + kBK - 1) / kBK;
 
   bool ok = true;
   if (warp == 0) {
@@ -460,7 +463,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M_max, int N, int K,
                         const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp,
                         int* __restrict__ status, const int* __restrict__ m_dev) {
-  const int M = m_dev ? min(*m_dev, M_max) : M_max;
   using G = PairCfg;
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -484,10 +486,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int num_pairs = gridDim.x >> 1;
-  const int num_m = (M + 255) / 256;
-  const int num_n = (N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
-  const int num_kb = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G::kStages; ++s) {
@@ -514,6 +512,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();                               // barriers of both CTAs are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();                                   // the previous kernel's writes (A, m_dev) are visible
+  pdl_trigger();
+  const int M = m_dev ? min(*m_dev, M_max) : M_max;
+  const int num_m = (M + 255) / 256;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + kBK - 1) / kBK;
 
   bool ok = true;
   uint32_t issued = 0;
@@ -641,10 +646,278 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   if (max_clusters <= 0) return cudaErrorInvalidConfiguration;
   const int tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
-  gemm_tc_pair_kernel<EPI><<<2 * pairs, kThreads, G::kSmem, stream>>>(
-      *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c, a.split,
-      a.status, a.m_dev);
-  return cudaGetLastError();
+  return launch_kernel(gemm_tc_pair_kernel<EPI>, dim3(2 * pairs), dim3(kThreads), G::kSmem, stream, nullptr, 0,
+                       *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias,
+                       a.c, a.split, a.status, a.m_dev);
+}
+
+// ---------------------------------------------------------------------------
+// Split-K variant for small M, where 128x128 tiles alone would leave most SMs
+// idle while a few stream all of the weights.  A cluster of `splits` CTAs
+// (one per SM) shares each tile; CTA r (its rank in the cluster) accumulates
+// the r-th balanced range of the k-blocks in TMEM:
+//   warp 0      TMA producer (4-stage ring of 128x64 A and B tiles)
+//   warp 1      TMEM owner and MMA issuer (M=128, N=128, K=16)
+//   warps 2..9  copy the FP32 partial tile from TMEM to this CTA's shared
+//               memory; after a cluster barrier each CTA reduces its band of
+//               128/splits rows over all CTAs' partials through distributed
+//               shared memory, in rank order (so the sum does not depend on
+//               timing), applies the epilogue and stores FP16.
+// Nothing goes through global memory but the operands and the result.
+// ---------------------------------------------------------------------------
+struct SplitCfg {
+  static constexpr int kBN = 128;
+  static constexpr int kStages = 4;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = kBN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kPartOffset = kStages * kStageBytes;      // FP32 partial, 128 rows x 512 bytes
+  static constexpr int kPartBytes = kBM * kBN * 4;
+  static constexpr int kBarOffset = kPartOffset + kPartBytes;
+  static constexpr int kNumBars = 2 * kStages + 2;                // full, empty, tfull, drain
+  static constexpr int kSmem = 1024 + kBarOffset + kNumBars * 8 + 16;
+  static constexpr int kTmemCols = 128;
+  static constexpr int kMaxSplits = 16;
+};
+
+// Byte offset of float4 unit u (0..31) of partial row r: units swizzled by r
+// so that a warp writing 32 rows (one unit each) and a warp reading one row
+// (all 32 units) both spread over the banks.
+__device__ __forceinline__ uint32_t part_offset(int r, int u) {
+  return SplitCfg::kPartOffset + r * 512 + 16 * (u ^ (r & 31));
+}
+
+// Bias and the epilogue's element-wise function on 4 consecutive columns.
+template <Epi EPI>
+__device__ __forceinline__ void epilogue4(float (&v)[4], const float* __restrict__ bias, int col) {
+  if constexpr (EPI != Epi::kStore) {
+    const float4 b = __ldg(reinterpret_cast<const float4*>(bias + col));
+    v[0] += b.x; v[1] += b.y; v[2] += b.z; v[3] += b.w;
+  }
+  if constexpr (EPI == Epi::kBiasGelu) {
+    gelu_erf_pair(v[0], v[1]);
+    gelu_erf_pair(v[2], v[3]);
+  }
+  if constexpr (EPI == Epi::kBiasGeluTanh) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = gelu_tanh(v[i]);
+  }
+}
+
+template <Epi EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_splitk_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                          int M_max, int N, int K, const float* __restrict__ bias, __half* __restrict__ C,
+                          SplitShape sp, int* __restrict__ status, const int* __restrict__ m_dev, int splits) {
+  using G = SplitCfg;
+  const int num_n = (N + G::kBN - 1) / G::kBN;
+  const int tile = blockIdx.x / splits;
+  const int ks = static_cast<int>(cluster_ctarank());
+  const int m_blk = tile / num_n;
+  const int n_blk = tile - m_blk * num_n;
+  const int num_kb = (K + kBK - 1) / kBK;
+  const int kb0 = ks * num_kb / splits;
+  const int kb1 = (ks + 1) * num_kb / splits;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::kBarOffset);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::kNumBars);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (G::kStages + s); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * G::kStages);
+  const uint32_t drain_bar = bar0 + 8u * (2 * G::kStages + 1);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(tfull_bar, 1);
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), G::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();                                 // the previous kernel's writes (A, m_dev) are visible
+  pdl_trigger();
+  const int M = m_dev ? min(*m_dev, M_max) : M_max;
+  if (m_blk * kBM >= M) {                     // a tile past the device row count: the whole cluster leaves
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, G::kTmemCols);
+    }
+    return;
+  }
+
+  bool ok = true;
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % G::kStages;
+        const uint32_t ph = (it / G::kStages) & 1u;
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+        mbar_arrive_expect_tx(full_bar(s), G::kStageBytes);
+        tma_load_2d(&tm_a, sbase + s * G::kStageBytes, full_bar(s), kb * kBK, m_blk * kBM);
+        tma_load_2d(&tm_b, sbase + s * G::kStageBytes + G::kABytes, full_bar(s), kb * kBK, n_blk * G::kBN);
+      }
+      const uint32_t first = it > (uint32_t)G::kStages ? it - G::kStages : 0u;
+      for (uint32_t j = first; j < it; ++j)
+        mbar_wait(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(kBM, G::kBN);
+      uint32_t it = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % G::kStages;
+        const uint32_t ph = (it / G::kStages) & 1u;
+        if (!mbar_wait(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = sbase + s * G::kStageBytes;
+        const uint32_t b_addr = a_addr + G::kABytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          mma_f16_ss(tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
+                     (kb > kb0 || kk > 0) ? 1u : 0u);
+        mma_commit(empty_bar(s));
+      }
+      if (ok) mma_commit(tfull_bar);
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, kWaitLimitNs);
+    }
+  } else {
+    // TMEM lanes of quadrant warp % 4; columns [64 * slice, 64 * slice + 64).
+    const int quad = warp & 3;
+    const int slice = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;
+    int got = 0;
+    if (lane == 0) got = mbar_wait(tfull_bar, 0, kWaitLimitNs) ? 1 : 0;
+    got = __shfl_sync(0xffffffffu, got, 0);
+    if (got) {
+      tc_fence_after();
+      uint32_t v[32];
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + slice * 64 + 32 * j, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(smem + part_offset(r, slice * 16 + 8 * j + q)) =
+              make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+    } else {
+      ok = false;
+    }
+  }
+  __syncwarp();
+  cluster_sync();                             // every CTA's partial is in its shared memory
+
+  if (warp >= 2) {
+    // Rows [row0, row1) of the tile, 8 rows per pass, one float4 column unit per lane.
+    const int t = threadIdx.x - 64;
+    const int u = t & 31;
+    const int row0 = ks * kBM / splits;
+    const int row1 = (ks + 1) * kBM / splits;
+    const int col = n_blk * G::kBN + 4 * u;
+    if (col < N) {
+      for (int r = row0 + (t >> 5); r < row1; r += 8) {
+        const int grow = m_blk * kBM + r;
+        if (grow >= M) break;
+        const uint32_t off = sbase + part_offset(r, u);
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int s = 0; s < splits; ++s) {      // rank order: the same sum on every run
+          const float4 p = ld_cluster_f4(mapa_shared(off, (uint32_t)s));
+          a[0] += p.x; a[1] += p.y; a[2] += p.z; a[3] += p.w;
+        }
+        epilogue4<EPI>(a, bias, col);
+        __half* dst = C + row_offset<EPI>(grow, N, sp) + col_offset<EPI>(col, sp);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_half2(a[0], a[1]), pack_half2(a[2], a[3]));
+      }
+    }
+  }
+  __syncwarp();
+  cluster_sync();                             // no CTA leaves while a peer may still read its partial
+
+  if (!ok) atomicCAS(status, 0, kStatusWaitTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, G::kTmemCols);
+  }
+}
+
+// Most clusters of `size` split-K CTAs resident at once (0 when none fit).
+int splitk_max_clusters(int size) {
+  static std::mutex mu;
+  static int cache[16][SplitCfg::kMaxSplits + 1] = {};
+  static bool done[16][SplitCfg::kMaxSplits + 1] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 16 || size < 1 || size > SplitCfg::kMaxSplits) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev][size]) {
+    auto kern = gemm_tc_splitk_kernel<Epi::kStore>;    // every epilogue has the same resources
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SplitCfg::kSmem) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(size * 64, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = SplitCfg::kSmem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = size;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cache[dev][size] = n;
+    done[dev][size] = true;
+  }
+  return cache[dev][size];
+}
+
+template <Epi EPI>
+cudaError_t launch_splitk(const TcGemmArgs& a, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tc_splitk_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SplitCfg::kSmem);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(gemm_tc_splitk_kernel<EPI>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + SplitCfg::kBN - 1) / SplitCfg::kBN);
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = a.splits;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  return launch_kernel(gemm_tc_splitk_kernel<EPI>, dim3(tiles * a.splits), dim3(kThreads), SplitCfg::kSmem, stream,
+                       &attr, 1, *a.tmap_a, *a.tmap_b, a.M, a.N, a.K, a.bias, a.c, a.split, a.status, a.m_dev,
+                       a.splits);
 }
 
 template <int BN, Epi EPI>
@@ -659,10 +932,9 @@ cudaError_t launch_impl(const TcGemmArgs& a, cudaStream_t stream) {
   if (attr_err != cudaSuccess) return attr_err;
   const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + BN - 1) / BN);
   const int grid = tiles < a.num_sms ? tiles : a.num_sms;
-  gemm_tc_kernel<BN, EPI><<<grid, kThreads, G::kSmem, stream>>>(
-      *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c, a.split,
-      a.status, a.m_dev);
-  return cudaGetLastError();
+  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), G::kSmem, stream, nullptr, 0, *a.tmap_a,
+                       *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c,
+                       a.split, a.status, a.m_dev);
 }
 
 template <int BN>
@@ -732,11 +1004,31 @@ bool encode_output_map_split(CUtensorMap* map, void* base, const SplitShape& sp)
          CUDA_SUCCESS;
 }
 
+int choose_gemm_splits(int tiles, int num_kb, int num_sms) {
+  if (tiles <= 0) return 1;
+  for (int s = std::min(SplitCfg::kMaxSplits, num_kb); s >= 2; --s)
+    if ((long)tiles * s <= num_sms && tiles <= splitk_max_clusters(s)) return s;
+  return 1;
+}
+
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0 || (a.N % 8) != 0 || (a.K % 8) != 0) return cudaErrorInvalidValue;
   if (a.epi == Epi::kBiasQkvSplit && (a.split.size_per_head % 32) != 0) return cudaErrorInvalidValue;
   // The head-split store map needs every 32-row chunk inside one sequence.
   if (a.epi == Epi::kBiasQkvSplit && a.tmap_c && (a.split.seq % 32) != 0) return cudaErrorInvalidValue;
+  if (a.splits > 1) {
+    // every CTA of a cluster needs at least one k-block
+    if (a.bn != 128 || a.splits > SplitCfg::kMaxSplits || a.splits > (a.K + kBK - 1) / kBK)
+      return cudaErrorInvalidValue;
+    switch (a.epi) {
+      case Epi::kStore: return launch_splitk<Epi::kStore>(a, stream);
+      case Epi::kBiasGelu: return launch_splitk<Epi::kBiasGelu>(a, stream);
+      case Epi::kBiasQkvSplit: return launch_splitk<Epi::kBiasQkvSplit>(a, stream);
+      case Epi::kBiasGeluTanh: return launch_splitk<Epi::kBiasGeluTanh>(a, stream);
+      case Epi::kBiasStore: return launch_splitk<Epi::kBiasStore>(a, stream);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (a.bn == kPairTile) {
     if ((a.N % 256) != 0) return cudaErrorInvalidValue;
     switch (a.epi) {

@@ -29,6 +29,44 @@ struct SplitShape {
 // Device status codes written by kernels (first failure wins).
 constexpr int kStatusWaitTimeout = 1;
 
+// ---- programmatic dependent launch ----
+// The kernels of a forward are launched with programmatic stream
+// serialization: a kernel may start while the previous kernel on the stream is
+// still running.  It sets up what needs no memory the predecessor may touch
+// (barriers, TMEM, tensor-map prefetch), then pdl_wait() returns once the
+// predecessor has completed and its writes are visible; pdl_trigger() lets the
+// successor begin launching (every kernel calls it only after taking its TMEM,
+// so that a successor cannot hold TMEM a running kernel still has to allocate).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// False when ENC_NO_PDL=1 (plain stream order, for comparison runs).
+bool pdl_enabled();
+
+// <<<grid, block, smem, stream>>> with programmatic stream serialization
+// (unless disabled); extra launch attributes (e.g. a cluster shape) may be
+// passed in `extra`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          const cudaLaunchAttribute* extra, int num_extra, Args... args) {
+  cudaLaunchAttribute attrs[4];
+  int n = 0;
+  for (int i = 0; i < num_extra && n < 3; ++i) attrs[n++] = extra[i];
+  if (pdl_enabled()) {
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---- FP16 tensor-core GEMM (tcgen05 + TMEM + TMA), gemm_tc.cu ----
 // TcGemmArgs::bn selects the tile: 128 or 256 (one CTA, 128 x bn), or kPairTile
 // (a 2-CTA cluster per 256 x 256 tile; B map box of 128 rows; N % 256 == 0).
@@ -48,7 +86,15 @@ struct TcGemmArgs {
   int* status;                 // device status word
   int num_sms;
   const int* m_dev = nullptr;  // optional device row count (<= M): rows past it are neither computed nor stored
+  // Split-K (bn == 128 only): a cluster of `splits` CTAs shares each 128 x 128
+  // tile, CTA r taking the r-th of `splits` balanced ranges of the k-blocks;
+  // the partial sums meet in the cluster's shared memory (no global scratch).
+  int splits = 1;
 };
+// The split count for a GEMM of `tiles` 128 x 128 tiles and `num_kb` 64-wide
+// k-blocks: the largest s <= min(16, num_kb) whose clusters of s CTAs all fit
+// on the GPU at once with tiles * s <= num_sms; 1 when no s >= 2 does.
+int choose_gemm_splits(int tiles, int num_kb, int num_sms);
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream);
 
 // Encode a 2-D K-major FP16 tensor map over [rows, cols=K] with a {64, box_rows} box.

@@ -102,11 +102,13 @@ __global__ void __launch_bounds__(kLnWarps * 32)
   constexpr int E = Vec<T>::kN;
   extern __shared__ __align__(16) uint8_t params_raw[];   // [3][H] of T: bias, gamma, beta
   T* params = reinterpret_cast<T*>(params_raw);
-  for (int i = threadIdx.x * 4; i < H; i += blockDim.x * 4) {
+  for (int i = threadIdx.x * 4; i < H; i += blockDim.x * 4) {   // parameters: written by no kernel
     store_param4<T>(params + i, *reinterpret_cast<const float4*>(bias + i));
     store_param4<T>(params + H + i, *reinterpret_cast<const float4*>(gamma + i));
     store_param4<T>(params + 2 * H + i, *reinterpret_cast<const float4*>(beta + i));
   }
+  pdl_wait();                                   // the rows of the previous kernels are visible
+  pdl_trigger();
   __syncthreads();
   const T* sb = params;
   const T* sg = params + H;
@@ -198,6 +200,8 @@ __global__ void __launch_bounds__(128)
                                     const __half* __restrict__ beta, __half* __restrict__ out, int rows, int H,
                                     const int* __restrict__ rows_dev) {
   constexpr int E = 8;
+  pdl_wait();                                   // the rows of the previous kernels are visible
+  pdl_trigger();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (rows_dev) rows = min(rows, *rows_dev);   // packed tokens: the row count lives on the device
@@ -271,9 +275,8 @@ cudaError_t launch_ln(const T* a, const float* bias, const T* resid, const float
   if (vpt <= V) {                                                                                      \
     const int cap = blocks_per_sm((const void*)bias_residual_ln_kernel<T, V>, smem) * device_sm_count(); \
     const dim3 grid(want < cap ? want : cap);                                                          \
-    bias_residual_ln_kernel<T, V><<<grid, kLnWarps * 32, smem, stream>>>(a, bias, resid, gamma, beta,   \
-                                                                        out, rows, H);                 \
-    return cudaGetLastError();                                                                         \
+    return launch_kernel(bias_residual_ln_kernel<T, V>, grid, dim3(kLnWarps * 32), smem, stream, nullptr, \
+                         0, a, bias, resid, gamma, beta, out, rows, H);                                \
   }
   ENC_LN_CASE(1)
   ENC_LN_CASE(2)
@@ -295,9 +298,8 @@ cudaError_t launch_bias_residual_ln_f16h(const __half* a, const __half* bias, co
   const dim3 grid((rows + 3) / 4);
 #define ENC_LN_ROW_CASE(V)                                                                                  \
   if (vpt <= V) {                                                                                           \
-    bias_residual_ln_rowwarp_kernel<V><<<grid, 128, 0, stream>>>(a, bias, resid, gamma, beta, out, rows, hidden, \
-                                                                 rows_dev);                                  \
-    return cudaGetLastError();                                                                              \
+    return launch_kernel(bias_residual_ln_rowwarp_kernel<V>, grid, dim3(128), 0, stream, nullptr, 0, a, bias,   \
+                         resid, gamma, beta, out, rows, hidden, rows_dev);                                  \
   }
   ENC_LN_ROW_CASE(1)
   ENC_LN_ROW_CASE(2)

@@ -21,6 +21,8 @@ constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads)
     valid_offsets_kernel(const int32_t* __restrict__ valid_len, int batch, int seq, int32_t* __restrict__ offsets) {
   __shared__ int warp_tot[kScanThreads / 32];
+  pdl_wait();
+  pdl_trigger();
   const int per = (batch + kScanThreads - 1) / kScanThreads;
   const int b0 = threadIdx.x * per;
   const int b1 = min(b0 + per, batch);
@@ -58,6 +60,8 @@ template <bool PACK>
 __global__ void __launch_bounds__(128)
     move_rows_kernel(const __half* __restrict__ src, const int32_t* __restrict__ valid_len,
                      const int32_t* __restrict__ offsets, __half* __restrict__ dst, int batch, int seq, int hidden) {
+  pdl_wait();
+  pdl_trigger();
   const long tok = (long)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= (long)batch * seq) return;
@@ -85,26 +89,24 @@ __global__ void __launch_bounds__(128)
 cudaError_t launch_valid_offsets(const int32_t* valid_len, int batch, int seq, int32_t* offsets,
                                  cudaStream_t stream) {
   if (batch <= 0 || seq <= 0) return cudaErrorInvalidValue;
-  valid_offsets_kernel<<<1, kScanThreads, 0, stream>>>(valid_len, batch, seq, offsets);
-  return cudaGetLastError();
+  return launch_kernel(valid_offsets_kernel, dim3(1), dim3(kScanThreads), 0, stream, nullptr, 0, valid_len, batch, seq,
+                       offsets);
 }
 
 cudaError_t launch_pack_rows(const __half* x, const int32_t* valid_len, const int32_t* offsets, __half* xp,
                              int batch, int seq, int hidden, cudaStream_t stream) {
   if (batch <= 0 || seq <= 0 || hidden % 8 != 0) return cudaErrorInvalidValue;
   const long tokens = (long)batch * seq;
-  move_rows_kernel<true><<<(unsigned)((tokens + 3) / 4), 128, 0, stream>>>(x, valid_len, offsets, xp, batch, seq,
-                                                                          hidden);
-  return cudaGetLastError();
+  return launch_kernel(move_rows_kernel<true>, dim3((unsigned)((tokens + 3) / 4)), dim3(128), 0, stream, nullptr, 0, x,
+                       valid_len, offsets, xp, batch, seq, hidden);
 }
 
 cudaError_t launch_unpack_rows(const __half* yp, const int32_t* valid_len, const int32_t* offsets, __half* out,
                                int batch, int seq, int hidden, cudaStream_t stream) {
   if (batch <= 0 || seq <= 0 || hidden % 8 != 0) return cudaErrorInvalidValue;
   const long tokens = (long)batch * seq;
-  move_rows_kernel<false><<<(unsigned)((tokens + 3) / 4), 128, 0, stream>>>(yp, valid_len, offsets, out, batch,
-                                                                           seq, hidden);
-  return cudaGetLastError();
+  return launch_kernel(move_rows_kernel<false>, dim3((unsigned)((tokens + 3) / 4)), dim3(128), 0, stream, nullptr, 0,
+                       yp, valid_len, offsets, out, batch, seq, hidden);
 }
 
 }  // namespace enc

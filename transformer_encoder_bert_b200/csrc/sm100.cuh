@@ -300,6 +300,16 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
+// 16-byte load from another CTA's shared memory (address from mapa_shared).
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
 // ---- packed FP32 pairs (sm_100 .f32x2 arithmetic) ------------------------
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
