@@ -2,16 +2,19 @@
 """Throughput of the BERT-style encoder forward on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload KIND:BATCH[:SEQ]] [--graph] [--no-cpu-baseline]
+                    [--workload KIND:BATCH[:SEQ]] [--no-graph] [--packed] [--no-cpu-baseline]
 
-A step is one enc_forward over one batch of the workload (every layer, every
-kernel of the path), inputs already in HBM; the L2 is flushed (256 MiB write)
+A step is one forward over one batch of the workload (every layer, every kernel
+of the path; by default one replay of the recorded forward, enc_graph_launch,
+else one enc_forward call), inputs already in HBM; the L2 is flushed (256 MiB write)
 before every timed step.  value = sequences/s over all ranks (weak scaling:
 each rank runs its own batch; no collective on the data path).  e2e = the same
-metric through enc_forward_host (pinned host input, copies inside the timed
-region).  The per-kernel breakdown and the roofline come from CUDA events the
-library records between its kernels on the launching stream, during the timed
-steps.  --impl reference times the float64 CPU oracle on a bounded sample.
+metric through enc_forward_host_async: every step copies its input from pinned
+host memory and its output back inside the timed region, consecutive steps
+overlapping their copies with the encoder.  The per-kernel breakdown and the
+roofline come from CUDA events the library records between its kernels on the
+launching stream: during the timed steps with --no-graph, else in as many traced
+enc_forward calls right after them (a recorded forward carries no events).  --impl reference times the float64 CPU oracle on a bounded sample.
 Default workload: 12-layer BERT-Base shape (12x64, FFN 3072), seq 32, batch 512.
 """
 from __future__ import annotations
@@ -294,24 +297,27 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         for j in range(nk):
             per_kernel[names[j]].append(evs[j].elapsed_time(evs[j + 1]))
 
-    # e2e through enc_forward_host: pinned host input, copies inside the timed region.
+    # e2e through the pipelined host entry point (enc_forward_host_async): every
+    # step copies its input from pinned host memory and its output back to host
+    # memory inside the timed region; consecutive steps overlap their copies with
+    # the encoder.  Timed over all steps, from before the first input copy to
+    # after the last output copy (enc_host_join).
     hx = torch.from_numpy(inp.x).pin_memory()
     hvl = torch.from_numpy(inp.valid_len).pin_memory()
     hout = torch.empty_like(hx).pin_memory()
     for _ in range(2):
         enc.forward_host_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), wl.batch, wl.seq)
-    e2e_ms = []
     barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
     for i in range(args.steps):
         flush.zero_()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record(stream)
-        enc.forward_host_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), wl.batch, wl.seq)
-        e.record(stream)
-        e.synchronize()
-        e2e_ms.append(s.elapsed_time(e))
+        enc.forward_host_async_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), wl.batch, wl.seq)
+    enc.host_join()
+    e.record(stream)
+    e.synchronize()
     barrier()
-    e2e_step = sum(e2e_ms) / len(e2e_ms)
+    e2e_step = s.elapsed_time(e) / args.steps
     status = enc.device_status()
     if graph is not None:
         graph.close()
@@ -390,8 +396,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--packed", action="store_true",
                     help="padding removal (enc_set_packing): compute the valid tokens only")
-    ap.add_argument("--graph", action="store_true",
-                    help="time replays of a recorded forward (enc_graph_launch) instead of enc_forward calls")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="time replays of a recorded forward (enc_graph_launch); the default")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time enc_forward calls instead of graph replays")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-sample", type=int, default=8, help="sequences per reference-arm step")
     ap.add_argument("--traffic", type=float, default=None,

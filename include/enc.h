@@ -150,6 +150,24 @@ ENC_API enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len,
 ENC_API enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, void* out,
                             int batch, int seq, enc_stream_t stream);
 
+/* enc_forward_host_async - enc_forward_host for a stream of batches: returns
+ * once the work is enqueued, without synchronising.  Consecutive calls use two
+ * handle-owned device staging slots in turn, so that the input copy of call
+ * i+1 and the output copy of call i overlap the encoder runs (copies on two
+ * handle-owned streams, the encoder on `stream`).  Host buffers should be
+ * pinned; the caller keeps x and valid_len unchanged and out untouched until
+ * the call's copies are done, which enc_host_join makes `stream` wait for.
+ * Calls of one handle must use one `stream`.  Same arguments and errors as
+ * enc_forward_host.  Not part of the source pages' design (they describe the
+ * device computation only): it serves throughput from host memory. */
+ENC_API enc_status enc_forward_host_async(enc_t h, const void* x, const int32_t* valid_len, void* out,
+                                          int batch, int seq, enc_stream_t stream);
+
+/* enc_host_join - make `stream` wait until every copy enqueued by earlier
+ * enc_forward_host_async calls has completed (no host synchronisation).  After
+ * `stream` reaches that point the outputs are in host memory. */
+ENC_API enc_status enc_host_join(enc_t h, enc_stream_t stream);
+
 /* enc_reserve - grow the workspace to hold batch*seq tokens now (synchronous). */
 ENC_API enc_status enc_reserve(enc_t h, int batch, int seq);
 

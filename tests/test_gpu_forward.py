@@ -239,6 +239,32 @@ def test_host_entry_point_chunked_pipeline_matches_device_forward(chunks, layers
     assert np.array_equal(pageable, dev)
 
 
+def test_pipelined_host_entry_point_matches_device_forward():
+    """enc_forward_host_async: four different batches in flight through the two
+    staging slots (each call's input copy and the previous call's output copy
+    overlap the encoder); every output equals the device forward bit for bit,
+    and a synchronous host call after them sees the slots free."""
+    import torch
+    wl = EI.named_workload("bert-base-s32", 64)
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    batches = [EI.make_inputs(wl.with_(shape=sh, seed=100 + i)) for i in range(4)]
+    enc = encoder_from_inputs(batches[0])        # one set of weights; x and valid_len differ per batch
+    refs = [to_host(enc.forward(to_dev(b.x), to_dev(b.valid_len))) for b in batches]
+    hx = [torch.from_numpy(b.x).pin_memory() for b in batches]
+    hvl = [torch.from_numpy(b.valid_len).pin_memory() for b in batches]
+    hout = [torch.zeros_like(t).pin_memory() for t in hx]
+    stream = torch.cuda.current_stream()
+    for i in range(4):
+        enc.forward_host_async_ptr(hx[i].data_ptr(), hvl[i].data_ptr(), hout[i].data_ptr(), 64, 32)
+    enc.host_join()
+    stream.synchronize()
+    for i in range(4):
+        assert np.array_equal(hout[i].numpy(), refs[i]), i
+    again = enc.forward_host(batches[1].x, batches[1].valid_len)
+    assert np.array_equal(again, refs[1])
+    assert enc.device_status() == 0
+
+
 # ---------------------------------------------------------------- padding removal
 
 @pytest.mark.parametrize("seq,lo,hi,L", [(32, 1, 32, 12), (37, 0, 37, 2), (96, 64, 96, 2), (128, 64, 128, 2),

@@ -30,6 +30,8 @@ SIGNATURES = {
     "enc_create": (_i, [_i, _i, _i, _i, _i, _vp, ctypes.POINTER(_vp)]),
     "enc_forward": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "enc_forward_host": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
+    "enc_forward_host_async": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
+    "enc_host_join": (_i, [_vp, _vp]),
     "enc_reserve": (_i, [_vp, _i, _i]),
     "enc_workspace_bytes": (_sz, [_vp, _i, _i]),
     "enc_destroy": (_i, [_vp]),
@@ -198,6 +200,15 @@ class Encoder:
         """enc_forward_host on raw host pointers (e.g. pinned torch tensors)."""
         _check(self.lib.enc_forward_host(self.handle, x_ptr, vl_ptr, out_ptr, batch, seq,
                                          _current_stream(stream)))
+
+    def forward_host_async_ptr(self, x_ptr: int, vl_ptr: int, out_ptr: int, batch: int, seq: int, stream=None):
+        """enc_forward_host_async on raw (pinned) host pointers; see host_join."""
+        _check(self.lib.enc_forward_host_async(self.handle, x_ptr, vl_ptr, out_ptr, batch, seq,
+                                               _current_stream(stream)))
+
+    def host_join(self, stream=None):
+        """Make the stream wait for every copy of earlier forward_host_async calls."""
+        _check(self.lib.enc_host_join(self.handle, _current_stream(stream)))
 
     def record(self, x, valid_len, out) -> "RecordedForward":
         """Record one forward on these CUDA tensors as a CUDA graph (see enc_graph_create)."""

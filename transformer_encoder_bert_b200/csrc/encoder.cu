@@ -103,6 +103,10 @@ struct enc_handle {
   cudaStream_t copy_out = nullptr;  // enc_forward_host: device-to-host copies
   static constexpr int kMaxChunks = 4;
   cudaEvent_t ev_in[kMaxChunks] = {}, ev_done[kMaxChunks] = {}, ev_out = nullptr, ev_start = nullptr;
+  // enc_forward_host_async: two staging slots used in turn; per slot, its input
+  // copy landed, its encoder run done, its output copy done (slot free again).
+  int host_slot = 0;
+  cudaEvent_t ev_slot_in[2] = {}, ev_slot_done[2] = {}, ev_slot_free[2] = {};
   int* status = nullptr;
   uint64_t launches = 0;            // kernels launched through this handle
   int graphs_alive = 0;             // recorded forwards that reference the workspace
@@ -339,6 +343,11 @@ void free_handle(enc_handle* h) {
   }
   if (h->ev_out) cudaEventDestroy(h->ev_out);
   if (h->ev_start) cudaEventDestroy(h->ev_start);
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_slot_in[i]) cudaEventDestroy(h->ev_slot_in[i]);
+    if (h->ev_slot_done[i]) cudaEventDestroy(h->ev_slot_done[i]);
+    if (h->ev_slot_free[i]) cudaEventDestroy(h->ev_slot_free[i]);
+  }
   if (h->copy_in) cudaStreamDestroy(h->copy_in);
   if (h->copy_out) cudaStreamDestroy(h->copy_out);
   if (h->param_block) cudaFree(h->param_block);
@@ -346,6 +355,48 @@ void free_handle(enc_handle* h) {
   if (h->stage) cudaFree(h->stage);
   if (h->status) cudaFree(h->status);
   delete h;
+}
+
+// Device staging for the host entry points: two slots of {x, out, valid_len}
+// for a batch*seq-token run (slot 0 serves enc_forward_host), plus the copy
+// streams and events.  Growing the staging synchronises the device.
+size_t host_slot_bytes(const enc_handle* h, int batch, int seq) {
+  const size_t act_al = align_up((size_t)batch * seq * h->H * h->esize, 256);
+  return 2 * act_al + align_up((size_t)batch * 4, 256);
+}
+
+enc_status host_setup(enc_handle* h, int batch, int seq) {
+  const size_t need = 2 * host_slot_bytes(h, batch, seq);
+  if (need > h->stage_bytes) {
+    if (h->stage) {
+      cudaDeviceSynchronize();
+      cudaFree(h->stage);
+      h->stage = nullptr;
+      h->stage_bytes = 0;
+    }
+    if (cudaMalloc(&h->stage, need) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ENC_ERR_OOM, "staging allocation of %zu bytes failed", need);
+    }
+    h->stage_bytes = need;
+  }
+  if (!h->copy_in) {
+    cudaError_t e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
+    for (int i = 0; i < enc_handle::kMaxChunks && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
+    }
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&h->ev_slot_in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_slot_done[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_slot_free[i], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "copy stream setup");
+  }
+  return ENC_OK;
 }
 
 }  // namespace
@@ -730,33 +781,8 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if (!x || !valid_len || !out) return fail(ENC_ERR_INVALID_ARG, "null host buffer");
   const size_t seq_bytes = (size_t)seq * h->H * h->esize;
-  const size_t act = (size_t)batch * seq_bytes;
-  const size_t act_al = align_up(act, 256);
-  const size_t need = 2 * act_al + align_up((size_t)batch * 4, 256);
-  if (need > h->stage_bytes) {
-    if (h->stage) {
-      cudaDeviceSynchronize();
-      cudaFree(h->stage);
-      h->stage = nullptr;
-      h->stage_bytes = 0;
-    }
-    if (cudaMalloc(&h->stage, need) != cudaSuccess) {
-      cudaGetLastError();
-      return fail(ENC_ERR_OOM, "staging allocation of %zu bytes failed", need);
-    }
-    h->stage_bytes = need;
-  }
-  if (!h->copy_in) {
-    cudaError_t e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
-    for (int i = 0; i < enc_handle::kMaxChunks && e == cudaSuccess; ++i) {
-      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
-    }
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming);
-    if (e != cudaSuccess) return cuda_fail(e, "copy stream setup");
-  }
+  const size_t act_al = align_up((size_t)batch * seq_bytes, 256);
+  if ((s = host_setup(h, batch, seq)) != ENC_OK) return s;
   // Sequences are independent, so the batch can be cut into chunks: the first
   // layer runs chunk by chunk as each chunk's input lands, the middle layers
   // run on the whole batch, and the last layer runs chunk by chunk so that each
@@ -774,10 +800,12 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const char* hx = static_cast<const char*>(x);
   char* hout = static_cast<char*>(out);
-  // Copies start after the caller's earlier work on `st` (the staging buffers may be in use).
+  // Copies start after the caller's earlier work on `st` and after any output
+  // copy of enc_forward_host_async still reading the staging.
   cudaError_t e = cudaEventRecord(h->ev_start, st);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_in, h->ev_start, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_start, 0);
+  for (int k = 0; k < 2 && e == cudaSuccess; ++k) e = cudaStreamWaitEvent(h->copy_in, h->ev_slot_free[k], 0);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dvl, valid_len, (size_t)batch * 4, cudaMemcpyHostToDevice, h->copy_in);
   if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
   int cb[enc_handle::kMaxChunks + 1];
@@ -833,6 +861,48 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->ev_out, 0);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return ok();
+}
+
+enc_status enc_forward_host_async(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                                  enc_stream_t stream) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if (!x || !valid_len || !out) return fail(ENC_ERR_INVALID_ARG, "null host buffer");
+  if ((s = host_setup(h, batch, seq)) != ENC_OK) return s;
+  const int k = h->host_slot;
+  const size_t act = (size_t)batch * seq * h->H * h->esize;
+  const size_t act_al = align_up(act, 256);
+  char* base = static_cast<char*>(h->stage) + (size_t)k * host_slot_bytes(h, batch, seq);
+  char* dx = base;
+  char* dout = base + act_al;
+  int32_t* dvl = reinterpret_cast<int32_t*>(base + 2 * act_al);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The slot's previous run (two calls ago) has copied its output out.
+  cudaError_t e = cudaStreamWaitEvent(h->copy_in, h->ev_slot_free[k], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dvl, valid_len, (size_t)batch * 4, cudaMemcpyHostToDevice, h->copy_in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dx, x, act, cudaMemcpyHostToDevice, h->copy_in);
+  if (e == cudaSuccess) e = cudaEventRecord(h->ev_slot_in[k], h->copy_in);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->ev_slot_in[k], 0);
+  if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  if ((s = forward_impl(h, dx, dvl, dout, batch, seq, st, false)) != ENC_OK) return s;
+  e = cudaEventRecord(h->ev_slot_done[k], st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_slot_done[k], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(out, dout, act, cudaMemcpyDeviceToHost, h->copy_out);
+  if (e == cudaSuccess) e = cudaEventRecord(h->ev_slot_free[k], h->copy_out);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  h->host_slot = k ^ 1;
+  return ok();
+}
+
+enc_status enc_host_join(enc_t h, enc_stream_t stream) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if (!h->copy_out) return ok();                       // no host call yet
+  cudaError_t e = cudaEventRecord(h->ev_out, h->copy_out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(stream), h->ev_out, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "join");
   return ok();
 }
 
