@@ -82,11 +82,11 @@ def kernel_work(wl: EI.Workload, attn_seq=None, attn_tokens=None):
     return {
         "qkv_gemm": gemm(3 * H, H),
         "attention": (4.0 * M * S * H, es * 4.0 * M * H + 4 * wl.batch),
-        "out_proj_gemm": gemm(H, H),
-        "ln1": (0.0, es * 3.0 * M * H),
+        "out_proj_gemm": gemm(H, H, extra_out=es * M * H),     # epilogue reads the residual
+        "ln1": (0.0, es * 2.0 * M * H),                       # z in, normalised row out
         "ffn1_gemm": gemm(F, H),
-        "ffn2_gemm": gemm(H, F),
-        "ln2": (0.0, es * 3.0 * M * H),
+        "ffn2_gemm": gemm(H, F, extra_out=es * M * H),
+        "ln2": (0.0, es * 2.0 * M * H),
     }
 
 

@@ -248,27 +248,31 @@ ENC_API enc_status enc_op_qkv(enc_t h, int layer, const void* x, void* qkv, int 
 ENC_API enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, void* ctx,
                             int batch, int seq, enc_stream_t stream);
 
-/* Step output projection without its bias (the bias is added by the next step):
- *   a = ctx Wo,  ctx: [M, H], a: [M, H]. */
-ENC_API enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, void* a, int tokens,
-                           enc_stream_t stream);
+/* Step output projection with the add-bias and residual of the first
+ * add-bias + residual + LayerNorm ([FT] "Faster Transformer 优化原理") done in
+ * the GEMM epilogue:
+ *   z = ctx Wo + bo + resid,  ctx, resid, z: [M, H]  (resid = the layer input). */
+ENC_API enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, const void* resid, void* z,
+                                   int tokens, enc_stream_t stream);
 
-/* Step add-bias + residual + LayerNorm ([FT] "Faster Transformer 优化原理"):
- *   which = 1: out = LN(resid + a + bo; ln1_g, ln1_b)
- *   which = 2: out = LN(resid + a + b2; ln2_g, ln2_b)
- *   a, resid, out: [tokens, H]. */
-ENC_API enc_status enc_op_bias_residual_layernorm(enc_t h, int layer, int which, const void* a,
-                                          const void* resid, void* out, int tokens,
-                                          enc_stream_t stream);
+/* Step LayerNorm of a row that already holds bias + residual (the rest of the
+ * page's add-bias + residual + LayerNorm kernel):
+ *   which = 1: out = LN(z; ln1_g, ln1_b);  which = 2: out = LN(z; ln2_g, ln2_b)
+ *   z, out: [tokens, H]; mean and biased variance over H, eps 1e-12. */
+ENC_API enc_status enc_op_layernorm(enc_t h, int layer, int which, const void* z, void* out, int tokens,
+                                    enc_stream_t stream);
 
 /* Step FFN1 + add-bias + GELU (erf form) fused in the GEMM epilogue:
  *   u = GELU(h1 W1 + b1),  h1: [tokens, H], u: [tokens, F]. */
 ENC_API enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens,
                        enc_stream_t stream);
 
-/* Step FFN2 without its bias (added by the next step):  y = u W2,  u: [tokens, F], y: [tokens, H]. */
-ENC_API enc_status enc_op_ffn2(enc_t h, int layer, const void* u, void* y, int tokens,
-                       enc_stream_t stream);
+/* Step FFN2 with the add-bias and residual of the second add-bias + residual +
+ * LayerNorm done in the GEMM epilogue:
+ *   z = u W2 + b2 + resid,  u: [tokens, F], resid, z: [tokens, H]  (resid = h1,
+ *   the first LayerNorm's output). */
+ENC_API enc_status enc_op_ffn2(enc_t h, int layer, const void* u, const void* resid, void* z, int tokens,
+                               enc_stream_t stream);
 
 #ifdef __cplusplus
 }

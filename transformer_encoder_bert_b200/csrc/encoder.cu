@@ -80,8 +80,7 @@ struct LayerDev {
   float *ln1_g = nullptr, *ln1_b = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
   // FP16 copies (FP16 mode only; exact, the caller supplied halves) for the LayerNorm kernel:
   // b_o, ln1_g, ln1_b, b_ff2, ln2_g, ln2_b.
-  __half *h_b_o = nullptr, *h_ln1_g = nullptr, *h_ln1_b = nullptr, *h_b_ff2 = nullptr, *h_ln2_g = nullptr,
-         *h_ln2_b = nullptr;
+  __half *h_ln1_g = nullptr, *h_ln1_b = nullptr, *h_ln2_g = nullptr, *h_ln2_b = nullptr;
   CUtensorMap tm_qkv[2], tm_o[2], tm_ff1[2], tm_ff2[2];   // [0]: 128-row box, [1]: 256-row box
 };
 
@@ -208,7 +207,7 @@ int choose_splits(const enc_handle* h, int M, int N, int K, int bn) {
 // One GEMM step: C = A * W (+ epilogue), dispatched on the handle's dtype.
 enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const CUtensorMap* wmaps, int N,
                     enc::Epi epi, const float* bias, void* C, enc::SplitShape sp, cudaStream_t st,
-                    const int* m_dev = nullptr) {
+                    const int* m_dev = nullptr, const void* resid = nullptr) {
   if (h->dtype == ENC_FP16) {
     const int bn = choose_bn(h, M, N);
     CUtensorMap ta;
@@ -224,9 +223,15 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
       else
         use_tc = enc::encode_output_map_2d(&tc, C, (uint64_t)M, (uint64_t)N);
     }
+    // The residual of kBiasResidStore comes in by TMA in the same 32x32 boxes
+    // the output leaves in (only with TMA stores).
+    CUtensorMap tr;
+    const bool use_tr = use_tc && epi == enc::Epi::kBiasResidStore && resid &&
+                        enc::encode_output_map_2d(&tr, const_cast<void*>(resid), (uint64_t)M, (uint64_t)N);
     enc::TcGemmArgs a;
     a.tmap_a = &ta;
     a.tmap_c = use_tc ? &tc : nullptr;
+    a.tmap_r = use_tr ? &tr : nullptr;
     a.tmap_b = &wmaps[bn == 256 ? 1 : 0];      // the pair tile loads 128-row halves of B
     a.M = M; a.N = N; a.K = K; a.bn = bn; a.epi = epi; a.bias = bias;
     a.c = static_cast<__half*>(C);
@@ -235,12 +240,13 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
     a.num_sms = h->num_sms;
     a.m_dev = m_dev;
     a.splits = choose_splits(h, M, N, K, bn);
+    a.resid = static_cast<const __half*>(resid);
     cudaError_t e = enc::launch_gemm_tc(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
     ++h->launches;
   } else {
     cudaError_t e = enc::launch_gemm_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K,
-                                         epi, bias, static_cast<float*>(C), sp, st);
+                                         epi, bias, static_cast<float*>(C), sp, st, static_cast<const float*>(resid));
     if (e != cudaSuccess) return cuda_fail(e, "FP32 GEMM launch");
     ++h->launches;
   }
@@ -278,32 +284,30 @@ enc_status step_attention(enc_handle* h, const void* qkv, const int32_t* vl, voi
   return ENC_OK;
 }
 
-enc_status step_out_proj(enc_handle* h, int l, const void* ctx, void* a, int tokens, cudaStream_t st) {
+// Output projection with add-bias and residual in the epilogue:
+// z = ctx Wo + bo + resid (resid = the layer input).
+enc_status step_out_proj(enc_handle* h, int l, const void* ctx, const void* resid, void* z, int tokens,
+                         cudaStream_t st, const int* m_dev = nullptr) {
   LayerDev& L = h->layers[l];
-  return run_gemm(h, ctx, tokens, h->H, L.w_o, L.tm_o, h->H, enc::Epi::kStore, nullptr, a, {}, st);
+  return run_gemm(h, ctx, tokens, h->H, L.w_o, L.tm_o, h->H, enc::Epi::kBiasResidStore, L.b_o, z, {}, st, m_dev,
+                  resid);
 }
 
-enc_status step_ln(enc_handle* h, int l, int which, const void* a, const void* resid, void* out, int tokens,
-                   cudaStream_t st) {
+// LayerNorm `which` (1 or 2) of z (bias and residual already added).
+enc_status step_ln(enc_handle* h, int l, int which, const void* z, void* out, int tokens, cudaStream_t st,
+                   const int* rows_dev = nullptr) {
   LayerDev& L = h->layers[l];
-  const float* bias = which == 1 ? L.b_o : L.b_ff2;
-  const float* g = which == 1 ? L.ln1_g : L.ln2_g;
-  const float* b = which == 1 ? L.ln1_b : L.ln2_b;
   cudaError_t e;
-#ifndef ENC_LN_SMEM
   if (h->dtype == ENC_FP16 && h->H <= 1024)
-    e = enc::launch_bias_residual_ln_f16h(static_cast<const __half*>(a), which == 1 ? L.h_b_o : L.h_b_ff2,
-                                          static_cast<const __half*>(resid), which == 1 ? L.h_ln1_g : L.h_ln2_g,
-                                          which == 1 ? L.h_ln1_b : L.h_ln2_b, static_cast<__half*>(out), tokens,
-                                          h->H, st);
+    e = enc::launch_layernorm_f16h(static_cast<const __half*>(z), which == 1 ? L.h_ln1_g : L.h_ln2_g,
+                                   which == 1 ? L.h_ln1_b : L.h_ln2_b, static_cast<__half*>(out), tokens, h->H, st,
+                                   rows_dev);
+  else if (h->dtype == ENC_FP16)
+    e = enc::launch_layernorm_f16(static_cast<const __half*>(z), which == 1 ? L.ln1_g : L.ln2_g,
+                                  which == 1 ? L.ln1_b : L.ln2_b, static_cast<__half*>(out), tokens, h->H, st);
   else
-#endif
-  if (h->dtype == ENC_FP16)
-    e = enc::launch_bias_residual_ln_f16(static_cast<const __half*>(a), bias, static_cast<const __half*>(resid),
-                                         g, b, static_cast<__half*>(out), tokens, h->H, st);
-  else
-    e = enc::launch_bias_residual_ln_f32(static_cast<const float*>(a), bias, static_cast<const float*>(resid), g,
-                                         b, static_cast<float*>(out), tokens, h->H, st);
+    e = enc::launch_layernorm_f32(static_cast<const float*>(z), which == 1 ? L.ln1_g : L.ln2_g,
+                                  which == 1 ? L.ln1_b : L.ln2_b, static_cast<float*>(out), tokens, h->H, st);
   if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
   ++h->launches;
   return ENC_OK;
@@ -315,9 +319,13 @@ enc_status step_ffn1(enc_handle* h, int l, const void* h1, void* u, int tokens, 
   return run_gemm(h, h1, tokens, h->H, L.w_ff1, L.tm_ff1, h->F, epi, L.b_ff1, u, {}, st);
 }
 
-enc_status step_ffn2(enc_handle* h, int l, const void* u, void* y, int tokens, cudaStream_t st) {
+// FFN2 with add-bias and residual in the epilogue: z = u W2 + b2 + resid
+// (resid = the first LayerNorm's output).
+enc_status step_ffn2(enc_handle* h, int l, const void* u, const void* resid, void* z, int tokens, cudaStream_t st,
+                     const int* m_dev = nullptr) {
   LayerDev& L = h->layers[l];
-  return run_gemm(h, u, tokens, h->F, L.w_ff2, L.tm_ff2, h->H, enc::Epi::kStore, nullptr, y, {}, st);
+  return run_gemm(h, u, tokens, h->F, L.w_ff2, L.tm_ff2, h->H, enc::Epi::kBiasResidStore, L.b_ff2, z, {}, st, m_dev,
+                  resid);
 }
 
 enc_status check_tokens(int batch, int seq) {
@@ -473,7 +481,7 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   size_t per_layer = 0;
   for (size_t s : wsz) per_layer += align_up(s * es, 256);
   for (size_t s : vsz) per_layer += align_up(s * 4, 256);
-  if (dtype == ENC_FP16) per_layer += 6 * align_up((size_t)H * 2, 256);
+  if (dtype == ENC_FP16) per_layer += 4 * align_up((size_t)H * 2, 256);
   size_t staging = 0;
   for (size_t s : wsz) staging = std::max(staging, align_up(s * es, 256));
   if (cudaMalloc(&h->param_block, per_layer * num_layers + staging) != cudaSuccess) {
@@ -529,9 +537,9 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
       p += align_up(n * 4, 256);
     }
     if (dtype == ENC_FP16) {
-      const void* hsrc[6] = {w.b_o, w.ln1_g, w.ln1_b, w.b_ff2, w.ln2_g, w.ln2_b};
-      __half** hdst[6] = {&L.h_b_o, &L.h_ln1_g, &L.h_ln1_b, &L.h_b_ff2, &L.h_ln2_g, &L.h_ln2_b};
-      for (int i = 0; i < 6; ++i) {
+      const void* hsrc[4] = {w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b};
+      __half** hdst[4] = {&L.h_ln1_g, &L.h_ln1_b, &L.h_ln2_g, &L.h_ln2_b};
+      for (int i = 0; i < 4; ++i) {
         *hdst[i] = reinterpret_cast<__half*>(p);
         cudaError_t e = cudaMemcpy(p, hsrc[i], (size_t)H * 2, cudaMemcpyDefault);
         if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "parameter upload"); }
@@ -614,24 +622,16 @@ enc_status forward_packed(enc_handle* h, const void* x, const int32_t* valid_len
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     ++h->launches;
     mark();
-    if ((s = run_gemm(h, w.ctx, M, H, L.w_o, L.tm_o, H, enc::Epi::kStore, nullptr, w.a, {}, st, T)) != ENC_OK)
-      return s;
+    if ((s = step_out_proj(h, l, w.ctx, xin, w.a, M, st, T)) != ENC_OK) return s;
     mark();
-    e = enc::launch_bias_residual_ln_f16h(static_cast<const __half*>(w.a), L.h_b_o, static_cast<const __half*>(xin),
-                                          L.h_ln1_g, L.h_ln1_b, static_cast<__half*>(w.h1), M, H, st, T);
-    if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
-    ++h->launches;
+    if ((s = step_ln(h, l, 1, w.a, w.h1, M, st, T)) != ENC_OK) return s;
     mark();
     const enc::Epi gelu = h->gelu == ENC_GELU_TANH ? enc::Epi::kBiasGeluTanh : enc::Epi::kBiasGelu;
     if ((s = run_gemm(h, w.h1, M, H, L.w_ff1, L.tm_ff1, h->F, gelu, L.b_ff1, w.u, {}, st, T)) != ENC_OK) return s;
     mark();
-    if ((s = run_gemm(h, w.u, M, h->F, L.w_ff2, L.tm_ff2, H, enc::Epi::kStore, nullptr, w.a, {}, st, T)) != ENC_OK)
-      return s;
+    if ((s = step_ffn2(h, l, w.u, w.h1, w.a, M, st, T)) != ENC_OK) return s;
     mark();
-    e = enc::launch_bias_residual_ln_f16h(static_cast<const __half*>(w.a), L.h_b_ff2, static_cast<const __half*>(w.h1),
-                                          L.h_ln2_g, L.h_ln2_b, static_cast<__half*>(xout), M, H, st, T);
-    if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
-    ++h->launches;
+    if ((s = step_ln(h, l, 2, w.a, xout, M, st, T)) != ENC_OK) return s;
     last = xout;
   }
   mark();
@@ -655,15 +655,15 @@ enc_status run_layer(enc_handle* h, int l, const void* xin, void* xout, const in
   mark();
   if ((s = step_attention(h, w.qkv, valid_len, w.ctx, batch, seq, st)) != ENC_OK) return s;
   mark();
-  if ((s = step_out_proj(h, l, w.ctx, w.a, tokens, st)) != ENC_OK) return s;
+  if ((s = step_out_proj(h, l, w.ctx, xin, w.a, tokens, st)) != ENC_OK) return s;
   mark();
-  if ((s = step_ln(h, l, 1, w.a, xin, w.h1, tokens, st)) != ENC_OK) return s;
+  if ((s = step_ln(h, l, 1, w.a, w.h1, tokens, st)) != ENC_OK) return s;
   mark();
   if ((s = step_ffn1(h, l, w.h1, w.u, tokens, st)) != ENC_OK) return s;
   mark();
-  if ((s = step_ffn2(h, l, w.u, w.a, tokens, st)) != ENC_OK) return s;
+  if ((s = step_ffn2(h, l, w.u, w.h1, w.a, tokens, st)) != ENC_OK) return s;
   mark();
-  return step_ln(h, l, 2, w.a, w.h1, xout, tokens, st);
+  return step_ln(h, l, 2, w.a, xout, tokens, st);
 }
 
 // Checks, workspace, and the per-layer launches of one forward on `st`.
@@ -997,22 +997,23 @@ enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, 
   return ok();
 }
 
-enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, void* a, int tokens, enc_stream_t stream) {
+enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, const void* resid, void* z, int tokens,
+                           enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
-  if ((s = check_ptrs({ctx, a})) != ENC_OK) return s;
-  if ((s = step_out_proj(h, layer, ctx, a, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  if ((s = check_ptrs({ctx, resid, z})) != ENC_OK) return s;
+  if ((s = step_out_proj(h, layer, ctx, resid, z, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK)
+    return s;
   return ok();
 }
 
-enc_status enc_op_bias_residual_layernorm(enc_t h, int layer, int which, const void* a, const void* resid,
-                                          void* out, int tokens, enc_stream_t stream) {
+enc_status enc_op_layernorm(enc_t h, int layer, int which, const void* z, void* out, int tokens,
+                            enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
   if (which != 1 && which != 2) return fail(ENC_ERR_INVALID_ARG, "which must be 1 or 2");
-  if ((s = check_ptrs({a, resid, out})) != ENC_OK) return s;
-  if ((s = step_ln(h, layer, which, a, resid, out, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK)
-    return s;
+  if ((s = check_ptrs({z, out})) != ENC_OK) return s;
+  if ((s = step_ln(h, layer, which, z, out, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
   return ok();
 }
 
@@ -1024,11 +1025,12 @@ enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens, 
   return ok();
 }
 
-enc_status enc_op_ffn2(enc_t h, int layer, const void* u, void* y, int tokens, enc_stream_t stream) {
+enc_status enc_op_ffn2(enc_t h, int layer, const void* u, const void* resid, void* z, int tokens,
+                       enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
-  if ((s = check_ptrs({u, y})) != ENC_OK) return s;
-  if ((s = step_ffn2(h, layer, u, y, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  if ((s = check_ptrs({u, resid, z})) != ENC_OK) return s;
+  if ((s = step_ffn2(h, layer, u, resid, z, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
   return ok();
 }
 

@@ -17,7 +17,8 @@ template <Epi EPI>
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A,
                                                        const float* __restrict__ W, int M, int N,
                                                        int K, const float* __restrict__ bias,
-                                                       float* __restrict__ C, SplitShape sp) {
+                                                       float* __restrict__ C, SplitShape sp,
+                                                       const float* __restrict__ resid) {
   __shared__ float As[TK][TM + 4];
   __shared__ float Ws[TK][TN + 4];
   pdl_wait();
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
       if (n >= N) continue;
       float v = acc[i][j];
       if constexpr (EPI != Epi::kStore) v += bias[n];
+      if constexpr (EPI == Epi::kBiasResidStore) v += resid[(size_t)m * N + n];
       if constexpr (EPI == Epi::kBiasGelu) v = 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
       if constexpr (EPI == Epi::kBiasGeluTanh)
         v = 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)));
@@ -83,25 +85,30 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
 }  // namespace
 
 cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K, Epi epi,
-                            const float* bias, float* C, SplitShape split, cudaStream_t stream) {
+                            const float* bias, float* C, SplitShape split, cudaStream_t stream,
+                            const float* resid) {
   if (M <= 0 || N <= 0 || K <= 0) return cudaErrorInvalidValue;
   const dim3 grid((N + TN - 1) / TN, (M + TM - 1) / TM);
   switch (epi) {
     case Epi::kStore:
       return launch_kernel(gemm_f32_kernel<Epi::kStore>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
-                           C, split);
+                           C, split, resid);
     case Epi::kBiasGelu:
       return launch_kernel(gemm_f32_kernel<Epi::kBiasGelu>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
-                           C, split);
+                           C, split, resid);
     case Epi::kBiasQkvSplit:
       return launch_kernel(gemm_f32_kernel<Epi::kBiasQkvSplit>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
-                           C, split);
+                           C, split, resid);
     case Epi::kBiasGeluTanh:
       return launch_kernel(gemm_f32_kernel<Epi::kBiasGeluTanh>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
-                           C, split);
+                           C, split, resid);
     case Epi::kBiasStore:
       return launch_kernel(gemm_f32_kernel<Epi::kBiasStore>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N, K, bias,
-                           C, split);
+                           C, split, resid);
+    case Epi::kBiasResidStore:
+      if (!resid) return cudaErrorInvalidValue;
+      return launch_kernel(gemm_f32_kernel<Epi::kBiasResidStore>, grid, dim3(256), 0, stream, nullptr, 0, A, W, M, N,
+                           K, bias, C, split, resid);
   }
   return cudaErrorInvalidValue;
 }

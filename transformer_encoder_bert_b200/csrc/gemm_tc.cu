@@ -54,10 +54,12 @@ struct Cfg {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kNumBars = 2 * kStages + 5;
+  // full[kStages], empty[kStages], tfull[2], tempty[2], drain, then two residual barriers per epilogue warp
+  static constexpr int kResBar0 = 2 * kStages + 5;
+  static constexpr int kNumBars = kResBar0 + 2 * kEpiWarps;
   static constexpr int kBiasOffset = (kStages * kStageBytes + kNumBars * 8 + 16 + 15) / 16 * 16;
   static constexpr int kStoreOffset = (kBiasOffset + kEpiWarps * (BN / kEpiSlices) * 4 + 1023) / 1024 * 1024;
-  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * (32 * 32 * 2);
+  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * 2 * (32 * 32 * 2);   // two staging buffers per warp
 };
 
 // GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), with erf from the
@@ -148,12 +150,11 @@ __device__ __forceinline__ size_t col_offset(int col0, const SplitShape& sp) {
   }
 }
 
-// Epilogue math for one thread: 32 accumulator columns of one row -> 16 packed
-// half2 words.  `bias_s` holds the bias of these 32 columns (shared memory,
-// read as a broadcast).
+// Epilogue math for one thread: 32 accumulator columns of one row, plus bias
+// and the element-wise function.  `bias_s` holds the bias of these 32 columns
+// (shared memory, read as a broadcast).
 template <Epi EPI>
-__device__ __forceinline__ void epilogue_math(const uint32_t (&r)[32], const float* bias_s, uint32_t (&p)[16]) {
-  float v[32];
+__device__ __forceinline__ void epilogue_values(const uint32_t (&r)[32], const float* bias_s, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
   if constexpr (EPI != Epi::kStore) {
@@ -171,12 +172,36 @@ __device__ __forceinline__ void epilogue_math(const uint32_t (&r)[32], const flo
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
   }
+}
+
+// v += 8 halves (one 16-byte unit) of the residual, columns 8u .. 8u+7.
+__device__ __forceinline__ void add_residual_unit(float (&v)[32], int u, const uint4& res) {
+  const __half2* h = reinterpret_cast<const __half2*>(&res);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) p[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(h[j]);
+    v[8 * u + 2 * j] += f.x;
+    v[8 * u + 2 * j + 1] += f.y;
+  }
 }
 
 // Bytes of one warp's staging buffer: a 32x32 FP16 chunk.
 constexpr int kStageChunkBytes = 32 * 32 * 2;
+
+// Byte offset of 16-byte unit u (0..3) of row r in a staging buffer with the
+// output map's 64-byte swizzle: unit u of row r sits at unit u ^ ((r >> 1) & 3).
+__device__ __forceinline__ int stage_unit(int r, int u) { return r * 64 + 16 * (u ^ ((r >> 1) & 3)); }
+
+// An epilogue warp's state across tiles: two staging buffers used in turn
+// (chunk i in buffer i & 1), and for kBiasResidStore through TMA the two
+// mbarriers on which the residual chunk loaded into each buffer completes.
+struct EpiWarpState {
+  uint8_t* stage;             // 2 x kStageChunkBytes
+  uint32_t seq = 0;           // chunks written so far
+  const CUtensorMap* tm_r = nullptr;
+  uint32_t res_bar = 0;       // buffer k's barrier at res_bar + 8k
+  uint32_t res_phase = 0;     // bit k: parity of buffer k's next completion
+};
 
 // One epilogue warp's share of a tile: rows [32*quad, 32*quad+32) of the
 // accumulator (one row per lane), global columns [col_begin, col_begin +
@@ -187,16 +212,20 @@ constexpr int kStageChunkBytes = 32 * 32 * 2;
 // chunk j is converted and stored.  `release` runs once the last TMEM load of
 // the tile has completed (it frees the accumulator for the next tile).
 // Stores: with an output map (tm_c != nullptr) each 32x32 chunk is written to
-// the warp's staging buffer in the map's 64-byte swizzle and stored by a TMA
-// bulk copy (full lines, no per-lane stores); the buffer is reused once the
-// previous copy has read it.  Otherwise each lane stores its row with 16-byte
-// stores.
+// a staging buffer in the map's 64-byte swizzle and stored by a TMA bulk copy
+// (full lines, no per-lane stores).  Otherwise each lane stores its row with
+// 16-byte stores.
+// Residual (kBiasResidStore): with an output map, the residual chunk is
+// brought into the chunk's staging buffer by a TMA load (the next chunk's
+// while this one is processed) and added in place; otherwise each lane loads
+// its row's halves.
 template <Epi EPI, int CHUNKS, typename WaitFull, typename Release>
 __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, int col_begin, int M, int N,
                                                    const float* __restrict__ bias, float* bias_s,
                                                    __half* __restrict__ C, const SplitShape& sp,
-                                                   const CUtensorMap* tm_c, uint8_t* stage, uint32_t& store_seq,
-                                                   WaitFull wait_full, Release release) {
+                                                   const CUtensorMap* tm_c, EpiWarpState& ws,
+                                                   const __half* __restrict__ resid, WaitFull wait_full,
+                                                   Release release) {
   const int lane = threadIdx.x & 31;
   if constexpr (EPI != Epi::kStore) {
     for (int i = lane * 4; i < 32 * CHUNKS; i += 128) {   // CHUNKS <= 4
@@ -211,6 +240,30 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
   // Token coordinates of the chunk's first row for the head-split store map.
   const int b0 = EPI == Epi::kBiasQkvSplit ? row0 / sp.seq : 0;
   const int s0 = EPI == Epi::kBiasQkvSplit ? row0 - b0 * sp.seq : 0;
+  constexpr bool kResid = EPI == Epi::kBiasResidStore;
+  const bool tma_resid = kResid && tm_c != nullptr && ws.tm_r != nullptr;
+  auto buf_of = [&](uint32_t seq) { return ws.stage + (seq & 1u) * kStageChunkBytes; };
+  // Lane 0: residual chunk j into the buffer of chunk number `seq`, once every
+  // store this thread issued has read its buffer.
+  auto issue_res = [&](uint32_t seq, int j) {
+    sm100::bulk_wait_group_read<0>();
+    const uint32_t bar = ws.res_bar + 8u * (seq & 1u);
+    sm100::mbar_arrive_expect_tx(bar, kStageChunkBytes);
+    sm100::tma_load_2d(ws.tm_r, sm100::smem_u32(buf_of(seq)), bar, col_begin + 32 * j, row0);
+  };
+  if (tma_resid && lane == 0 && col_begin < N) issue_res(ws.seq, 0);
+  // Per-lane residual path: chunk 0 before the accumulator is awaited, chunk
+  // j+1 while chunk j is processed.
+  uint4 res_a[4] = {}, res_b[kResid ? 4 : 1] = {};
+  auto load_res = [&](int j, uint4* dst) {
+    const int c0 = col_begin + 32 * j;
+    if (!row_ok || c0 >= N) return;
+    const uint4* rp = reinterpret_cast<const uint4*>(resid + (size_t)row * N + c0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c0 + 8 * u < N) dst[u] = rp[u];
+  };
+  if (kResid && !tma_resid) load_res(0, res_a);
   int got = 0;
   if (lane == 0) got = wait_full() ? 1 : 0;
   got = __shfl_sync(0xffffffffu, got, 0);     // also orders the bias staging before its use
@@ -242,19 +295,37 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
     uint32_t(&cur)[32] = *reinterpret_cast<uint32_t(*)[32]>(cur_p);
     const int col0 = col_begin + 32 * j;
     if (col0 >= N) continue;
-    uint32_t p[16];
-    epilogue_math<EPI>(cur, bias_s + 32 * j, p);
-    if (tm_c != nullptr) {
-      uint8_t* buf = stage;
-      ++store_seq;
-      if (lane == 0) sm100::bulk_wait_group_read<0>();   // the previous store has read the buffer
-      __syncwarp();
-      // 64-byte swizzle: 16-byte unit u of row r sits at unit u ^ ((r >> 1) & 3).
+    if (kResid && !tma_resid && j + 1 < CHUNKS) load_res(j + 1, (j & 1) ? res_a : res_b);
+    if (tma_resid && lane == 0 && j + 1 < CHUNKS && col0 + 32 < N) issue_res(ws.seq + 1, j + 1);
+    float v[32];
+    epilogue_values<EPI>(cur, bias_s + 32 * j, v);
+    uint8_t* buf = buf_of(ws.seq);
+    if (tma_resid) {
+      const uint32_t k = ws.seq & 1u;
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      ws.res_phase ^= 1u << k;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        *reinterpret_cast<uint4*>(buf + lane * 64 + 16 * (u ^ ((lane >> 1) & 3))) =
+      for (int u = 0; u < 4; ++u) add_residual_unit(v, u, *reinterpret_cast<const uint4*>(buf + stage_unit(lane, u)));
+    } else if constexpr (kResid) {
+      const uint4* res = (j & 1) ? res_b : res_a;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) add_residual_unit(v, u, res[u]);
+    }
+    uint32_t p[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) p[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+    if (tm_c != nullptr) {
+      // The buffer was last read by the store two chunks back (with a TMA
+      // residual load, that wait came before the load was issued).
+      if (!tma_resid && lane == 0) sm100::bulk_wait_group_read<1>();
+      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4*>(buf + stage_unit(lane, u)) =
             make_uint4(p[4 * u], p[4 * u + 1], p[4 * u + 2], p[4 * u + 3]);
-      }
       sm100::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -270,6 +341,7 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
         }
         sm100::bulk_commit_group();
       }
+      ++ws.seq;
     } else if (row_ok) {
       __half* dst = C + roff + col_offset<EPI>(col0, sp);
 #pragma unroll
@@ -285,9 +357,10 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
 template <int BN, Epi EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M_max, int N, int K,
+                   const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
+                   int use_tma_store, int M_max, int N, int K,
                    const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp, int* __restrict__ status,
-                   const int* __restrict__ m_dev) {
+                   const int* __restrict__ m_dev, const __half* __restrict__ resid) {
   using G = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -318,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tempty_bar(a), kEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(bar0 + 8u * (G::kResBar0 + i), 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -398,9 +472,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kCols = BN / kEpiSlices;
     constexpr int kChunks = kCols / 32;        // 32-column chunks per warp
     float* bias_s = bias_smem + (warp - 2) * kCols;
-    uint8_t* stage = store_smem + (warp - 2) * kStageChunkBytes;
-    const CUtensorMap* tmc = use_tma_store ? &tm_c : nullptr;
-    uint32_t store_seq = 0;
+    const CUtensorMap* tmc = (use_tma_store & 1) ? &tm_c : nullptr;
+    EpiWarpState ws;
+    ws.stage = store_smem + (warp - 2) * 2 * kStageChunkBytes;
+    ws.tm_r = (use_tma_store & 2) ? &tm_r : nullptr;     // residual through TMA (kBiasResidStore)
+    ws.res_bar = bar0 + 8u * (G::kResBar0 + 2 * (warp - 2));
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int m_blk = tile / num_n;
@@ -410,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + slice * kCols;
       const int row0 = m_blk * kBM + quad * 32;
       const bool got = epilogue_warp_tile<EPI, kChunks>(
-          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, stage, store_seq,
+          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, ws, resid,
           [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); },
           [&] { mbar_arrive(tempty_bar(acc)); });
       if (!got) { ok = false; break; }
@@ -451,18 +527,20 @@ struct PairCfg {
   static constexpr int kBBytes = 128 * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;             // two 256-column accumulators
-  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kResBar0 = 2 * kStages + 5;
+  static constexpr int kNumBars = kResBar0 + 2 * kEpiWarps;
   static constexpr int kBiasOffset = (kStages * kStageBytes + kNumBars * 8 + 16 + 15) / 16 * 16;
   static constexpr int kStoreOffset = (kBiasOffset + kEpiWarps * (256 / kEpiSlices) * 4 + 1023) / 1024 * 1024;
-  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * (32 * 32 * 2);
+  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * 2 * (32 * 32 * 2);
 };
 
 template <Epi EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ CUtensorMap tm_c, int use_tma_store, int M_max, int N, int K,
+                        const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
+                        int use_tma_store, int M_max, int N, int K,
                         const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp,
-                        int* __restrict__ status, const int* __restrict__ m_dev) {
+                        int* __restrict__ status, const int* __restrict__ m_dev, const __half* __restrict__ resid) {
   using G = PairCfg;
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -497,6 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(tempty_bar(a), 2 * kEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(bar0 + 8u * (G::kResBar0 + i), 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -583,9 +662,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     constexpr int kCols = BN / kEpiSlices;
     constexpr int kChunks = kCols / 32;
     float* bias_s = bias_smem + (warp - 2) * kCols;
-    uint8_t* stage = store_smem + (warp - 2) * kStageChunkBytes;
-    const CUtensorMap* tmc = use_tma_store ? &tm_c : nullptr;
-    uint32_t store_seq = 0;
+    const CUtensorMap* tmc = (use_tma_store & 1) ? &tm_c : nullptr;
+    EpiWarpState ws;
+    ws.stage = store_smem + (warp - 2) * 2 * kStageChunkBytes;
+    ws.tm_r = (use_tma_store & 2) ? &tm_r : nullptr;     // residual through TMA (kBiasResidStore)
+    ws.res_bar = bar0 + 8u * (G::kResBar0 + 2 * (warp - 2));
     const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
     const uint32_t leader_tempty1 = mapa_shared(tempty_bar(1), 0);
     uint32_t local = 0;
@@ -597,7 +678,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + slice * kCols;
       const int row0 = m_blk * 256 + (int)rank * 128 + quad * 32;
       const bool got = epilogue_warp_tile<EPI, kChunks>(
-          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, stage, store_seq,
+          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, ws, resid,
           [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); },
           [&] { mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0); });
       if (!got) { ok = false; break; }
@@ -615,6 +696,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_dealloc_pair(tmem_base, G::kTmemCols);
   }
 }
+
+// Epilogue store flags: bit 0 = TMA stores through tmap_c, bit 1 = residual
+// tiles through tmap_r (only with TMA stores).
+int store_flags(const TcGemmArgs& a) { return (a.tmap_c ? 1 : 0) | (a.tmap_c && a.tmap_r ? 2 : 0); }
 
 template <Epi EPI>
 cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
@@ -647,8 +732,8 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   const int tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
   return launch_kernel(gemm_tc_pair_kernel<EPI>, dim3(2 * pairs), dim3(kThreads), G::kSmem, stream, nullptr, 0,
-                       *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias,
-                       a.c, a.split, a.status, a.m_dev);
+                       *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_r ? *a.tmap_r : *a.tmap_a,
+                       store_flags(a), a.M, a.N, a.K, a.bias, a.c, a.split, a.status, a.m_dev, a.resid);
 }
 
 // ---------------------------------------------------------------------------
@@ -687,12 +772,20 @@ __device__ __forceinline__ uint32_t part_offset(int r, int u) {
   return SplitCfg::kPartOffset + r * 512 + 16 * (u ^ (r & 31));
 }
 
-// Bias and the epilogue's element-wise function on 4 consecutive columns.
+// Bias, residual and the epilogue's element-wise function on 4 consecutive
+// columns of row `row`.
 template <Epi EPI>
-__device__ __forceinline__ void epilogue4(float (&v)[4], const float* __restrict__ bias, int col) {
+__device__ __forceinline__ void epilogue4(float (&v)[4], const float* __restrict__ bias,
+                                          const __half* __restrict__ resid, int row, int N, int col) {
   if constexpr (EPI != Epi::kStore) {
     const float4 b = __ldg(reinterpret_cast<const float4*>(bias + col));
     v[0] += b.x; v[1] += b.y; v[2] += b.z; v[3] += b.w;
+  }
+  if constexpr (EPI == Epi::kBiasResidStore) {
+    const uint2 u = *reinterpret_cast<const uint2*>(resid + (size_t)row * N + col);
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+    v[0] += lo.x; v[1] += lo.y; v[2] += hi.x; v[3] += hi.y;
   }
   if constexpr (EPI == Epi::kBiasGelu) {
     gelu_erf_pair(v[0], v[1]);
@@ -708,7 +801,8 @@ template <Epi EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_splitk_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           int M_max, int N, int K, const float* __restrict__ bias, __half* __restrict__ C,
-                          SplitShape sp, int* __restrict__ status, const int* __restrict__ m_dev, int splits) {
+                          SplitShape sp, int* __restrict__ status, const int* __restrict__ m_dev, int splits,
+                          const __half* __restrict__ resid) {
   using G = SplitCfg;
   const int num_n = (N + G::kBN - 1) / G::kBN;
   const int tile = blockIdx.x / splits;
@@ -846,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 p = ld_cluster_f4(mapa_shared(off, (uint32_t)s));
           a[0] += p.x; a[1] += p.y; a[2] += p.z; a[3] += p.w;
         }
-        epilogue4<EPI>(a, bias, col);
+        epilogue4<EPI>(a, bias, resid, grow, N, col);
         __half* dst = C + row_offset<EPI>(grow, N, sp) + col_offset<EPI>(col, sp);
         *reinterpret_cast<uint2*>(dst) = make_uint2(pack_half2(a[0], a[1]), pack_half2(a[2], a[3]));
       }
@@ -917,7 +1011,7 @@ cudaError_t launch_splitk(const TcGemmArgs& a, cudaStream_t stream) {
   attr.val.clusterDim.z = 1;
   return launch_kernel(gemm_tc_splitk_kernel<EPI>, dim3(tiles * a.splits), dim3(kThreads), SplitCfg::kSmem, stream,
                        &attr, 1, *a.tmap_a, *a.tmap_b, a.M, a.N, a.K, a.bias, a.c, a.split, a.status, a.m_dev,
-                       a.splits);
+                       a.splits, a.resid);
 }
 
 template <int BN, Epi EPI>
@@ -933,8 +1027,8 @@ cudaError_t launch_impl(const TcGemmArgs& a, cudaStream_t stream) {
   const int tiles = ((a.M + kBM - 1) / kBM) * ((a.N + BN - 1) / BN);
   const int grid = tiles < a.num_sms ? tiles : a.num_sms;
   return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), G::kSmem, stream, nullptr, 0, *a.tmap_a,
-                       *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_c ? 1 : 0, a.M, a.N, a.K, a.bias, a.c,
-                       a.split, a.status, a.m_dev);
+                       *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_r ? *a.tmap_r : *a.tmap_a, store_flags(a),
+                       a.M, a.N, a.K, a.bias, a.c, a.split, a.status, a.m_dev, a.resid);
 }
 
 template <int BN>
@@ -945,6 +1039,7 @@ cudaError_t launch_bn(const TcGemmArgs& a, cudaStream_t stream) {
     case Epi::kBiasQkvSplit: return launch_impl<BN, Epi::kBiasQkvSplit>(a, stream);
     case Epi::kBiasGeluTanh: return launch_impl<BN, Epi::kBiasGeluTanh>(a, stream);
     case Epi::kBiasStore: return launch_impl<BN, Epi::kBiasStore>(a, stream);
+    case Epi::kBiasResidStore: return launch_impl<BN, Epi::kBiasResidStore>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -1014,6 +1109,7 @@ int choose_gemm_splits(int tiles, int num_kb, int num_sms) {
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0 || (a.N % 8) != 0 || (a.K % 8) != 0) return cudaErrorInvalidValue;
   if (a.epi == Epi::kBiasQkvSplit && (a.split.size_per_head % 32) != 0) return cudaErrorInvalidValue;
+  if (a.epi == Epi::kBiasResidStore && !a.resid) return cudaErrorInvalidValue;
   // The head-split store map needs every 32-row chunk inside one sequence.
   if (a.epi == Epi::kBiasQkvSplit && a.tmap_c && (a.split.seq % 32) != 0) return cudaErrorInvalidValue;
   if (a.splits > 1) {
@@ -1026,6 +1122,7 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
       case Epi::kBiasQkvSplit: return launch_splitk<Epi::kBiasQkvSplit>(a, stream);
       case Epi::kBiasGeluTanh: return launch_splitk<Epi::kBiasGeluTanh>(a, stream);
       case Epi::kBiasStore: return launch_splitk<Epi::kBiasStore>(a, stream);
+      case Epi::kBiasResidStore: return launch_splitk<Epi::kBiasResidStore>(a, stream);
     }
     return cudaErrorInvalidValue;
   }
@@ -1037,6 +1134,7 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
       case Epi::kBiasQkvSplit: return launch_pair<Epi::kBiasQkvSplit>(a, stream);
       case Epi::kBiasGeluTanh: return launch_pair<Epi::kBiasGeluTanh>(a, stream);
       case Epi::kBiasStore: return launch_pair<Epi::kBiasStore>(a, stream);
+      case Epi::kBiasResidStore: return launch_pair<Epi::kBiasResidStore>(a, stream);
     }
     return cudaErrorInvalidValue;
   }

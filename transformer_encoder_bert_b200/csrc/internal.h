@@ -18,7 +18,8 @@ enum class Epi : int {
   kBiasGelu = 1,     // C[m][n] = GELU(acc + bias[n]), erf form
   kBiasQkvSplit = 2, // Q/K/V head split: dst[t][b][h][s][c] = acc + bias[n]
   kBiasGeluTanh = 3, // C[m][n] = GELU_tanh(acc + bias[n])
-  kBiasStore = 4     // C[m][n] = acc + bias[n]
+  kBiasStore = 4,    // C[m][n] = acc + bias[n]
+  kBiasResidStore = 5  // C[m][n] = acc + bias[n] + R[m][n]  (R: the residual, [M, N] like C)
 };
 
 // Addressing for the head-split epilogue (n = t*H + h*d + c, m = b*seq + s).
@@ -90,6 +91,8 @@ struct TcGemmArgs {
   // tile, CTA r taking the r-th of `splits` balanced ranges of the k-blocks;
   // the partial sums meet in the cluster's shared memory (no global scratch).
   int splits = 1;
+  const __half* resid = nullptr;  // [M, N] (kBiasResidStore)
+  const CUtensorMap* tmap_r = nullptr;  // the residual as an output-style map (32x32 box), or nullptr
 };
 // The split count for a GEMM of `tiles` 128 x 128 tiles and `num_kb` 64-wide
 // k-blocks: the largest s <= min(16, num_kb) whose clusters of s CTAs all fit
@@ -118,7 +121,8 @@ cudaError_t launch_unpack_rows(const __half* yp, const int32_t* valid_len, const
 // ---- FP32 SIMT GEMM (FP32 mode, no TF32), gemm_f32.cu ----
 // C = A[M,K] * W[K,N] (W row-major [K,N]).
 cudaError_t launch_gemm_f32(const float* A, const float* W, int M, int N, int K, Epi epi,
-                            const float* bias, float* C, SplitShape split, cudaStream_t stream);
+                            const float* bias, float* C, SplitShape split, cudaStream_t stream,
+                            const float* resid = nullptr);
 
 // ---- attention, attention.cu ----
 cudaError_t launch_attention_f16(const __half* qkv, const int32_t* valid_len, __half* ctx,
@@ -140,18 +144,14 @@ bool attention_tc_supported(int size_per_head, int seq);
 cudaError_t launch_attention_tc(const __half* qkv, const int32_t* valid_len, const int32_t* offsets, __half* ctx,
                                 int batch, int seq, int head_num, int* status, cudaStream_t stream);
 
-// ---- add-bias + residual + LayerNorm, layernorm.cu ----
-cudaError_t launch_bias_residual_ln_f16(const __half* a, const float* bias, const __half* resid,
-                                        const float* gamma, const float* beta, __half* out,
-                                        int rows, int hidden, cudaStream_t stream);
+// ---- LayerNorm of z = a + bias + residual (added by the GEMM epilogue), layernorm.cu ----
+cudaError_t launch_layernorm_f16(const __half* z, const float* gamma, const float* beta, __half* out, int rows,
+                                 int hidden, cudaStream_t stream);
 // FP16 rows with FP16 parameters (hidden <= 1024): one row per warp.
-cudaError_t launch_bias_residual_ln_f16h(const __half* a, const __half* bias, const __half* resid,
-                                         const __half* gamma, const __half* beta, __half* out,
-                                         int rows, int hidden, cudaStream_t stream,
-                                         const int* rows_dev = nullptr);
-cudaError_t launch_bias_residual_ln_f32(const float* a, const float* bias, const float* resid,
-                                        const float* gamma, const float* beta, float* out,
-                                        int rows, int hidden, cudaStream_t stream);
+cudaError_t launch_layernorm_f16h(const __half* z, const __half* gamma, const __half* beta, __half* out, int rows,
+                                  int hidden, cudaStream_t stream, const int* rows_dev = nullptr);
+cudaError_t launch_layernorm_f32(const float* z, const float* gamma, const float* beta, float* out, int rows,
+                                 int hidden, cudaStream_t stream);
 
 // ---- weight repack, encoder.cu ----
 int device_sm_count();
