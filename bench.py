@@ -39,6 +39,9 @@ METRIC = "BERT-Base FP16 encoder fwd sequences/s (seq 32/128); % tensor/HBM roof
 UNIT = "sequences/s"
 DEFAULT_WORKLOAD = "bert-base-s32:512"
 KERNEL_NAMES = ["qkv_gemm", "attention", "out_proj_gemm", "ln1", "ffn1_gemm", "ffn2_gemm", "ln2"]
+# when the output-projection and FFN2 GEMMs write the LayerNorm of their rows
+KERNEL_NAMES_FUSED = ["qkv_gemm", "attention", "out_proj_ln_gemm", "ffn1_gemm", "ffn2_ln_gemm"]
+KERNEL_NAMES_FFN2_LN = ["qkv_gemm", "attention", "out_proj_gemm", "ln1", "ffn1_gemm", "ffn2_ln_gemm"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -56,6 +59,50 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# Sources each timed kernel is built from: a DRAM-traffic figure measured by
+# ncu holds only while these files are unchanged.
+KERNEL_SOURCES = {
+    "qkv_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "out_proj_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "ffn1_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "ffn2_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "out_proj_ln_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "ffn2_ln_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "attention": ["attention.cu", "attention_tc.cu", "sm100.cuh", "internal.h"],
+    "ln1": ["layernorm.cu", "internal.h"],
+    "ln2": ["layernorm.cu", "internal.h"],
+}
+
+
+def source_digest(kernel: str) -> str:
+    """First 16 hex digits of the SHA-256 of the kernel's source files."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(ROOT, "transformer_encoder_bert_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum) of
+    `kernel` on `workload` from profiles/traffic.md, or None when there is no
+    capture or the kernel's sources have changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
+        return None
+    digest = source_digest(kernel)
+    with open(path) as f:
+        for line in f:
+            cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 4 and cells[0] == kernel and cells[1] == workload and cells[3] == digest:
+                try:
+                    return float(cells[2].replace(",", ""))
+                except ValueError:
+                    return None
+    return None
 
 
 def blas_threads() -> int:
@@ -87,6 +134,8 @@ def kernel_work(wl: EI.Workload, attn_seq=None, attn_tokens=None):
         "ffn1_gemm": gemm(F, H),
         "ffn2_gemm": gemm(H, F, extra_out=es * M * H),
         "ln2": (0.0, es * 2.0 * M * H),
+        "out_proj_ln_gemm": gemm(H, H, extra_out=es * M * H),  # + residual read, normalised rows written
+        "ffn2_ln_gemm": gemm(H, F, extra_out=es * M * H),
     }
 
 
@@ -253,7 +302,7 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         step()
     torch.cuda.synchronize()
 
-    nk = enc.kernels_per_forward()
+    nk = enc.kernels_per_forward(wl.batch, wl.seq)
     ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -290,8 +339,10 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
 
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
-    names = (["offsets", "pack"] + KERNEL_NAMES * sh.num_layers + ["unpack"]) if args.packed \
-        else KERNEL_NAMES * sh.num_layers
+    per_layer = (nk - (3 if args.packed else 0)) // sh.num_layers
+    layer_names = {5: KERNEL_NAMES_FUSED, 6: KERNEL_NAMES_FFN2_LN}.get(per_layer, KERNEL_NAMES)
+    names = (["offsets", "pack"] + layer_names * sh.num_layers + ["unpack"]) if args.packed \
+        else layer_names * sh.num_layers
     per_kernel = {k: [] for k in names}
     for evs in ev_sets:
         for j in range(nk):
@@ -347,16 +398,17 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         kernels[k] = entry
     dominant = max(kernels, key=lambda k: kernels[k]["share"])
     d = kernels[dominant]
+    traffic = args.traffic if args.traffic is not None else measured_traffic(dominant, wl.name)
     if dominant.endswith("gemm"):
         peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         roof = {"bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
-                "frac": d["tflops"] / peak, "traffic": args.traffic,
+                "frac": d["tflops"] / peak, "traffic": traffic,
                 "kernel": dominant, "per_launch_flops": work[dominant][0],
                 "peak_source": f"{peak_src} sustained bf16 matmul (FP16 dense rate = BF16 dense rate)"}
     else:
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         roof = {"bound": "hbm", "achieved": d["gbs"], "peak": peak, "unit": "GB/s", "frac": d["gbs"] / peak,
-                "traffic": args.traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
+                "traffic": traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
                 "peak_source": f"{peak_src} HBM copy bandwidth"}
 
     value = job_throughput(wl.batch, world, ms)

@@ -205,21 +205,26 @@ ENC_API enc_status enc_graph_launch(enc_graph_t graph, enc_stream_t stream);
 /* enc_graph_destroy - release a recorded forward (synchronises the device). NULL is a no-op. */
 ENC_API enc_status enc_graph_destroy(enc_graph_t graph);
 
-/* enc_kernels_per_forward - kernel launches one enc_forward issues (7 per layer,
- * plus 3 with padding removal). */
-ENC_API int enc_kernels_per_forward(enc_t h);
+/* enc_kernels_per_forward - kernel launches one enc_forward of batch x seq
+ * issues: per layer 7, less one for each of the output-projection and FFN2
+ * GEMMs that writes the LayerNorm of its rows itself (FP16, enough tokens for
+ * the 2-CTA tiles; by default FFN2 with hidden size 256, 512 or 768); plus 3
+ * with padding removal.  0 for invalid arguments. */
+ENC_API int enc_kernels_per_forward(enc_t h, int batch, int seq);
 
 /* enc_launch_count - kernel launches this handle has issued since enc_create
  * (forward passes and single steps), for checking what ran. */
 ENC_API uint64_t enc_launch_count(enc_t h);
 
 /* enc_set_trace_events - optional per-kernel timing of enc_forward.  events
- * holds count CUDA events (cudaEvent_t, created by the caller); with count >=
- * enc_kernels_per_forward(h) + 1, each enc_forward records events[k] on its
+ * holds count CUDA events (cudaEvent_t, created by the caller; at least
+ * 5 * num_layers + 1, and a forward needing more fails with ENC_ERR_INVALID_ARG);
+ * with count >= enc_kernels_per_forward(h, batch, seq) + 1, each enc_forward records events[k] on its
  * stream just before its k-th kernel and events[kernels] after the last, so
  * cudaEventElapsedTime(events[k], events[k+1]) is kernel k's duration.
  * Kernel order per layer: QKV GEMM, attention, output GEMM, LayerNorm 1,
- * FFN1 GEMM, FFN2 GEMM, LayerNorm 2; with padding removal the offsets and
+ * FFN1 GEMM, FFN2 GEMM, LayerNorm 2 (without the two LayerNorm kernels when
+ * the GEMMs write the normalised rows); with padding removal the offsets and
  * pack kernels come first and the unpack kernel last.  events = NULL or count = 0 switches
  * tracing off.  The handle keeps the pointers; the caller keeps the events
  * alive while tracing is on. */
@@ -248,31 +253,28 @@ ENC_API enc_status enc_op_qkv(enc_t h, int layer, const void* x, void* qkv, int 
 ENC_API enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, void* ctx,
                             int batch, int seq, enc_stream_t stream);
 
-/* Step output projection with the add-bias and residual of the first
- * add-bias + residual + LayerNorm ([FT] "Faster Transformer 优化原理") done in
- * the GEMM epilogue:
- *   z = ctx Wo + bo + resid,  ctx, resid, z: [M, H]  (resid = the layer input). */
-ENC_API enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, const void* resid, void* z,
-                                   int tokens, enc_stream_t stream);
-
-/* Step LayerNorm of a row that already holds bias + residual (the rest of the
- * page's add-bias + residual + LayerNorm kernel):
- *   which = 1: out = LN(z; ln1_g, ln1_b);  which = 2: out = LN(z; ln2_g, ln2_b)
- *   z, out: [tokens, H]; mean and biased variance over H, eps 1e-12. */
-ENC_API enc_status enc_op_layernorm(enc_t h, int layer, int which, const void* z, void* out, int tokens,
-                                    enc_stream_t stream);
+/* Steps output projection + add-bias + residual + LayerNorm 1 ([FT] "Faster
+ * Transformer 优化原理": the output GEMM and the add-bias + residual + Layer
+ * Normalization kernel):
+ *   out = LN1(ctx Wo + bo + resid),  ctx, resid, out: [tokens, H]  (resid = the
+ *   layer input); LN over H, biased variance, eps 1e-12.
+ * One kernel when the GEMM writes the normalised rows itself (see
+ * enc_kernels_per_forward); otherwise the GEMM writes ctx Wo + bo + resid into
+ * the handle's workspace (which grows as enc_forward's does) and a LayerNorm
+ * kernel follows. */
+ENC_API enc_status enc_op_out_proj_ln(enc_t h, int layer, const void* ctx, const void* resid, void* out,
+                                      int tokens, enc_stream_t stream);
 
 /* Step FFN1 + add-bias + GELU (erf form) fused in the GEMM epilogue:
  *   u = GELU(h1 W1 + b1),  h1: [tokens, H], u: [tokens, F]. */
 ENC_API enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens,
                        enc_stream_t stream);
 
-/* Step FFN2 with the add-bias and residual of the second add-bias + residual +
- * LayerNorm done in the GEMM epilogue:
- *   z = u W2 + b2 + resid,  u: [tokens, F], resid, z: [tokens, H]  (resid = h1,
- *   the first LayerNorm's output). */
-ENC_API enc_status enc_op_ffn2(enc_t h, int layer, const void* u, const void* resid, void* z, int tokens,
-                               enc_stream_t stream);
+/* Steps FFN2 + add-bias + residual + LayerNorm 2, like enc_op_out_proj_ln:
+ *   out = LN2(u W2 + b2 + resid),  u: [tokens, F], resid, out: [tokens, H]
+ *   (resid = h1, the first LayerNorm's output). */
+ENC_API enc_status enc_op_ffn2_ln(enc_t h, int layer, const void* u, const void* resid, void* out, int tokens,
+                                  enc_stream_t stream);
 
 #ifdef __cplusplus
 }

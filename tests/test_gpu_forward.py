@@ -203,7 +203,7 @@ def test_recorded_forward_replays_bit_exact():
     for _ in range(3):
         g.launch(stream=s)
     s.synchronize()
-    assert enc.launch_count() - n0 == 3 * enc.kernels_per_forward()
+    assert enc.launch_count() - n0 == 3 * enc.kernels_per_forward(8, 32)
     assert np.array_equal(to_host(out), ref)
     # new input values in the same buffers are picked up at replay time
     x2 = EI.make_inputs(EI.named_workload("bert-base-s32", 8).with_(seed=5)).x
@@ -223,20 +223,28 @@ def test_recorded_forward_replays_bit_exact():
 @pytest.mark.parametrize("chunks,layers", [(2, 12), (4, 12), (4, 2), (3, 3)])
 def test_host_entry_point_chunked_pipeline_matches_device_forward(chunks, layers):
     # 256 x 32 tokens: the first and last layers run chunk by chunk while the
-    # copies of the other chunks are in flight; results are bit-identical.
+    # copies of the other chunks are in flight.  Bit-identical to the whole-batch
+    # forward when the chunks run the same kernels; when the chunks are too small
+    # for the GEMMs that fuse the LayerNorm (which keep z in FP32 instead of
+    # rounding it to FP16 first), within the FP16 per-layer bound.
     import torch
     wl = EI.named_workload("bert-base-s32", 256)
     inp = EI.make_inputs(wl.with_(shape=EI.EncoderShape(12, 64, 3072, layers)))
     enc = encoder_from_inputs(inp)
     dev = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    same_kernels = enc.kernels_per_forward(256 // chunks, 32) == enc.kernels_per_forward(256, 32)
     enc.set_host_chunks(chunks)
     hx = torch.from_numpy(inp.x).pin_memory()
     hvl = torch.from_numpy(inp.valid_len).pin_memory()
     hout = torch.empty_like(hx).pin_memory()
     enc.forward_host_ptr(hx.data_ptr(), hvl.data_ptr(), hout.data_ptr(), 256, 32)
-    assert np.array_equal(hout.numpy(), dev)
+    m = valid_mask(inp.valid_len, 32)
+    if same_kernels:
+        assert np.array_equal(hout.numpy(), dev)
+    else:
+        assert rel_l2(hout.numpy(), dev, m) < FP16_LAYER_REL_L2
     pageable = enc.forward_host(inp.x, inp.valid_len)
-    assert np.array_equal(pageable, dev)
+    assert np.array_equal(pageable, hout.numpy())
 
 
 def test_pipelined_host_entry_point_matches_device_forward():
@@ -277,7 +285,7 @@ def test_packed_forward_matches_oracle_and_zeroes_padding(seq, lo, hi, L):
     enc = encoder_from_inputs(inp)
     dense = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
     enc.set_packing(True)
-    assert enc.kernels_per_forward() == 7 * L + 3
+    assert enc.kernels_per_forward(6, seq) == 7 * L + 3
     got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
     m = valid_mask(inp.valid_len, seq)
     assert np.all(got[~m] == 0)

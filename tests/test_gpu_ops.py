@@ -80,10 +80,11 @@ def test_out_proj_ffn1_ffn2(shape, batch, seq):
     ctx = EI.random_array((M, H), "fp16", seed=11)
     resid = EI.random_array((M, H), "fp16", seed=14)
     a = empty_dev((M, H), "fp16")
-    enc.op_out_proj(0, to_dev(ctx), to_dev(resid), a, M)      # epilogue: + bias + residual
-    ref = ctx.astype(np.float64) @ lw["w_o"] + lw["b_o"] + resid.astype(np.float64)
+    enc.op_out_proj_ln(0, to_dev(ctx), to_dev(resid), a, M)
+    ref = O.bias_residual_layernorm(ctx.astype(np.float64) @ lw["w_o"], lw["b_o"], resid.astype(np.float64),
+                                    lw["ln1_g"], lw["ln1_b"])
     got = to_host(a)
-    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < LN_MAX_ABS
 
     h1 = EI.random_array((M, H), "fp16", seed=12)
     u = empty_dev((M, F), "fp16")
@@ -94,29 +95,50 @@ def test_out_proj_ffn1_ffn2(shape, batch, seq):
 
     uu = EI.random_array((M, F), "fp16", seed=13, std=0.5)
     y = empty_dev((M, H), "fp16")
-    enc.op_ffn2(0, to_dev(uu), to_dev(h1), y, M)              # epilogue: + bias + residual (h1)
-    ref = uu.astype(np.float64) @ lw["w_ff2"] + lw["b_ff2"] + h1.astype(np.float64)
+    enc.op_ffn2_ln(0, to_dev(uu), to_dev(h1), y, M)
+    ref = O.bias_residual_layernorm(uu.astype(np.float64) @ lw["w_ff2"], lw["b_ff2"], h1.astype(np.float64),
+                                    lw["ln2_g"], lw["ln2_b"])
     got = to_host(y)
-    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < LN_MAX_ABS
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}_F{s[2]}")
-@pytest.mark.parametrize("which", [1, 2])
-def test_layernorm(shape, which):
-    """LayerNorm of rows that already hold bias + residual (added by the GEMM epilogue)."""
+@pytest.mark.parametrize("shape,M", [((4, 64, 1024), 9300), ((12, 64, 3072), 4000), ((16, 64, 4096), 2600),
+                                     ((12, 64, 3072), 16384)], ids=lambda v: str(v))
+def test_fused_layernorm_gemms(monkeypatch, shape, M):
+    """Enough tokens for the 2-CTA tiles: the GEMMs write the LayerNorm of their rows
+    (row statistics exchanged across the cluster that covers the row; clusters of
+    2, 6 and 8 CTAs for H = 256, 768, 1024).  FFN2 is fused by default for H <= 768,
+    the output projection through ENC_LN_FUSE_OPROJ=1.  Against the oracle step,
+    and against the unfused path (GEMM writing bias + residual, then the LayerNorm
+    kernel; ENC_LN_NO_FUSE=1)."""
+    monkeypatch.setenv("ENC_LN_FUSE_OPROJ", "1")
     nh, d, F = shape
     H = nh * d
-    batch, seq = 5, 131
-    M = batch * seq
-    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
-    z = EI.random_array((M, H), "fp16", seed=21, std=1.2, mean=0.3)
-    out = empty_dev((M, H), "fp16")
-    enc.op_layernorm(0, which, to_dev(z), out, M)
-    tag = "1" if which == 1 else "2"
-    ref = O.layer_norm(z.astype(np.float64), lw[f"ln{tag}_g"], lw[f"ln{tag}_b"])
-    got = to_host(out)
-    assert max_abs(got, ref) < LN_MAX_ABS
-    assert rel_l2(got, ref) < GEMM_REL_L2
+    wl, inp, enc, x64, vl, lw = _setup(shape, 1, M)
+    ctx = EI.random_array((M, H), "fp16", seed=41)
+    resid = EI.random_array((M, H), "fp16", seed=42, mean=0.2)
+    uu = EI.random_array((M, F), "fp16", seed=43, std=0.5)
+
+    def run(e):
+        a = empty_dev((M, H), "fp16")
+        e.op_out_proj_ln(0, to_dev(ctx), to_dev(resid), a, M)
+        y = empty_dev((M, H), "fp16")
+        e.op_ffn2_ln(0, to_dev(uu), a, y, M)
+        return to_host(a), to_host(y)
+
+    got_a, got_y = run(enc)
+    ref_a = O.bias_residual_layernorm(ctx.astype(np.float64) @ lw["w_o"], lw["b_o"], resid.astype(np.float64),
+                                      lw["ln1_g"], lw["ln1_b"])
+    ref_y = O.bias_residual_layernorm(uu.astype(np.float64) @ lw["w_ff2"], lw["b_ff2"], got_a.astype(np.float64),
+                                      lw["ln2_g"], lw["ln2_b"])
+    for g, r in ((got_a, ref_a), (got_y, ref_y)):
+        assert rel_l2(g, r) < GEMM_REL_L2 and max_abs(g, r) < LN_MAX_ABS
+    assert enc.device_status() == 0
+    monkeypatch.setenv("ENC_LN_NO_FUSE", "1")
+    monkeypatch.delenv("ENC_LN_FUSE_OPROJ")
+    wl, inp, enc1, x64, vl, lw = _setup(shape, 1, M)
+    un_a, un_y = run(enc1)
+    assert rel_l2(got_a, un_a) < GEMM_REL_L2 and rel_l2(got_y, un_y) < GEMM_REL_L2
 
 
 @pytest.mark.parametrize("shape", [(4, 32, 512), (12, 64, 3072)], ids=lambda s: f"{s[0]}x{s[1]}")
@@ -139,18 +161,16 @@ def test_fp32_steps(shape):
     u = empty_dev((M, F), "fp32")
     enc.op_ffn1(0, to_dev(h1), u, M)
     assert rel_l2(to_host(u), O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"])) < FP32_REL_L2
-    z = empty_dev((M, H), "fp32")
-    enc.op_out_proj(0, ctx, to_dev(h1), z, M)
-    ref_z = to_host(ctx).astype(np.float64) @ lw["w_o"] + lw["b_o"] + h1.astype(np.float64)
-    assert rel_l2(to_host(z), ref_z) < FP32_REL_L2
     out = empty_dev((M, H), "fp32")
-    enc.op_layernorm(0, 1, z, out, M)
-    ref = O.layer_norm(to_host(z).astype(np.float64), lw["ln1_g"], lw["ln1_b"])
+    enc.op_out_proj_ln(0, ctx, to_dev(h1), out, M)
+    ref = O.bias_residual_layernorm(to_host(ctx).astype(np.float64) @ lw["w_o"], lw["b_o"], h1.astype(np.float64),
+                                    lw["ln1_g"], lw["ln1_b"])
     assert rel_l2(to_host(out), ref) < FP32_REL_L2
     uu = EI.random_array((M, F), "fp32", seed=7, std=0.5)
     y = empty_dev((M, H), "fp32")
-    enc.op_ffn2(0, to_dev(uu), out, y, M)
-    ref_y = uu.astype(np.float64) @ lw["w_ff2"] + lw["b_ff2"] + to_host(out).astype(np.float64)
+    enc.op_ffn2_ln(0, to_dev(uu), out, y, M)
+    ref_y = O.bias_residual_layernorm(uu.astype(np.float64) @ lw["w_ff2"], lw["b_ff2"],
+                                      to_host(out).astype(np.float64), lw["ln2_g"], lw["ln2_b"])
     assert rel_l2(to_host(y), ref_y) < FP32_REL_L2
 
 
@@ -179,7 +199,7 @@ def test_gemm_bounded_waits_never_fired():
     M = 5 * 131
     y = empty_dev((M, 768), "fp16")
     resid = to_dev(EI.random_array((M, 768), "fp16", seed=2))
-    enc.op_ffn2(0, to_dev(EI.random_array((M, 3072), "fp16", seed=1)), resid, y, M)
+    enc.op_ffn2_ln(0, to_dev(EI.random_array((M, 3072), "fp16", seed=1)), resid, y, M)
     assert enc.device_status() == 0
 
 
@@ -231,10 +251,11 @@ def test_alternative_gemm_paths(monkeypatch, env, batch, seq):
     ctx = EI.random_array((M, H), "fp16", seed=15)
     resid = EI.random_array((M, H), "fp16", seed=16)
     z = empty_dev((M, H), "fp16")
-    enc.op_out_proj(0, to_dev(ctx), to_dev(resid), z, M)
-    ref = ctx.astype(np.float64) @ lw["w_o"] + lw["b_o"] + resid.astype(np.float64)
+    enc.op_out_proj_ln(0, to_dev(ctx), to_dev(resid), z, M)
+    ref = O.bias_residual_layernorm(ctx.astype(np.float64) @ lw["w_o"], lw["b_o"], resid.astype(np.float64),
+                                    lw["ln1_g"], lw["ln1_b"])
     got = to_host(z)
-    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < _ulp_bound(ref)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < LN_MAX_ABS
 
 
 @pytest.mark.parametrize("batch,seq", [(3, 128), (4, 96), (3, 65)], ids=str)
@@ -259,7 +280,7 @@ def test_split_k_gemms(monkeypatch, batch, seq):
     """At small M the GEMMs run split-K: a cluster of CTAs shares each 128x128 tile,
     each CTA one range of the k-blocks, and the partial tiles are summed in rank
     order through distributed shared memory.  Every epilogue (head split, plain,
-    erf-GELU, tanh-GELU, bias + residual) against its oracle step; a repeated call is bit-identical
+    erf-GELU, tanh-GELU, bias + residual + LayerNorm) against its oracle step; a repeated call is bit-identical
     (the sum's order does not depend on timing); the unsplit kernel
     (ENC_GEMM_NO_SPLITK=1) agrees within the GEMM bound."""
     shape = (12, 64, 3072)
@@ -274,7 +295,7 @@ def test_split_k_gemms(monkeypatch, batch, seq):
         qkv = empty_dev((3, batch, nh, seq, d), "fp16")
         enc.op_qkv(0, to_dev(inp.x), qkv, batch, seq)
         a = empty_dev((M, H), "fp16")
-        enc.op_out_proj(0, to_dev(ctx), to_dev(h1), a, M)
+        enc.op_out_proj_ln(0, to_dev(ctx), to_dev(h1), a, M)
         u = empty_dev((M, F), "fp16")
         enc.op_ffn1(0, to_dev(h1), u, M)
         enc.set_gelu("tanh")
@@ -282,20 +303,22 @@ def test_split_k_gemms(monkeypatch, batch, seq):
         enc.op_ffn1(0, to_dev(h1), ut, M)
         enc.set_gelu("erf")
         y = empty_dev((M, H), "fp16")
-        enc.op_ffn2(0, to_dev(uu), to_dev(ctx), y, M)
+        enc.op_ffn2_ln(0, to_dev(uu), to_dev(ctx), y, M)
         return [to_host(t) for t in (qkv, a, u, ut, y)]
 
     wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
     got = run(enc)
     refs = [
         O.head_split(O.qkv_projection(x64.reshape(-1, H), lw["w_qkv"], lw["b_qkv"]), batch, seq, nh, d),
-        ctx.astype(np.float64) @ lw["w_o"] + lw["b_o"] + h1.astype(np.float64),
+        O.bias_residual_layernorm(ctx.astype(np.float64) @ lw["w_o"], lw["b_o"], h1.astype(np.float64),
+                                  lw["ln1_g"], lw["ln1_b"]),
         O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"]),
         O.ffn1_gelu(h1.astype(np.float64), lw["w_ff1"], lw["b_ff1"], gelu="tanh"),
-        uu.astype(np.float64) @ lw["w_ff2"] + lw["b_ff2"] + ctx.astype(np.float64),
+        O.bias_residual_layernorm(uu.astype(np.float64) @ lw["w_ff2"], lw["b_ff2"], ctx.astype(np.float64),
+                                  lw["ln2_g"], lw["ln2_b"]),
     ]
     for g, r in zip(got, refs):
-        assert rel_l2(g, r) < GEMM_REL_L2 and max_abs(g, r) < _ulp_bound(r)
+        assert rel_l2(g, r) < GEMM_REL_L2 and max_abs(g, r) < max(_ulp_bound(r), LN_MAX_ABS)
     again = run(enc)
     for g, a in zip(got, again):
         assert np.array_equal(g, a)

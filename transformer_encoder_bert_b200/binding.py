@@ -43,15 +43,14 @@ SIGNATURES = {
     "enc_graph_create": (_i, [_vp, _vp, _vp, _vp, _i, _i, ctypes.POINTER(_vp)]),
     "enc_graph_launch": (_i, [_vp, _vp]),
     "enc_graph_destroy": (_i, [_vp]),
-    "enc_kernels_per_forward": (_i, [_vp]),
+    "enc_kernels_per_forward": (_i, [_vp, _i, _i]),
     "enc_launch_count": (ctypes.c_uint64, [_vp]),
     "enc_set_trace_events": (_i, [_vp, _vp, _i]),
     "enc_op_qkv": (_i, [_vp, _i, _vp, _vp, _i, _i, _vp]),
     "enc_op_attention": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
-    "enc_op_out_proj": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp]),
-    "enc_op_layernorm": (_i, [_vp, _i, _i, _vp, _vp, _i, _vp]),
+    "enc_op_out_proj_ln": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp]),
     "enc_op_ffn1": (_i, [_vp, _i, _vp, _vp, _i, _vp]),
-    "enc_op_ffn2": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp]),
+    "enc_op_ffn2_ln": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp]),
 }
 
 
@@ -218,8 +217,8 @@ class Encoder:
                                          ctypes.byref(g)))
         return RecordedForward(self, g, (x, valid_len, out))
 
-    def kernels_per_forward(self) -> int:
-        return int(self.lib.enc_kernels_per_forward(self.handle))
+    def kernels_per_forward(self, batch: int, seq: int) -> int:
+        return int(self.lib.enc_kernels_per_forward(self.handle, batch, seq))
 
     def launch_count(self) -> int:
         return int(self.lib.enc_launch_count(self.handle))
@@ -259,23 +258,18 @@ class Encoder:
         _check(self.lib.enc_op_attention(self.handle, _dptr(qkv), _dptr(valid_len), _dptr(ctx), batch, seq,
                                          _current_stream(stream)))
 
-    def op_out_proj(self, layer: int, ctx, resid, z, tokens: int, stream=None):
-        """z = ctx Wo + bo + resid."""
-        _check(self.lib.enc_op_out_proj(self.handle, layer, _dptr(ctx), _dptr(resid), _dptr(z), tokens,
-                                        _current_stream(stream)))
-
-    def op_layernorm(self, layer: int, which: int, z, out, tokens: int, stream=None):
-        """out = LN(z) with the layer's first (which=1) or second (which=2) gamma/beta."""
-        _check(self.lib.enc_op_layernorm(self.handle, layer, which, _dptr(z), _dptr(out), tokens,
-                                         _current_stream(stream)))
+    def op_out_proj_ln(self, layer: int, ctx, resid, out, tokens: int, stream=None):
+        """out = LN1(ctx Wo + bo + resid)."""
+        _check(self.lib.enc_op_out_proj_ln(self.handle, layer, _dptr(ctx), _dptr(resid), _dptr(out), tokens,
+                                           _current_stream(stream)))
 
     def op_ffn1(self, layer: int, h1, u, tokens: int, stream=None):
         _check(self.lib.enc_op_ffn1(self.handle, layer, _dptr(h1), _dptr(u), tokens, _current_stream(stream)))
 
-    def op_ffn2(self, layer: int, u, resid, z, tokens: int, stream=None):
-        """z = u W2 + b2 + resid."""
-        _check(self.lib.enc_op_ffn2(self.handle, layer, _dptr(u), _dptr(resid), _dptr(z), tokens,
-                                    _current_stream(stream)))
+    def op_ffn2_ln(self, layer: int, u, resid, out, tokens: int, stream=None):
+        """out = LN2(u W2 + b2 + resid)."""
+        _check(self.lib.enc_op_ffn2_ln(self.handle, layer, _dptr(u), _dptr(resid), _dptr(out), tokens,
+                                       _current_stream(stream)))
 
 
 class RecordedForward:

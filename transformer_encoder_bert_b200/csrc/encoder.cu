@@ -116,6 +116,8 @@ struct enc_handle {
   bool no_tma_store = false;        // ENC_GEMM_NO_TMA_STORE=1: epilogue stores without TMA
   bool no_tc_attn = false;          // ENC_ATTN_NO_TC=1: mma.sync attention for every length
   bool no_splitk = false;           // ENC_GEMM_NO_SPLITK=1: no split-K for small GEMMs (comparison runs)
+  bool no_ln_fuse = false;          // ENC_LN_NO_FUSE=1: LayerNorm as its own kernel (comparison runs)
+  bool ln_fuse_oproj = false;       // ENC_LN_FUSE_OPROJ=1: fuse LayerNorm 1 into the out-proj GEMM too
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -207,7 +209,8 @@ int choose_splits(const enc_handle* h, int M, int N, int K, int bn) {
 // One GEMM step: C = A * W (+ epilogue), dispatched on the handle's dtype.
 enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const CUtensorMap* wmaps, int N,
                     enc::Epi epi, const float* bias, void* C, enc::SplitShape sp, cudaStream_t st,
-                    const int* m_dev = nullptr, const void* resid = nullptr) {
+                    const int* m_dev = nullptr, const void* resid = nullptr, const float* ln_g = nullptr,
+                    const float* ln_b = nullptr) {
   if (h->dtype == ENC_FP16) {
     const int bn = choose_bn(h, M, N);
     CUtensorMap ta;
@@ -223,10 +226,10 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
       else
         use_tc = enc::encode_output_map_2d(&tc, C, (uint64_t)M, (uint64_t)N);
     }
-    // The residual of kBiasResidStore comes in by TMA in the same 32x32 boxes
+    // The residual of kBiasResidStore / kBiasResidLN comes in by TMA in the same 32x32 boxes
     // the output leaves in (only with TMA stores).
     CUtensorMap tr;
-    const bool use_tr = use_tc && epi == enc::Epi::kBiasResidStore && resid &&
+    const bool use_tr = use_tc && (epi == enc::Epi::kBiasResidStore || epi == enc::Epi::kBiasResidLN) && resid &&
                         enc::encode_output_map_2d(&tr, const_cast<void*>(resid), (uint64_t)M, (uint64_t)N);
     enc::TcGemmArgs a;
     a.tmap_a = &ta;
@@ -241,6 +244,10 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
     a.m_dev = m_dev;
     a.splits = choose_splits(h, M, N, K, bn);
     a.resid = static_cast<const __half*>(resid);
+    a.ln_gamma = ln_g;
+    a.ln_beta = ln_b;
+    if (epi == enc::Epi::kBiasResidLN && (bn != enc::kPairTile || a.splits != 1 || !use_tr))
+      return fail(ENC_ERR_UNSUPPORTED, "fused LayerNorm GEMM needs 2-CTA tiles and TMA residual/output maps");
     cudaError_t e = enc::launch_gemm_tc(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core GEMM launch");
     ++h->launches;
@@ -293,6 +300,25 @@ enc_status step_out_proj(enc_handle* h, int l, const void* ctx, const void* resi
                   resid);
 }
 
+// Whether GEMM `which` (1: output projection, 2: FFN2) writes the LayerNorm of
+// its rows (kBiasResidLN) instead of z = acc + bias + residual for a LayerNorm
+// kernel.  Needs the 2-CTA tiles to be the ones chosen for the shape (large M)
+// and H a multiple of 256.  Measured on BERT-Base shapes, the fused epilogue
+// (two passes over the accumulator and a row-statistics exchange per tile)
+// pays off behind FFN2's long K = F main loop with clusters of at most 6 CTAs
+// (H <= 768), and not behind the output projection's K = H main loop, nor with
+// 8-CTA clusters (H = 1024): those keep the separate LayerNorm kernel.
+bool ln_fused(const enc_handle* h, int tokens, int which) {
+  if (h->dtype != ENC_FP16 || h->no_ln_fuse || h->no_tma_store || !enc::gemm_ln_supported(tokens, h->H) ||
+      choose_bn(h, tokens, h->H) != enc::kPairTile)
+    return false;
+  return which == 2 ? h->H <= 768 : h->ln_fuse_oproj;
+}
+
+int kernels_per_layer(const enc_handle* h, int tokens) {
+  return 7 - (ln_fused(h, tokens, 1) ? 1 : 0) - (ln_fused(h, tokens, 2) ? 1 : 0);
+}
+
 // LayerNorm `which` (1 or 2) of z (bias and residual already added).
 enc_status step_ln(enc_handle* h, int l, int which, const void* z, void* out, int tokens, cudaStream_t st,
                    const int* rows_dev = nullptr) {
@@ -319,6 +345,15 @@ enc_status step_ffn1(enc_handle* h, int l, const void* h1, void* u, int tokens, 
   return run_gemm(h, h1, tokens, h->H, L.w_ff1, L.tm_ff1, h->F, epi, L.b_ff1, u, {}, st);
 }
 
+// Output projection + add-bias + residual + LayerNorm 1 in one GEMM:
+// out = LN1(ctx Wo + bo + resid).
+enc_status step_out_proj_ln(enc_handle* h, int l, const void* ctx, const void* resid, void* out, int tokens,
+                            cudaStream_t st, const int* m_dev = nullptr) {
+  LayerDev& L = h->layers[l];
+  return run_gemm(h, ctx, tokens, h->H, L.w_o, L.tm_o, h->H, enc::Epi::kBiasResidLN, L.b_o, out, {}, st, m_dev, resid,
+                  L.ln1_g, L.ln1_b);
+}
+
 // FFN2 with add-bias and residual in the epilogue: z = u W2 + b2 + resid
 // (resid = the first LayerNorm's output).
 enc_status step_ffn2(enc_handle* h, int l, const void* u, const void* resid, void* z, int tokens, cudaStream_t st,
@@ -326,6 +361,14 @@ enc_status step_ffn2(enc_handle* h, int l, const void* u, const void* resid, voi
   LayerDev& L = h->layers[l];
   return run_gemm(h, u, tokens, h->F, L.w_ff2, L.tm_ff2, h->H, enc::Epi::kBiasResidStore, L.b_ff2, z, {}, st, m_dev,
                   resid);
+}
+
+// FFN2 + add-bias + residual + LayerNorm 2 in one GEMM: out = LN2(u W2 + b2 + resid).
+enc_status step_ffn2_ln(enc_handle* h, int l, const void* u, const void* resid, void* out, int tokens,
+                        cudaStream_t st, const int* m_dev = nullptr) {
+  LayerDev& L = h->layers[l];
+  return run_gemm(h, u, tokens, h->F, L.w_ff2, L.tm_ff2, h->H, enc::Epi::kBiasResidLN, L.b_ff2, out, {}, st, m_dev,
+                  resid, L.ln2_g, L.ln2_b);
 }
 
 enc_status check_tokens(int batch, int seq) {
@@ -460,6 +503,8 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   if (const char* e = getenv("ENC_GEMM_NO_TMA_STORE")) h->no_tma_store = e[0] == '1';
   if (const char* e = getenv("ENC_ATTN_NO_TC")) h->no_tc_attn = e[0] == '1';
   if (const char* e = getenv("ENC_GEMM_NO_SPLITK")) h->no_splitk = e[0] == '1';
+  if (const char* e = getenv("ENC_LN_NO_FUSE")) h->no_ln_fuse = e[0] == '1';
+  if (const char* e = getenv("ENC_LN_FUSE_OPROJ")) h->ln_fuse_oproj = e[0] == '1';
   if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
   if (dtype == ENC_FP16) {
     cudaDeviceProp prop;
@@ -622,16 +667,24 @@ enc_status forward_packed(enc_handle* h, const void* x, const int32_t* valid_len
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     ++h->launches;
     mark();
-    if ((s = step_out_proj(h, l, w.ctx, xin, w.a, M, st, T)) != ENC_OK) return s;
-    mark();
-    if ((s = step_ln(h, l, 1, w.a, w.h1, M, st, T)) != ENC_OK) return s;
+    if (ln_fused(h, M, 1)) {
+      if ((s = step_out_proj_ln(h, l, w.ctx, xin, w.h1, M, st, T)) != ENC_OK) return s;
+    } else {
+      if ((s = step_out_proj(h, l, w.ctx, xin, w.a, M, st, T)) != ENC_OK) return s;
+      mark();
+      if ((s = step_ln(h, l, 1, w.a, w.h1, M, st, T)) != ENC_OK) return s;
+    }
     mark();
     const enc::Epi gelu = h->gelu == ENC_GELU_TANH ? enc::Epi::kBiasGeluTanh : enc::Epi::kBiasGelu;
     if ((s = run_gemm(h, w.h1, M, H, L.w_ff1, L.tm_ff1, h->F, gelu, L.b_ff1, w.u, {}, st, T)) != ENC_OK) return s;
     mark();
-    if ((s = step_ffn2(h, l, w.u, w.h1, w.a, M, st, T)) != ENC_OK) return s;
-    mark();
-    if ((s = step_ln(h, l, 2, w.a, xout, M, st, T)) != ENC_OK) return s;
+    if (ln_fused(h, M, 2)) {
+      if ((s = step_ffn2_ln(h, l, w.u, w.h1, xout, M, st, T)) != ENC_OK) return s;
+    } else {
+      if ((s = step_ffn2(h, l, w.u, w.h1, w.a, M, st, T)) != ENC_OK) return s;
+      mark();
+      if ((s = step_ln(h, l, 2, w.a, xout, M, st, T)) != ENC_OK) return s;
+    }
     last = xout;
   }
   mark();
@@ -655,12 +708,17 @@ enc_status run_layer(enc_handle* h, int l, const void* xin, void* xout, const in
   mark();
   if ((s = step_attention(h, w.qkv, valid_len, w.ctx, batch, seq, st)) != ENC_OK) return s;
   mark();
-  if ((s = step_out_proj(h, l, w.ctx, xin, w.a, tokens, st)) != ENC_OK) return s;
-  mark();
-  if ((s = step_ln(h, l, 1, w.a, w.h1, tokens, st)) != ENC_OK) return s;
+  if (ln_fused(h, tokens, 1)) {
+    if ((s = step_out_proj_ln(h, l, w.ctx, xin, w.h1, tokens, st)) != ENC_OK) return s;
+  } else {
+    if ((s = step_out_proj(h, l, w.ctx, xin, w.a, tokens, st)) != ENC_OK) return s;
+    mark();
+    if ((s = step_ln(h, l, 1, w.a, w.h1, tokens, st)) != ENC_OK) return s;
+  }
   mark();
   if ((s = step_ffn1(h, l, w.h1, w.u, tokens, st)) != ENC_OK) return s;
   mark();
+  if (ln_fused(h, tokens, 2)) return step_ffn2_ln(h, l, w.u, w.h1, xout, tokens, st);
   if ((s = step_ffn2(h, l, w.u, w.h1, w.a, tokens, st)) != ENC_OK) return s;
   mark();
   return step_ln(h, l, 2, w.a, xout, tokens, st);
@@ -683,6 +741,9 @@ enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, 
   Workspace w = carve(h, M);
   const int tokens = (int)M;
   tracing = tracing && !h->trace.empty();
+  if (tracing && (int)h->trace.size() < enc_kernels_per_forward(h, batch, seq) + 1)
+    return fail(ENC_ERR_INVALID_ARG, "need %d trace events for this forward, got %d",
+                enc_kernels_per_forward(h, batch, seq) + 1, (int)h->trace.size());
   int k = 0;
   auto mark = [&]() {
     if (tracing) cudaEventRecord(h->trace[k++], st);
@@ -702,6 +763,7 @@ enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, 
 
 struct enc_graph_s {
   enc_handle* h = nullptr;
+  int kernels = 0;          // launches one replay issues
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
 };
@@ -735,6 +797,7 @@ enc_status enc_graph_create(enc_t h, const void* x, const int32_t* valid_len, vo
   cudaGraph_t g = nullptr;
   e = cudaStreamEndCapture(st, &g);
   cudaStreamDestroy(st);
+  const int recorded = static_cast<int>(h->launches - launches_before);
   h->launches = launches_before;            // recording launches nothing
   if (s != ENC_OK) {
     if (g) cudaGraphDestroy(g);
@@ -749,6 +812,7 @@ enc_status enc_graph_create(enc_t h, const void* x, const int32_t* valid_len, vo
   }
   enc_graph_s* out_g = new enc_graph_s();
   out_g->h = h;
+  out_g->kernels = recorded;
   out_g->graph = g;
   out_g->exec = exec;
   ++h->graphs_alive;
@@ -760,7 +824,7 @@ enc_status enc_graph_launch(enc_graph_t graph, enc_stream_t stream) {
   if (!graph) return fail(ENC_ERR_INVALID_ARG, "null graph");
   cudaError_t e = cudaGraphLaunch(graph->exec, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaGraphLaunch");
-  graph->h->launches += enc_kernels_per_forward(graph->h);
+  graph->h->launches += graph->kernels;
   return ok();
 }
 
@@ -927,7 +991,10 @@ enc_status enc_device_status(enc_t h, int32_t* code) {
   return ok();
 }
 
-int enc_kernels_per_forward(enc_t h) { return h ? 7 * h->L + (h->packed ? 3 : 0) : 0; }
+int enc_kernels_per_forward(enc_t h, int batch, int seq) {
+  if (!h || batch <= 0 || seq <= 0) return 0;
+  return kernels_per_layer(h, batch * seq) * h->L + (h->packed ? 3 : 0);
+}
 
 enc_status enc_set_packing(enc_t h, int enable) {
   if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
@@ -960,8 +1027,8 @@ enc_status enc_set_trace_events(enc_t h, void* const* events, int count) {
     h->trace.clear();
     return ok();
   }
-  if (count < 7 * h->L + 1)
-    return fail(ENC_ERR_INVALID_ARG, "need %d trace events, got %d", 7 * h->L + 1, count);
+  if (count < 5 * h->L + 1)
+    return fail(ENC_ERR_INVALID_ARG, "need at least %d trace events, got %d", 5 * h->L + 1, count);
   h->trace.assign(reinterpret_cast<cudaEvent_t const*>(events), reinterpret_cast<cudaEvent_t const*>(events) + count);
   return ok();
 }
@@ -997,23 +1064,20 @@ enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, 
   return ok();
 }
 
-enc_status enc_op_out_proj(enc_t h, int layer, const void* ctx, const void* resid, void* z, int tokens,
-                           enc_stream_t stream) {
+enc_status enc_op_out_proj_ln(enc_t h, int layer, const void* ctx, const void* resid, void* out, int tokens,
+                              enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
-  if ((s = check_ptrs({ctx, resid, z})) != ENC_OK) return s;
-  if ((s = step_out_proj(h, layer, ctx, resid, z, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK)
-    return s;
-  return ok();
-}
-
-enc_status enc_op_layernorm(enc_t h, int layer, int which, const void* z, void* out, int tokens,
-                            enc_stream_t stream) {
-  enc_status s = op_prologue(h, layer, true, tokens);
-  if (s != ENC_OK) return s;
-  if (which != 1 && which != 2) return fail(ENC_ERR_INVALID_ARG, "which must be 1 or 2");
-  if ((s = check_ptrs({z, out})) != ENC_OK) return s;
-  if ((s = step_ln(h, layer, which, z, out, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  if ((s = check_ptrs({ctx, resid, out})) != ENC_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (ln_fused(h, tokens, 1)) {
+    if ((s = step_out_proj_ln(h, layer, ctx, resid, out, tokens, st)) != ENC_OK) return s;
+    return ok();
+  }
+  if ((s = ensure_workspace(h, (size_t)tokens)) != ENC_OK) return s;   // z in the workspace
+  const Workspace w = carve(h, (size_t)tokens);
+  if ((s = step_out_proj(h, layer, ctx, resid, w.a, tokens, st)) != ENC_OK) return s;
+  if ((s = step_ln(h, layer, 1, w.a, out, tokens, st)) != ENC_OK) return s;
   return ok();
 }
 
@@ -1025,12 +1089,20 @@ enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens, 
   return ok();
 }
 
-enc_status enc_op_ffn2(enc_t h, int layer, const void* u, const void* resid, void* z, int tokens,
-                       enc_stream_t stream) {
+enc_status enc_op_ffn2_ln(enc_t h, int layer, const void* u, const void* resid, void* out, int tokens,
+                          enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
-  if ((s = check_ptrs({u, resid, z})) != ENC_OK) return s;
-  if ((s = step_ffn2(h, layer, u, resid, z, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
+  if ((s = check_ptrs({u, resid, out})) != ENC_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (ln_fused(h, tokens, 2)) {
+    if ((s = step_ffn2_ln(h, layer, u, resid, out, tokens, st)) != ENC_OK) return s;
+    return ok();
+  }
+  if ((s = ensure_workspace(h, (size_t)tokens)) != ENC_OK) return s;   // z in the workspace
+  const Workspace w = carve(h, (size_t)tokens);
+  if ((s = step_ffn2(h, layer, u, resid, w.a, tokens, st)) != ENC_OK) return s;
+  if ((s = step_ln(h, layer, 2, w.a, out, tokens, st)) != ENC_OK) return s;
   return ok();
 }
 

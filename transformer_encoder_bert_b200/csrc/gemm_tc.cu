@@ -354,6 +354,189 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
   return true;
 }
 
+// ---------------------------------------------------------------------------
+// Fused LayerNorm epilogue (kBiasResidLN) for the 2-CTA kernel run in clusters
+// of P pairs that cover a whole row of N = 256 P columns.  The source page
+// ("Faster Transformer 优化原理") runs add-bias + residual + LayerNorm as a
+// separate kernel after the GEMM; here the GEMM writes the normalised row.
+//   Pass 1: each epilogue warp forms z = acc + bias + residual for its 32 rows
+//     x 128 columns (residual by TMA, as in kBiasResidStore), writes z back
+//     into the accumulator's TMEM columns and keeps per-row (mean, M2) of its
+//     128 values, merged chunk by chunk with the pairwise update of Chan,
+//     Golub and LeVeque (1979), which has no E[z^2] - E[z]^2 cancellation.
+//   Exchange: the (mean, M2) halves go to shared memory; once the CTA's 8 warps
+//     have written theirs, one thread arrives (release, cluster scope) on the
+//     matching barrier of the CTA with the same rows in each other pair; each
+//     CTA then reads the other pairs' halves through distributed shared
+//     memory and merges all 2P of them in a fixed order.
+//   Pass 2: out = (z - mean) * rsqrt(M2 / N + eps) * gamma + beta, from TMEM,
+//     stored as FP16 through the staging buffers and TMA stores.
+// The statistics are double-buffered by tile parity: a pair writes buffer b
+// again only two tiles later, after every other pair has signalled the tile in
+// between, i.e. after they have read buffer b.
+// ---------------------------------------------------------------------------
+struct LnCtx {
+  float2* stats;          // [2 buffers][2 halves][128 rows] (mean, M2)
+  uint32_t local_bar;     // 8 epilogue warps of this CTA, one phase per tile
+  uint32_t ready_bar0;    // + 8 * buffer: one arrival from each other pair
+  int pairs;              // P
+  int pair;               // this CTA's pair in the cluster
+  int rir;                // this CTA's index in its pair (its 128 rows)
+};
+
+// Pairwise update (Chan, Golub and LeVeque 1979) of (count, mean, M2) with a
+// group of nb values whose mean is mb and sum of squared deviations qb.
+__device__ __forceinline__ void chan_merge(float& n, float& mean, float& m2, float nb, float mb, float qb) {
+  const float nn = n + nb;
+  const float d = mb - mean;
+  mean = fmaf(d, nb / nn, mean);
+  m2 = m2 + qb + d * d * (n * nb / nn);
+  n = nn;
+}
+
+template <typename WaitFull, typename Release>
+__device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int col_begin, int N,
+                                                 const float* __restrict__ bias, const float* __restrict__ gamma,
+                                                 const float* __restrict__ beta, float* par_s, const CUtensorMap* tm_c,
+                                                 EpiWarpState& ws, const LnCtx& ln, int slice, int rloc,
+                                                 bool signaller, uint32_t local, WaitFull wait_full,
+                                                 Release release) {
+  constexpr int CHUNKS = 4;                    // 128 columns per warp
+  const int lane = threadIdx.x & 31;
+  {
+    const int i = lane * 4;                    // bias, gamma, beta of the warp's 128 columns
+    float4 b = make_float4(0.f, 0.f, 0.f, 0.f), g = b, t = b;
+    if (col_begin + i < N) {
+      b = __ldg(reinterpret_cast<const float4*>(bias + col_begin + i));
+      g = __ldg(reinterpret_cast<const float4*>(gamma + col_begin + i));
+      t = __ldg(reinterpret_cast<const float4*>(beta + col_begin + i));
+    }
+    *reinterpret_cast<float4*>(par_s + i) = b;
+    *reinterpret_cast<float4*>(par_s + 128 + i) = g;
+    *reinterpret_cast<float4*>(par_s + 256 + i) = t;
+  }
+  auto buf_of = [&](int j) { return ws.stage + ((ws.seq + j) & 1u) * kStageChunkBytes; };
+  auto issue_res = [&](int j) {                // lane 0: residual chunk j, once every store has read its buffer
+    sm100::bulk_wait_group_read<0>();
+    const uint32_t bar = ws.res_bar + 8u * ((ws.seq + j) & 1u);
+    sm100::mbar_arrive_expect_tx(bar, kStageChunkBytes);
+    sm100::tma_load_2d(ws.tm_r, sm100::smem_u32(buf_of(j)), bar, col_begin + 32 * j, row0);
+  };
+  if (lane == 0) issue_res(0);
+  int got = 0;
+  if (lane == 0) got = wait_full() ? 1 : 0;
+  got = __shfl_sync(0xffffffffu, got, 0);      // also orders the parameter staging before its use
+  if (!got) return false;
+  sm100::tc_fence_after();
+
+  // Pass 1.
+  float n = 0.f, mean = 0.f, m2 = 0.f;
+  uint32_t ra[32], rb[32];
+  sm100::tmem_ld_32x32b_x32_async(t_cols, ra);
+#pragma unroll
+  for (int j = 0; j < CHUNKS; ++j) {
+    uint32_t(&cur)[32] = (j & 1) ? rb : ra;
+    uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
+    sm100::tmem_wait_ld(cur);
+    if (j + 1 < CHUNKS) sm100::tmem_ld_32x32b_x32_async(t_cols + 32 * (j + 1), nxt);
+    if (lane == 0 && j + 1 < CHUNKS) issue_res(j + 1);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]) + par_s[32 * j + i];
+    const uint32_t k = (ws.seq + j) & 1u;
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) return false;
+    ws.res_phase ^= 1u << k;
+    const uint8_t* buf = buf_of(j);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) add_residual_unit(v, u, *reinterpret_cast<const uint4*>(buf + stage_unit(lane, u)));
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s4[i & 3] += v[i];
+    const float mc = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * (1.0f / 32.0f);
+    float q4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float d = v[i] - mc;
+      q4[i & 3] = fmaf(d, d, q4[i & 3]);
+    }
+    chan_merge(n, mean, m2, 32.0f, mc, (q4[0] + q4[1]) + (q4[2] + q4[3]));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) cur[i] = __float_as_uint(v[i]);
+    sm100::tmem_st_32x32b_x32(t_cols + 32 * j, cur);     // z replaces the accumulator
+  }
+
+  // Exchange.
+  const uint32_t b = local & 1u;
+  ln.stats[(b * 2 + slice) * 128 + rloc] = make_float2(mean, m2);
+  __syncwarp();
+  int ok = 1;
+  if (lane == 0) {
+    mbar_arrive(ln.local_bar);
+    ok = mbar_wait(ln.local_bar, local & 1u, kWaitLimitNs) ? 1 : 0;
+    if (ok && signaller) {
+      for (int p = 0; p < ln.pairs; ++p)
+        if (p != ln.pair) mbar_arrive_remote_release(mapa_shared(ln.ready_bar0 + 8u * b, 2 * p + ln.rir));
+    }
+    if (ok && ln.pairs > 1)
+      ok = mbar_wait_acquire_cluster(ln.ready_bar0 + 8u * b, (local >> 1) & 1u, kWaitLimitNs) ? 1 : 0;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (!ok) return false;
+  float tn = 0.f, tmean = 0.f, tm2 = 0.f;
+  const uint32_t st0 = sm100::smem_u32(ln.stats + (b * 2) * 128 + rloc);
+  for (int p = 0; p < ln.pairs; ++p) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint32_t addr = st0 + hf * 128 * 8;
+      const float2 h = p == ln.pair ? ln.stats[(b * 2 + hf) * 128 + rloc]
+                                    : ld_cluster_f2(mapa_shared(addr, 2 * p + ln.rir));
+      chan_merge(tn, tmean, tm2, 128.0f, h.x, h.y);
+    }
+  }
+  const float rstd = rsqrtf(tm2 / (float)N + kLnEps);
+
+  // Pass 2.
+  sm100::tmem_ld_32x32b_x32_async(t_cols, ra);
+#pragma unroll
+  for (int j = 0; j < CHUNKS; ++j) {
+    uint32_t(&cur)[32] = (j & 1) ? rb : ra;
+    uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
+    sm100::tmem_wait_ld(cur);
+    if (j + 1 < CHUNKS) sm100::tmem_ld_32x32b_x32_async(t_cols + 32 * (j + 1), nxt);
+    if (j + 1 == CHUNKS) {
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) release();
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float o0 = fmaf((__uint_as_float(cur[i]) - tmean) * rstd, par_s[128 + 32 * j + i], par_s[256 + 32 * j + i]);
+      const float o1 =
+          fmaf((__uint_as_float(cur[i + 1]) - tmean) * rstd, par_s[128 + 32 * j + i + 1], par_s[256 + 32 * j + i + 1]);
+      pk[i >> 1] = pack_half2(o0, o1);
+    }
+    uint8_t* buf = buf_of(j);
+    if (lane == 0) sm100::bulk_wait_group_read<1>();   // the store two chunks back has read buf
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4*>(buf + stage_unit(lane, u)) =
+          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+    sm100::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      sm100::tma_store_2d(tm_c, sm100::smem_u32(buf), col_begin + 32 * j, row0);
+      sm100::bulk_commit_group();
+    }
+  }
+  ws.seq += CHUNKS;
+  return true;
+}
+
 template <int BN, Epi EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -528,19 +711,30 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;             // two 256-column accumulators
   static constexpr int kResBar0 = 2 * kStages + 5;
-  static constexpr int kNumBars = kResBar0 + 2 * kEpiWarps;
+  static constexpr int kLnBar0 = kResBar0 + 2 * kEpiWarps;   // LayerNorm: local, ready[2]
+  static constexpr int kNumBars = kLnBar0 + 3;
   static constexpr int kBiasOffset = (kStages * kStageBytes + kNumBars * 8 + 16 + 15) / 16 * 16;
-  static constexpr int kStoreOffset = (kBiasOffset + kEpiWarps * (256 / kEpiSlices) * 4 + 1023) / 1024 * 1024;
+  // Per epilogue warp: bias (and, for the fused LayerNorm, gamma and beta) of its columns.
+  static constexpr int kParamFloats = 3 * (256 / kEpiSlices);
+  static constexpr int kStatsOffset = (kBiasOffset + kEpiWarps * kParamFloats * 4 + 15) / 16 * 16;
+  static constexpr int kStatsBytes = 2 * 2 * 128 * 8;       // LayerNorm statistics, [2][2][128] float2
+  static constexpr int kStoreOffset = (kStatsOffset + kStatsBytes + 1023) / 1024 * 1024;
   static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * 2 * (32 * 32 * 2);
 };
 
-template <Epi EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// CL = CTAs per cluster: 2 (one pair) for every epilogue but the fused
+// LayerNorm, which runs N / 128 CTAs (N / 256 pairs) per cluster, one pair
+// per 256-column block of the same 256 rows.  The pair of CTA rank r is
+// {r & ~1, r | 1}; its leader is r & ~1.
+template <Epi EPI, int CL>
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
                         int use_tma_store, int M_max, int N, int K,
                         const float* __restrict__ bias, __half* __restrict__ C, SplitShape sp,
-                        int* __restrict__ status, const int* __restrict__ m_dev, const __half* __restrict__ resid) {
+                        int* __restrict__ status, const int* __restrict__ m_dev, const __half* __restrict__ resid,
+                        const float* __restrict__ ln_gamma, const float* __restrict__ ln_beta) {
+  constexpr bool kLn = EPI == Epi::kBiasResidLN;
   using G = PairCfg;
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -562,8 +756,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1;
-  const int num_pairs = gridDim.x >> 1;
+  const uint32_t rir = rank & 1u;                 // CTA within its pair: rows [128 rir, 128 rir + 128)
+  const uint32_t lead = rank & ~1u;               // the pair's leader (issues the MMAs)
+  const uint16_t pair_mask = static_cast<uint16_t>(3u << lead);
+  const int pic = static_cast<int>(rank >> 1);    // pair within the cluster (column block, fused LayerNorm)
+  const int cluster = blockIdx.x / CL;
+  const int num_clusters = gridDim.x / CL;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G::kStages; ++s) {
@@ -576,6 +774,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain_bar, 1);
     for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(bar0 + 8u * (G::kResBar0 + i), 1);
+    mbar_init(bar0 + 8u * G::kLnBar0, kEpiWarps);
+    for (int i = 1; i <= 2; ++i) mbar_init(bar0 + 8u * (G::kLnBar0 + i), CL > 2 ? CL / 2 - 1 : 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -596,29 +796,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int M = m_dev ? min(*m_dev, M_max) : M_max;
   const int num_m = (M + 255) / 256;
   const int num_n = (N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
   const int num_kb = (K + kBK - 1) / kBK;
+  // Work items walked by each cluster: 256x256 tiles, or (fused LayerNorm)
+  // 256-row blocks whose column block is the pair's index in the cluster.
+  const int num_work = kLn ? num_m : num_m * num_n;
+  auto work_tile = [&](int w, int& m_blk, int& n_blk) {
+    if (kLn) {
+      m_blk = w;
+      n_blk = pic;
+    } else {
+      m_blk = w / num_n;
+      n_blk = w - m_blk * num_n;
+    }
+  };
 
   bool ok = true;
   uint32_t issued = 0;
   if (warp == 0) {
     if (lane == 0) {
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int m_blk = tile / num_n;
-        const int n_blk = tile - m_blk * num_n;
-        const int a_row = m_blk * 256 + (int)rank * 128;
-        const int b_row = n_blk * BN + (int)rank * 128;
+      for (int w = cluster; w < num_work && ok; w += num_clusters) {
+        int m_blk, n_blk;
+        work_tile(w, m_blk, n_blk);
+        const int a_row = m_blk * 256 + (int)rir * 128;
+        const int b_row = n_blk * BN + (int)rir * 128;
         for (int kb = 0; kb < num_kb; ++kb, ++issued) {
           const int s = issued % G::kStages;
           const uint32_t ph = (issued / G::kStages) & 1u;
           if (!mbar_wait(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
-          const uint32_t leader_full = mapa_shared(full_bar(s), 0);
+          const uint32_t leader_full = mapa_shared(full_bar(s), lead);
           mbar_arrive_expect_tx_cluster(leader_full, G::kStageBytes);
           tma_load_2d_pair(&tm_a, smem_u32(sA + s * G::kABytes), leader_full, kb * kBK, a_row);
           tma_load_2d_pair(&tm_b, smem_u32(sB + s * G::kBBytes), leader_full, kb * kBK, b_row);
         }
       }
-      if (rank == 0) {
+      if (rir == 0) {
         // Every copy of both CTAs counted on the leader's full barriers has landed.
         const uint32_t first = issued > (uint32_t)G::kStages ? issued - G::kStages : 0u;
         for (uint32_t j = first; j < issued; ++j)
@@ -626,10 +837,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (lane == 0 && rir == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(256, BN);
       uint32_t it = 0, local = 0;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+      for (int w = cluster; w < num_work && ok; w += num_clusters, ++local) {
         const uint32_t acc = local & 1u;
         const uint32_t aph = (local >> 1) & 1u;
         if (!mbar_wait(tempty_bar(acc), aph ^ 1u, kWaitLimitNs)) { ok = false; break; }
@@ -647,12 +858,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mma_f16_ss_pair(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
                             (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit_pair(empty_bar(s), 0x3);
+          mma_commit_pair(empty_bar(s), pair_mask);
         }
         if (!ok) break;
-        mma_commit_pair(tfull_bar(acc), 0x3);
+        mma_commit_pair(tfull_bar(acc), pair_mask);
       }
-      mma_commit_pair(drain_bar, 0x3);
+      mma_commit_pair(drain_bar, pair_mask);
     }
     if (lane == 0) mbar_wait(drain_bar, 0, kWaitLimitNs);   // the leader's MMAs are done
     __syncwarp();
@@ -667,20 +878,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ws.stage = store_smem + (warp - 2) * 2 * kStageChunkBytes;
     ws.tm_r = (use_tma_store & 2) ? &tm_r : nullptr;     // residual through TMA (kBiasResidStore)
     ws.res_bar = bar0 + 8u * (G::kResBar0 + 2 * (warp - 2));
-    const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0);
-    const uint32_t leader_tempty1 = mapa_shared(tempty_bar(1), 0);
+    const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), lead);
+    const uint32_t leader_tempty1 = mapa_shared(tempty_bar(1), lead);
+    LnCtx ln;
+    ln.stats = reinterpret_cast<float2*>(smem + G::kStatsOffset);
+    ln.local_bar = bar0 + 8u * G::kLnBar0;
+    ln.ready_bar0 = bar0 + 8u * (G::kLnBar0 + 1);
+    ln.pairs = CL / 2;
+    ln.pair = pic;
+    ln.rir = static_cast<int>(rir);
+    float* par_s = reinterpret_cast<float*>(smem + G::kBiasOffset) + (warp - 2) * G::kParamFloats;
     uint32_t local = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
-      const int m_blk = tile / num_n;
-      const int n_blk = tile - m_blk * num_n;
+    for (int w = cluster; w < num_work; w += num_clusters, ++local) {
+      int m_blk, n_blk;
+      work_tile(w, m_blk, n_blk);
       const uint32_t acc = local & 1u;
       const uint32_t aph = (local >> 1) & 1u;
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + slice * kCols;
-      const int row0 = m_blk * 256 + (int)rank * 128 + quad * 32;
-      const bool got = epilogue_warp_tile<EPI, kChunks>(
-          t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, ws, resid,
-          [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); },
-          [&] { mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0); });
+      const int row0 = m_blk * 256 + (int)rir * 128 + quad * 32;
+      auto wait_full = [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); };
+      auto release = [&] { mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0); };
+      bool got;
+      if constexpr (kLn)
+        got = epilogue_ln_tile(t_cols, row0, n_blk * BN + slice * kCols, N, bias, ln_gamma, ln_beta, par_s, tmc,
+                               ws, ln, slice, quad * 32 + lane, warp == 2, local, wait_full, release);
+      else
+        got = epilogue_warp_tile<EPI, kChunks>(t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp,
+                                              tmc, ws, resid, wait_full, release);
       if (!got) { ok = false; break; }
     }
     if (lane == 0) bulk_wait_group_all();      // every TMA store of this warp has completed
@@ -701,39 +925,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // tiles through tmap_r (only with TMA stores).
 int store_flags(const TcGemmArgs& a) { return (a.tmap_c ? 1 : 0) | (a.tmap_c && a.tmap_r ? 2 : 0); }
 
-template <Epi EPI>
-cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
+// Clusters of CL CTAs of this kernel that fit on the GPU at once (a persistent
+// grid larger than that would run its last clusters as a second wave).
+template <Epi EPI, int CL>
+int pair_max_clusters(cudaError_t& err) {
   using G = PairCfg;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_tc_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(gemm_tc_pair_kernel<EPI, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     G::kSmem);
     if (attr_err != cudaSuccess) return;
-    // How many 2-CTA clusters of this kernel fit on the GPU at once: a persistent
-    // grid larger than that would run its last clusters as a second wave.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 512, 1, 1);
+    cfg.gridDim = dim3(CL * 256, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = G::kSmem;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.x = CL;
     attr.val.clusterDim.y = 1;
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, gemm_tc_pair_kernel<EPI>, &cfg);
-    if (getenv("ENC_DEBUG")) fprintf(stderr, "[enc] pair GEMM: %d co-resident clusters\n", max_clusters);
+    attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, gemm_tc_pair_kernel<EPI, CL>, &cfg);
+    if (getenv("ENC_DEBUG")) fprintf(stderr, "[enc] pair GEMM (%d-CTA clusters): %d co-resident\n", CL, max_clusters);
   });
-  if (attr_err != cudaSuccess) return attr_err;
+  err = attr_err;
+  return max_clusters;
+}
+
+template <Epi EPI, int CL>
+cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
+  using G = PairCfg;
+  cudaError_t err;
+  const int max_clusters = pair_max_clusters<EPI, CL>(err);
+  if (err != cudaSuccess) return err;
   if (max_clusters <= 0) return cudaErrorInvalidConfiguration;
-  const int tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
-  const int pairs = tiles < max_clusters ? tiles : max_clusters;
-  return launch_kernel(gemm_tc_pair_kernel<EPI>, dim3(2 * pairs), dim3(kThreads), G::kSmem, stream, nullptr, 0,
-                       *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_r ? *a.tmap_r : *a.tmap_a,
-                       store_flags(a), a.M, a.N, a.K, a.bias, a.c, a.split, a.status, a.m_dev, a.resid);
+  const int num_m = (a.M + 255) / 256;
+  const int work = EPI == Epi::kBiasResidLN ? num_m : num_m * ((a.N + 255) / 256);
+  const int clusters = work < max_clusters ? work : max_clusters;
+  return launch_kernel(gemm_tc_pair_kernel<EPI, CL>, dim3(CL * clusters), dim3(kThreads), G::kSmem, stream, nullptr,
+                       0, *a.tmap_a, *a.tmap_b, a.tmap_c ? *a.tmap_c : *a.tmap_a, a.tmap_r ? *a.tmap_r : *a.tmap_a,
+                       store_flags(a), a.M, a.N, a.K, a.bias, a.c, a.split, a.status, a.m_dev, a.resid, a.ln_gamma,
+                       a.ln_beta);
 }
 
 // ---------------------------------------------------------------------------
@@ -1099,6 +1334,8 @@ bool encode_output_map_split(CUtensorMap* map, void* base, const SplitShape& sp)
          CUDA_SUCCESS;
 }
 
+bool gemm_ln_supported(int M, int N) { return M >= 256 && N % 256 == 0 && N <= 1024; }
+
 int choose_gemm_splits(int tiles, int num_kb, int num_sms) {
   if (tiles <= 0) return 1;
   for (int s = std::min(SplitCfg::kMaxSplits, num_kb); s >= 2; --s)
@@ -1129,12 +1366,22 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream) {
   if (a.bn == kPairTile) {
     if ((a.N % 256) != 0) return cudaErrorInvalidValue;
     switch (a.epi) {
-      case Epi::kStore: return launch_pair<Epi::kStore>(a, stream);
-      case Epi::kBiasGelu: return launch_pair<Epi::kBiasGelu>(a, stream);
-      case Epi::kBiasQkvSplit: return launch_pair<Epi::kBiasQkvSplit>(a, stream);
-      case Epi::kBiasGeluTanh: return launch_pair<Epi::kBiasGeluTanh>(a, stream);
-      case Epi::kBiasStore: return launch_pair<Epi::kBiasStore>(a, stream);
-      case Epi::kBiasResidStore: return launch_pair<Epi::kBiasResidStore>(a, stream);
+      case Epi::kStore: return launch_pair<Epi::kStore, 2>(a, stream);
+      case Epi::kBiasGelu: return launch_pair<Epi::kBiasGelu, 2>(a, stream);
+      case Epi::kBiasQkvSplit: return launch_pair<Epi::kBiasQkvSplit, 2>(a, stream);
+      case Epi::kBiasGeluTanh: return launch_pair<Epi::kBiasGeluTanh, 2>(a, stream);
+      case Epi::kBiasStore: return launch_pair<Epi::kBiasStore, 2>(a, stream);
+      case Epi::kBiasResidStore: return launch_pair<Epi::kBiasResidStore, 2>(a, stream);
+      case Epi::kBiasResidLN:
+        // one cluster of N/128 CTAs per 256-row block; residual and output through TMA
+        if (!a.tmap_c || !a.tmap_r || !a.ln_gamma || !a.ln_beta) return cudaErrorInvalidValue;
+        switch (a.N) {
+          case 256: return launch_pair<Epi::kBiasResidLN, 2>(a, stream);
+          case 512: return launch_pair<Epi::kBiasResidLN, 4>(a, stream);
+          case 768: return launch_pair<Epi::kBiasResidLN, 6>(a, stream);
+          case 1024: return launch_pair<Epi::kBiasResidLN, 8>(a, stream);
+        }
+        return cudaErrorInvalidValue;
     }
     return cudaErrorInvalidValue;
   }

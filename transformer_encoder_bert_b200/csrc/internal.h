@@ -19,7 +19,8 @@ enum class Epi : int {
   kBiasQkvSplit = 2, // Q/K/V head split: dst[t][b][h][s][c] = acc + bias[n]
   kBiasGeluTanh = 3, // C[m][n] = GELU_tanh(acc + bias[n])
   kBiasStore = 4,    // C[m][n] = acc + bias[n]
-  kBiasResidStore = 5  // C[m][n] = acc + bias[n] + R[m][n]  (R: the residual, [M, N] like C)
+  kBiasResidStore = 5,  // C[m][n] = acc + bias[n] + R[m][n]  (R: the residual, [M, N] like C)
+  kBiasResidLN = 6      // C[m][:] = LayerNorm(acc + bias + R)[m][:] over the row (gamma, beta)
 };
 
 // Addressing for the head-split epilogue (n = t*H + h*d + c, m = b*seq + s).
@@ -93,11 +94,16 @@ struct TcGemmArgs {
   int splits = 1;
   const __half* resid = nullptr;  // [M, N] (kBiasResidStore)
   const CUtensorMap* tmap_r = nullptr;  // the residual as an output-style map (32x32 box), or nullptr
+  const float* ln_gamma = nullptr;      // [N] (kBiasResidLN)
+  const float* ln_beta = nullptr;       // [N] (kBiasResidLN)
 };
 // The split count for a GEMM of `tiles` 128 x 128 tiles and `num_kb` 64-wide
 // k-blocks: the largest s <= min(16, num_kb) whose clusters of s CTAs all fit
 // on the GPU at once with tiles * s <= num_sms; 1 when no s >= 2 does.
 int choose_gemm_splits(int tiles, int num_kb, int num_sms);
+// Whether kBiasResidLN can run for an [M, N] GEMM: the row of N columns is
+// covered by one cluster of N/128 CTAs (N a multiple of 256, N <= 1024), M >= 256.
+bool gemm_ln_supported(int M, int N);
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream);
 
 // Encode a 2-D K-major FP16 tensor map over [rows, cols=K] with a {64, box_rows} box.
