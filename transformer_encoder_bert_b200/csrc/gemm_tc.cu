@@ -442,7 +442,13 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
     if (lane == 0 && j + 1 < CHUNKS) issue_res(j + 1);
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]) + par_s[32 * j + i];
+    for (int i = 0; i < 32; i += 4) {          // bias: one 16-byte broadcast read per 4 columns
+      const float4 b4 = *reinterpret_cast<const float4*>(par_s + 32 * j + i);
+      v[i] = __uint_as_float(cur[i]) + b4.x;
+      v[i + 1] = __uint_as_float(cur[i + 1]) + b4.y;
+      v[i + 2] = __uint_as_float(cur[i + 2]) + b4.z;
+      v[i + 3] = __uint_as_float(cur[i + 3]) + b4.w;
+    }
     const uint32_t k = (ws.seq + j) & 1u;
     int ok = 0;
     if (lane == 0) ok = mbar_wait(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
@@ -513,11 +519,15 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
     }
     uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float o0 = fmaf((__uint_as_float(cur[i]) - tmean) * rstd, par_s[128 + 32 * j + i], par_s[256 + 32 * j + i]);
-      const float o1 =
-          fmaf((__uint_as_float(cur[i + 1]) - tmean) * rstd, par_s[128 + 32 * j + i + 1], par_s[256 + 32 * j + i + 1]);
+    for (int i = 0; i < 32; i += 4) {          // gamma, beta: 16-byte broadcast reads
+      const float4 g4 = *reinterpret_cast<const float4*>(par_s + 128 + 32 * j + i);
+      const float4 t4 = *reinterpret_cast<const float4*>(par_s + 256 + 32 * j + i);
+      const float o0 = fmaf((__uint_as_float(cur[i]) - tmean) * rstd, g4.x, t4.x);
+      const float o1 = fmaf((__uint_as_float(cur[i + 1]) - tmean) * rstd, g4.y, t4.y);
+      const float o2 = fmaf((__uint_as_float(cur[i + 2]) - tmean) * rstd, g4.z, t4.z);
+      const float o3 = fmaf((__uint_as_float(cur[i + 3]) - tmean) * rstd, g4.w, t4.w);
       pk[i >> 1] = pack_half2(o0, o1);
+      pk[(i >> 1) + 1] = pack_half2(o2, o3);
     }
     uint8_t* buf = buf_of(j);
     if (lane == 0) sm100::bulk_wait_group_read<1>();   // the store two chunks back has read buf
