@@ -115,7 +115,8 @@ ENC_API enc_status enc_set_gelu(enc_t h, enc_gelu form);
  * mode).  Valid outputs agree with the default mode to rounding.  The page
  * fixes the sequence length for performance and plans arbitrary lengths
  * ([FT] "什么是 Faster Transformer"); this removes the padding's cost instead.
- * A forward then launches 7 kernels per layer plus 3 (offsets, pack, unpack). */
+ * A forward then launches 3 kernels more (offsets, pack, unpack);
+ * enc_kernels_per_forward gives the total. */
 ENC_API enc_status enc_set_packing(enc_t h, int enable);
 
 /* enc_set_host_chunks - most chunks enc_forward_host cuts a batch into (1..4,

@@ -174,10 +174,11 @@ def test_fp32_steps(shape):
     assert rel_l2(to_host(y), ref_y) < FP32_REL_L2
 
 
-@pytest.mark.parametrize("seq", [40, 100], ids=str)
+@pytest.mark.parametrize("seq", [40, 100, 300], ids=str)
 def test_attention_valid_len_clamping_and_empty(seq):
     """Lengths outside [0, seq] are clamped; n == 0 gives ctx = 0 (seq 40 runs the
-    mma.sync kernel, seq 100 the tensor-core one)."""
+    mma.sync kernel, seq 100 the one-block tensor-core kernel, seq 300 the
+    multi-block one)."""
     shape = (12, 64, 3072)
     nh, d, _ = shape
     batch = 4
@@ -258,10 +259,11 @@ def test_alternative_gemm_paths(monkeypatch, env, batch, seq):
     assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < LN_MAX_ABS
 
 
-@pytest.mark.parametrize("batch,seq", [(3, 128), (4, 96), (3, 65)], ids=str)
+@pytest.mark.parametrize("batch,seq", [(3, 128), (4, 96), (3, 65), (2, 200)], ids=str)
 def test_attention_mma_sync_path_for_long_sequences(monkeypatch, batch, seq):
-    """Size-64 heads on sequences of 65..128 run on the tensor-core (tcgen05) kernel;
-    the mma.sync kernel for the same shapes stays checked through ENC_ATTN_NO_TC."""
+    """Size-64 heads on sequences longer than 64 run on the tensor-core (tcgen05)
+    kernels; the mma.sync kernel for the same shapes stays checked through
+    ENC_ATTN_NO_TC."""
     monkeypatch.setenv("ENC_ATTN_NO_TC", "1")
     shape = (12, 64, 3072)
     nh, d, _ = shape
@@ -273,6 +275,36 @@ def test_attention_mma_sync_path_for_long_sequences(monkeypatch, batch, seq):
     got = to_host(ctx).reshape(batch, seq, nh * d)
     ref = O.attention(qkv.astype(np.float64), vlen)
     assert rel_l2(got, ref) < ATTN_REL_L2
+
+
+@pytest.mark.parametrize("batch,seq,lens", [
+    (3, 300, [300, 129, 1]),          # 3 query blocks: the second CTA's upper block lies past seq
+    (2, 256, [256, 128]),             # key blocks exactly full; one block only
+    (4, 512, [512, 385, 257, 130]),   # 1 or 2 valid keys in the last block
+    (2, 129, [129, 65]),
+], ids=str)
+@pytest.mark.parametrize("key_boost", [1.0, 6.0], ids=["plain", "rescaled"])
+def test_attention_long_sequences_tensor_core(batch, seq, lens, key_boost):
+    """Sequences longer than one 128-key block: the tensor-core kernel walks the
+    key blocks with a running maximum.  key_boost multiplies the keys of block j
+    by key_boost**j, so later blocks raise the row maximum far above the first
+    block's and the accumulated output and row sum must be rescaled."""
+    shape = (16, 64, 4096)
+    nh, d, _ = shape
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=29).astype(np.float32)
+    for j in range(1, (seq + 127) // 128):
+        qkv[1, :, :, 128 * j:128 * (j + 1)] *= key_boost ** j
+    qkv = qkv.astype(np.float16)
+    vlen = np.array(lens, np.int32)
+    ctx = empty_dev((batch * seq, nh * d), "fp16")
+    enc.op_attention(to_dev(qkv), to_dev(vlen), ctx, batch, seq)
+    got = to_host(ctx).reshape(batch, seq, nh * d)
+    ref = O.attention(qkv.astype(np.float64), vlen)
+    assert np.all(np.isfinite(got))
+    assert rel_l2(got, ref) < ATTN_REL_L2
+    assert max_abs(got, ref) < 4 * _ulp_bound(ref)
+    assert enc.device_status() == 0
 
 
 @pytest.mark.parametrize("batch,seq", [(1, 32), (8, 32), (1, 7), (3, 37)], ids=str)

@@ -1,6 +1,8 @@
 // Masked scaled-dot-product attention on the 5th-generation tensor cores
-// (tcgen05 + TMEM + TMA) for size_per_head 64 and 64 < seq <= 128, where one
-// block of 128 keys covers every key of a sequence.
+// (tcgen05 + TMEM + TMA) for size_per_head 64 and seq > 64.  Two kernels:
+// attention_tc_kernel for seq <= 128, where one block of 128 keys covers every
+// key of a sequence (described here), and attention_tc_long_kernel for longer
+// sequences (described above it).
 //
 // The source page ("Faster Transformer 优化原理") runs attention as two batched
 // GEMMs around a SoftMax kernel.  Here both products run on tcgen05 and the
@@ -140,7 +142,9 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x, b = blockIdx.y;
+  // Sequences are taken last to first: the QKV GEMM before this kernel writes
+  // the rows of the last sequences last, so those are the ones still in L2.
+  const int h = blockIdx.x, b = B - 1 - (int)blockIdx.y;
   pdl_wait();                                          // Q/K/V (and offsets) of the previous kernels are visible
   int n = valid_len[b];
   n = n < 0 ? 0 : (n > S ? S : n);
@@ -341,6 +345,310 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
   }
 }
 
+// ---------------------------------------------------------------------------
+// Sequences longer than one key block (seq > 128): the same per-row softmax
+// over 128-key blocks with a running maximum (online softmax).  One CTA per
+// (sequence, head, 128 query rows), 160 threads, two CTAs per SM so that one
+// CTA's loads overlap the other's softmax:
+//   warps 0..3  softmax: thread r owns query row r = TMEM lane r.  For key
+//               block j it reads its row of S_j = Q K_j^T from TMEM, writes
+//               P_j = exp(S_j/sqrt(d) - m) (FP16, swizzled K-major) and adds its
+//               row sum to l.  m is a reference maximum: it moves only when a
+//               block's maximum exceeds it by more than 2^8 in the exponent, and
+//               then O (in TMEM) and l are scaled by exp(m_old - m_new) before
+//               the next P V accumulates.  At the end it stores O / l.
+//   warp 4      one thread issues every TMA load (Q once; K blocks through a
+//               two-stage ring; V one block at a time) and every MMA:
+//               S_j into TMEM columns [0, 128), O += P_j V_j into [128, 192).
+// S_{j+1} is issued right after P_j V_j, so the next scores are ready when the
+// softmax warps finish block j.  Key blocks past n are never loaded; in the
+// last block, keys >= n get weight 0 and their V rows are zeroed.
+namespace lng {
+constexpr int kThreads = 32 * (kSoftmaxWarps + 1);
+constexpr int kQ = 0;                                       // Q tile, later the output rows
+constexpr int kK = kTileBytes;                              // K of stage st (two stages)
+constexpr int kV = 3 * kTileBytes;                          // V of the current block
+constexpr int kP = 4 * kTileBytes;                          // P: two 64-key atoms
+constexpr int kBars = 6 * kTileBytes;
+// q_full, k_full[2], k_empty[2], v_full, v_empty, s_full, p_full, o_full, drain
+constexpr int kNumBars = 11;
+constexpr int kSlot = kBars + kNumBars * 8;
+constexpr int kSmemTotal = 1024 + kSlot + 16;
+constexpr int kTmemCols = 256;
+constexpr int kOCol = 128;
+constexpr float kRescaleLog2 = 8.f;                         // P < 2^8 between rescales
+static_assert(2 * (kSmemTotal + 1024) <= 228 * 1024, "two CTAs per SM");
+}  // namespace lng
+
+template <bool PACKED>
+__global__ void __launch_bounds__(lng::kThreads, 2)
+    attention_tc_long_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int32_t* __restrict__ valid_len,
+                             const int32_t* __restrict__ offsets, __half* __restrict__ ctx, int B, int S, int NH,
+                             float score_scale_log2, int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + lng::kBars;
+  const uint32_t q_full = bar0, v_full = bar0 + 40, v_empty = bar0 + 48, s_full = bar0 + 56, p_full = bar0 + 64,
+                 o_full = bar0 + 72, drain = bar0 + 80;
+  auto k_full = [&](int st) { return bar0 + 8 + 8 * st; };
+  auto k_empty = [&](int st) { return bar0 + 24 + 8 * st; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lng::kSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = B - 1 - (int)blockIdx.z;   // last sequences first, as above
+  const int q0 = blockIdx.x * kRows;
+  pdl_wait();
+  int n = valid_len[b];
+  n = n < 0 ? 0 : (n > S ? S : n);
+  const int rows_exist = PACKED ? n : S;
+  if (q0 >= rows_exist) return;                        // no query rows here (uniform per CTA)
+  const int H = NH * kD;
+  const size_t row0 = PACKED ? (size_t)offsets[b] : (size_t)b * S;
+  if (n == 0) {                                        // fixed-length layout, empty sequence: ctx = 0
+    const int rows = min(kRows, S - q0);
+    for (int i = threadIdx.x; i < rows * 8; i += lng::kThreads)
+      *reinterpret_cast<uint4*>(ctx + (row0 + q0 + (i >> 3)) * H + h * kD + (i & 7) * 8) = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const int nb = (n + kRows - 1) / kRows;              // key blocks holding valid keys
+
+  auto coord_x = [&](int t) { return PACKED ? t * H + h * kD : 0; };
+  auto coord_y = [&](int t, int s) { return PACKED ? offsets[b] + s : ((t * B + b) * NH + h) * S + s; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < lng::kNumBars; ++i) mbar_init(bar0 + 8 * i, bar0 + 8 * i == p_full ? kSoftmaxWarps : 1);
+    fence_barrier_init();
+  }
+  if (warp == kSoftmaxWarps) {
+    tmem_alloc(smem_u32(tmem_slot), lng::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_trigger();                                       // after taking TMEM
+
+  bool ok = true;
+  if (warp == kSoftmaxWarps) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_qkv);
+      auto load_k = [&](int j) {
+        const int st = j & 1;
+        mbar_arrive_expect_tx(k_full(st), kTileBytes);
+        tma_load_2d(&tm_qkv, sbase + lng::kK + st * kTileBytes, k_full(st), coord_x(1), coord_y(1, j * kRows));
+      };
+      auto load_v = [&](int j) {
+        mbar_arrive_expect_tx(v_full, kTileBytes);
+        tma_load_2d(&tm_qkv, sbase + lng::kV, v_full, coord_x(2), coord_y(2, j * kRows));
+      };
+      mbar_arrive_expect_tx(q_full, kTileBytes);
+      tma_load_2d(&tm_qkv, sbase + lng::kQ, q_full, coord_x(0), coord_y(0, q0));
+      load_k(0);
+      if (nb > 1) load_k(1);
+      load_v(0);
+      int k_loaded = nb > 1 ? 2 : 1, v_loaded = 1;
+      constexpr uint32_t idesc_s = idesc_f16_f32(kRows, kRows);
+      constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kRows, kD);
+      auto issue_s = [&](int j) {                      // S = Q K_j^T, then K stage j & 1 is free
+        const int st = j & 1;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          mma_f16_ss(tmem, smem_desc_sw128(sbase + lng::kQ + kk * 32),
+                     smem_desc_sw128(sbase + lng::kK + st * kTileBytes + kk * 32), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        mma_commit(k_empty(st));
+      };
+      ok = mbar_wait(q_full, 0, kWaitLimitNs) && mbar_wait(k_full(0), 0, kWaitLimitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; j < nb && ok; ++j) {
+        // P_j is written (so S_j has been read and O rescaled) and V_j has landed.
+        if (!mbar_wait(p_full, j & 1, kWaitLimitNs) || !mbar_wait(v_full, j & 1, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)        // O += P_j V_j
+          mma_f16_ss(tmem + lng::kOCol, smem_desc_sw128(sbase + lng::kP + (kk >> 2) * kTileBytes + (kk & 3) * 32),
+                     desc_mn_sw128(sbase + lng::kV + kk * 16 * 128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(o_full);
+        mma_commit(v_empty);
+        if (j + 1 < nb) {
+          if (!mbar_wait(k_full((j + 1) & 1), ((j + 1) >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        if (j + 2 < nb) {                              // K_{j+2} into the stage S_j has finished with
+          if (!mbar_wait(k_empty(j & 1), (j >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
+          load_k(j + 2);
+          k_loaded = j + 3;
+        }
+        if (j + 1 < nb) {                              // V_{j+1} once P_j V_j has read V_j
+          if (!mbar_wait(v_empty, j & 1, kWaitLimitNs)) { ok = false; break; }
+          load_v(j + 1);
+          v_loaded = j + 2;
+        }
+      }
+      mma_commit(drain);                               // every MMA issued here has completed
+      mbar_wait(drain, 0, kWaitLimitNs);
+      if (!ok) {                                       // let the copies land before the CTA exits
+        mbar_wait(q_full, 0, kWaitLimitNs);
+        for (int j = k_loaded > 2 ? k_loaded - 2 : 0; j < k_loaded; ++j)
+          mbar_wait(k_full(j & 1), (j >> 1) & 1, kWaitLimitNs);
+        mbar_wait(v_full, (v_loaded - 1) & 1, kWaitLimitNs);
+      }
+    }
+  } else {
+    const int r = warp * 32 + lane;                    // query row = TMEM lane
+    const uint32_t t_s = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t t_o = t_s + lng::kOCol;
+    uint8_t* prow = smem + lng::kP + r * 128;
+    const uint64_t scale2 = f2_pack(score_scale_log2, score_scale_log2);
+    uint32_t sa[32], sb[32];
+    uint64_t sum2 = 0;                                 // two partial row sums (0.0f, 0.0f)
+    float m_ref = 0.f;                                 // the max that P, O and l are taken against
+    for (int j = 0; j < nb && ok; ++j) {
+      ok = warp_wait(s_full, j & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const int lim_blk = min(n - j * kRows, kRows);   // valid keys in this block (>= 1)
+      const int nchunks = (lim_blk + 31) >> 5;
+      // Pass 1: block max over the valid keys.
+      float bmax = -INFINITY;
+      tmem_ld_32x32b_x32_async(t_s, sa);
+#pragma unroll
+      for (int c = 0; c < kRows / 32; ++c) {
+        if (c < nchunks) {
+          uint32_t(&cur)[32] = (c & 1) ? sb : sa;
+          uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
+          tmem_wait_ld(cur);
+          if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_s + 32 * (c + 1), nxt);
+          const int lim = lim_blk - 32 * c;
+          if (lim >= 32) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, __uint_as_float(cur[i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < lim) bmax = fmaxf(bmax, __uint_as_float(cur[i]));
+          }
+        }
+      }
+      // Every P, and every term of O and l, is taken against the same reference
+      // m, so O / l is the softmax-weighted sum whatever m is; m moves (and O and
+      // l are rescaled by alpha = exp(m_old - m_new)) only to keep P below 2^8.
+      float alpha = 1.f;
+      bool moved = false;
+      if (j == 0) {
+        m_ref = bmax;
+      } else if ((bmax - m_ref) * score_scale_log2 > lng::kRescaleLog2) {
+        alpha = ex2((m_ref - bmax) * score_scale_log2);
+        m_ref = bmax;
+        moved = true;
+      }
+      if (j > 0) {                                     // P_{j-1} V_{j-1} is done: P may be rewritten
+        ok = warp_wait(o_full, (j - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, moved)) {          // O *= alpha (alpha = 1 on rows that keep theirs)
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            tmem_ld_32x32b_x32(t_o + 32 * half, sa);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sa[i] = __float_as_uint(__uint_as_float(sa[i]) * alpha);
+            tmem_st_32x32b_x32(t_o + 32 * half, sa);
+          }
+        }
+        sum2 = f2_mul(sum2, f2_pack(alpha, alpha));
+      }
+      const uint64_t neg_m2 = f2_pack(-m_ref * score_scale_log2, -m_ref * score_scale_log2);
+      // Pass 2: P_j, its row sum, FP16 P into the swizzled tile.
+      tmem_ld_32x32b_x32_async(t_s, sa);
+#pragma unroll
+      for (int c = 0; c < kRows / 32; ++c) {
+        if (c < nchunks) {
+          uint32_t(&cur)[32] = (c & 1) ? sb : sa;
+          uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
+          tmem_wait_ld(cur);
+          if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_s + 32 * (c + 1), nxt);
+          const int lim = lim_blk - 32 * c;
+          if (lim >= 32)
+            p_chunk<false>(cur, 32, scale2, neg_m2, sum2, prow, c, r);
+          else
+            p_chunk<true>(cur, lim, scale2, neg_m2, sum2, prow, c, r);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) store_p_unit(prow, 4 * c + u, r, make_uint4(0, 0, 0, 0));
+        }
+      }
+      // Last, partial block: V rows of keys >= n may hold non-finite data from
+      // outside the sequence (0 * NaN = NaN in the MMA), so zero them.
+      if (lim_blk < kRows) {
+        ok = warp_wait(v_full, j & 1);
+        if (ok && r >= lim_blk) {
+          uint4* vrow = reinterpret_cast<uint4*>(smem + lng::kV + r * 128);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) vrow[u] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();                        // P (and zeroed V rows) visible to the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) {
+      ok = warp_wait(o_full, (nb - 1) & 1);
+      if (ok) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32_async(t_o, sa);
+        tmem_ld_32x32b_x32_async(t_o + 32, sb);
+        tmem_wait_ld(sa);
+        tmem_wait_ld(sb);
+      }
+    }
+    if (ok) {
+      // Row r of O / l as FP16 into the Q tile (its last reader, the MMA of
+      // S_{nb-1}, has completed), then coalesced stores.
+      float s0, s1;
+      f2_unpack(sum2, s0, s1);
+      const float l = s0 + s1;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint8_t* orow = smem + lng::kQ + r * 128;
+#pragma unroll
+      for (int unit = 0; unit < 8; ++unit) {
+        const uint32_t(&sv)[32] = unit < 4 ? sa : sb;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = 8 * (unit & 3) + 2 * k;
+          w[k] = cvt_half2(__uint_as_float(sv[i]) * inv, __uint_as_float(sv[i + 1]) * inv);
+        }
+        *reinterpret_cast<uint4*>(orow + 16 * (unit ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      __syncwarp();
+      const int unit = lane & 7;
+#pragma unroll 1
+      for (int it = 0; it < 8; ++it) {
+        const int rr = warp * 32 + it * 4 + (lane >> 3);
+        if (q0 + rr < rows_exist) {
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + lng::kQ + rr * 128 + 16 * (unit ^ (rr & 7)));
+          *reinterpret_cast<uint4*>(ctx + (row0 + q0 + rr) * H + h * kD + unit * 8) = v;
+        }
+      }
+    }
+  }
+
+  if (!ok) atomicCAS(status, 0, kStatusWaitTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kSoftmaxWarps) {
+    tc_fence_after();
+    tmem_dealloc(tmem, lng::kTmemCols);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -363,6 +671,9 @@ cudaError_t launch_tc(const __half* qkv, const int32_t* vl, const int32_t* offse
   std::call_once(once, [] {
     attr = cudaFuncSetAttribute(attention_tc_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kSmemTotal);
+    if (attr == cudaSuccess)
+      attr = cudaFuncSetAttribute(attention_tc_long_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  lng::kSmemTotal);
   });
   if (attr != cudaSuccess) return attr;
   auto fn = encode_fn();
@@ -383,15 +694,20 @@ cudaError_t launch_tc(const __half* qkv, const int32_t* vl, const int32_t* offse
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const dim3 grid(NH, B);
   const float scale_log2 = kLog2e / sqrtf((float)kD);
+  if (S > kRows) {
+    const dim3 grid((unsigned)((S + kRows - 1) / kRows), NH, B);
+    return launch_kernel(attention_tc_long_kernel<PACKED>, grid, dim3(lng::kThreads), lng::kSmemTotal, stream,
+                         nullptr, 0, map, vl, offsets, ctx, B, S, NH, scale_log2, status);
+  }
+  const dim3 grid(NH, B);
   return launch_kernel(attention_tc_kernel<PACKED>, grid, dim3(kThreads), kSmemTotal, stream, nullptr, 0, map, vl,
                        offsets, ctx, B, S, NH, scale_log2, status);
 }
 
 }  // namespace
 
-bool attention_tc_supported(int size_per_head, int seq) { return size_per_head == kD && seq > 64 && seq <= kRows; }
+bool attention_tc_supported(int size_per_head, int seq) { return size_per_head == kD && seq > 64; }
 
 cudaError_t launch_attention_tc(const __half* qkv, const int32_t* valid_len, const int32_t* offsets, __half* ctx,
                                 int batch, int seq, int head_num, int* status, cudaStream_t stream) {

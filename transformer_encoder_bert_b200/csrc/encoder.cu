@@ -267,9 +267,10 @@ enc_status step_qkv(enc_handle* h, int l, const void* x, void* qkv, int batch, i
                   sp, st);
 }
 
-// Attention kernel choice: the tensor-core kernel for size_per_head 64 when one
-// 128-key block covers a sequence longer than the short kernel's 64-row tiles;
-// mma.sync otherwise (and for every length under ENC_ATTN_NO_TC=1).
+// Attention kernel choice: the tensor-core kernels for size_per_head 64 and
+// sequences longer than the short kernel's 64-row tiles (one 128-key block up to
+// 128, key blocks with a running maximum beyond); mma.sync otherwise (and for
+// every length under ENC_ATTN_NO_TC=1).
 bool use_tc_attention(const enc_handle* h, int seq) {
   return enc::attention_tc_supported(h->d, seq) && !h->no_tc_attn;
 }

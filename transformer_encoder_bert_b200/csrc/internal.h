@@ -143,7 +143,7 @@ cudaError_t launch_attention_f32(const float* qkv, const int32_t* valid_len, flo
                                  int batch, int seq, int head_num, int size_per_head,
                                  cudaStream_t stream);
 
-// Tensor-core attention (attention_tc.cu): size_per_head 64 and 64 < seq <= 128
+// Tensor-core attention (attention_tc.cu): size_per_head 64 and seq > 64
 // (attention_tc_supported); offsets == nullptr reads the split layout
 // [3, B, nh, S, 64], else the packed [T, 3H] layout.
 bool attention_tc_supported(int size_per_head, int seq);
