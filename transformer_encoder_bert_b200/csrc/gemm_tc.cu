@@ -36,6 +36,11 @@ namespace {
 using namespace sm100;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+// Every wait in these kernels sleeps until its phase completes (suspend-time
+// hint 100 us) rather than polling: the polling warps (epilogue warps waiting
+// out a whole main loop, producer and MMA threads) otherwise take issue slots
+// from the warps doing work.  Measured 8-10 % faster GEMMs.
+constexpr uint32_t kSleepNs = 100000;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 // Epilogue warps: 8 (two per TMEM lane quadrant) measured faster than 16 on
@@ -303,7 +308,7 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
     if (tma_resid) {
       const uint32_t k = ws.seq & 1u;
       int ok = 0;
-      if (lane == 0) ok = mbar_wait(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait<kSleepNs>(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) return false;
       ws.res_phase ^= 1u << k;
@@ -451,7 +456,7 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
     }
     const uint32_t k = (ws.seq + j) & 1u;
     int ok = 0;
-    if (lane == 0) ok = mbar_wait(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
+    if (lane == 0) ok = mbar_wait<kSleepNs>(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) return false;
     ws.res_phase ^= 1u << k;
@@ -481,13 +486,13 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
   int ok = 1;
   if (lane == 0) {
     mbar_arrive(ln.local_bar);
-    ok = mbar_wait(ln.local_bar, local & 1u, kWaitLimitNs) ? 1 : 0;
+    ok = mbar_wait<kSleepNs>(ln.local_bar, local & 1u, kWaitLimitNs) ? 1 : 0;
     if (ok && signaller) {
       for (int p = 0; p < ln.pairs; ++p)
         if (p != ln.pair) mbar_arrive_remote_release(mapa_shared(ln.ready_bar0 + 8u * b, 2 * p + ln.rir));
     }
     if (ok && ln.pairs > 1)
-      ok = mbar_wait_acquire_cluster(ln.ready_bar0 + 8u * b, (local >> 1) & 1u, kWaitLimitNs) ? 1 : 0;
+      ok = mbar_wait_acquire_cluster<kSleepNs>(ln.ready_bar0 + 8u * b, (local >> 1) & 1u, kWaitLimitNs) ? 1 : 0;
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok) return false;
@@ -617,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % G::kStages;
           const uint32_t ph = (it / G::kStages) & 1u;
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait<kSleepNs>(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(s), G::kStageBytes);
           tma_load_2d(&tm_a, smem_u32(sA + s * G::kABytes), full_bar(s), kb * kBK, m_blk * kBM);
           tma_load_2d(&tm_b, smem_u32(sB + s * G::kBBytes), full_bar(s), kb * kBK, n_blk * BN);
@@ -626,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Let every copy this thread issued land before the CTA can exit.
       const uint32_t first = it > (uint32_t)G::kStages ? it - G::kStages : 0u;
       for (uint32_t j = first; j < it; ++j)
-        mbar_wait(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
+        mbar_wait<kSleepNs>(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -635,13 +640,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
         const uint32_t acc = local & 1u;
         const uint32_t aph = (local >> 1) & 1u;
-        if (!mbar_wait(tempty_bar(acc), aph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait<kSleepNs>(tempty_bar(acc), aph ^ 1u, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % G::kStages;
           const uint32_t ph = (it / G::kStages) & 1u;
-          if (!mbar_wait(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait<kSleepNs>(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + s * G::kABytes);
           const uint32_t b_addr = smem_u32(sB + s * G::kBBytes);
@@ -657,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Every MMA this thread issued has completed once drain_bar flips.
       mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kWaitLimitNs);
+      mbar_wait<kSleepNs>(drain_bar, 0, kWaitLimitNs);
     }
   } else {
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
@@ -680,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = m_blk * kBM + quad * 32;
       const bool got = epilogue_warp_tile<EPI, kChunks>(
           t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp, tmc, ws, resid,
-          [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); },
+          [&] { return mbar_wait<kSleepNs>(tfull_bar(acc), aph, kWaitLimitNs); },
           [&] { mbar_arrive(tempty_bar(acc)); });
       if (!got) { ok = false; break; }
     }
@@ -832,7 +837,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_kb; ++kb, ++issued) {
           const int s = issued % G::kStages;
           const uint32_t ph = (issued / G::kStages) & 1u;
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait<kSleepNs>(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
           const uint32_t leader_full = mapa_shared(full_bar(s), lead);
           mbar_arrive_expect_tx_cluster(leader_full, G::kStageBytes);
           tma_load_2d_pair(&tm_a, smem_u32(sA + s * G::kABytes), leader_full, kb * kBK, a_row);
@@ -843,7 +848,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
         // Every copy of both CTAs counted on the leader's full barriers has landed.
         const uint32_t first = issued > (uint32_t)G::kStages ? issued - G::kStages : 0u;
         for (uint32_t j = first; j < issued; ++j)
-          mbar_wait(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
+          mbar_wait<kSleepNs>(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
       }
     }
   } else if (warp == 1) {
@@ -853,13 +858,13 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
       for (int w = cluster; w < num_work && ok; w += num_clusters, ++local) {
         const uint32_t acc = local & 1u;
         const uint32_t aph = (local >> 1) & 1u;
-        if (!mbar_wait(tempty_bar(acc), aph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait<kSleepNs>(tempty_bar(acc), aph ^ 1u, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % G::kStages;
           const uint32_t ph = (it / G::kStages) & 1u;
-          if (!mbar_wait(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait<kSleepNs>(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + s * G::kABytes);
           const uint32_t b_addr = smem_u32(sB + s * G::kBBytes);
@@ -875,7 +880,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
       }
       mma_commit_pair(drain_bar, pair_mask);
     }
-    if (lane == 0) mbar_wait(drain_bar, 0, kWaitLimitNs);   // the leader's MMAs are done
+    if (lane == 0) mbar_wait<kSleepNs>(drain_bar, 0, kWaitLimitNs);   // the leader's MMAs are done
     __syncwarp();
   } else {
     const int quad = warp & 3;
@@ -906,7 +911,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t aph = (local >> 1) & 1u;
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + slice * kCols;
       const int row0 = m_blk * 256 + (int)rir * 128 + quad * 32;
-      auto wait_full = [&] { return mbar_wait(tfull_bar(acc), aph, kWaitLimitNs); };
+      auto wait_full = [&] { return mbar_wait<kSleepNs>(tfull_bar(acc), aph, kWaitLimitNs); };
       auto release = [&] { mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0); };
       bool got;
       if constexpr (kLn)
@@ -1112,14 +1117,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % G::kStages;
         const uint32_t ph = (it / G::kStages) & 1u;
-        if (!mbar_wait(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait<kSleepNs>(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
         mbar_arrive_expect_tx(full_bar(s), G::kStageBytes);
         tma_load_2d(&tm_a, sbase + s * G::kStageBytes, full_bar(s), kb * kBK, m_blk * kBM);
         tma_load_2d(&tm_b, sbase + s * G::kStageBytes + G::kABytes, full_bar(s), kb * kBK, n_blk * G::kBN);
       }
       const uint32_t first = it > (uint32_t)G::kStages ? it - G::kStages : 0u;
       for (uint32_t j = first; j < it; ++j)
-        mbar_wait(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
+        mbar_wait<kSleepNs>(full_bar(j % G::kStages), (j / G::kStages) & 1u, kWaitLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -1128,7 +1133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % G::kStages;
         const uint32_t ph = (it / G::kStages) & 1u;
-        if (!mbar_wait(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait<kSleepNs>(full_bar(s), ph, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = sbase + s * G::kStageBytes;
         const uint32_t b_addr = a_addr + G::kABytes;
@@ -1140,7 +1145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) mma_commit(tfull_bar);
       mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kWaitLimitNs);
+      mbar_wait<kSleepNs>(drain_bar, 0, kWaitLimitNs);
     }
   } else {
     // TMEM lanes of quadrant warp % 4; columns [64 * slice, 64 * slice + 64).
@@ -1148,7 +1153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int slice = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     int got = 0;
-    if (lane == 0) got = mbar_wait(tfull_bar, 0, kWaitLimitNs) ? 1 : 0;
+    if (lane == 0) got = mbar_wait<kSleepNs>(tfull_bar, 0, kWaitLimitNs) ? 1 : 0;
     got = __shfl_sync(0xffffffffu, got, 0);
     if (got) {
       tc_fence_after();

@@ -43,25 +43,42 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
       : "memory");
 }
 
+// mbarrier.try_wait may suspend the thread until the phase completes or a time
+// limit passes.  kSleepNs > 0 gives that limit as the suspend-time hint, so a
+// waiting thread sleeps until the phase completes instead of polling and leaves
+// its issue slots to the warps doing work; 0 keeps the hardware's own limit.
+template <uint32_t kSleepNs = 0>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if constexpr (kSleepNs > 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSleepNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// `limit_ns` nanoseconds of wall time and returns false.
+// `limit_ns` nanoseconds of wall time (checked every 256 tries, so at most
+// 256 suspend limits later) and returns false.
+template <uint32_t kSleepNs = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<kSleepNs>(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kSleepNs>(bar, parity)) return true;
     if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
@@ -257,16 +274,27 @@ __device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr
 
 // Bounded wait with acquire semantics at cluster scope (pairs with
 // mbar_arrive_remote_release).
+template <uint32_t kSleepNs = 0>
 __device__ __forceinline__ bool mbar_wait_acquire_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   auto try_once = [&]() {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+    if constexpr (kSleepNs > 0) {
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity), "r"(kSleepNs)
+          : "memory");
+    } else {
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    }
     return ok != 0;
   };
   if (try_once()) return true;
