@@ -1,0 +1,97 @@
+"""Host-side logic of bench.py that the JSON line depends on (CPU).
+
+- The algorithmic work per kernel (the numerators of the roofline fractions)
+  follows the formulas stated for each kernel: GEMM flops 2*M*N*K, attention
+  bytes 2*4*M*H (+ 4 bytes of valid length per sequence), LayerNorm bytes
+  2*2*M*H, residual reads added to the GEMMs that take one.
+- The DRAM traffic figure is taken from profiles/traffic.md only while the
+  kernel's sources are the ones it was measured on.
+- Named workloads have the shapes of the configurations they stand for.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import encoder_inputs as EI  # noqa: E402
+
+
+def test_kernel_work_formulas_bert_base_seq128():
+    wl = bench.parse_workload("bert-base:256:128")
+    M, H, F, S = 256 * 128, 768, 3072, 128
+    w = bench.kernel_work(wl)
+    assert w["qkv_gemm"][0] == 2 * M * H * 3 * H
+    assert w["qkv_gemm"][1] == 2 * (M * H + H * 3 * H + M * 3 * H)
+    assert w["out_proj_gemm"][0] == 2 * M * H * H
+    assert w["out_proj_gemm"][1] == 2 * (M * H + H * H + M * H) + 2 * M * H     # + residual
+    assert w["ffn1_gemm"][0] == 2 * M * H * F
+    assert w["ffn2_ln_gemm"][0] == 2 * M * F * H
+    assert w["ffn2_ln_gemm"][1] == 2 * (M * F + F * H + M * H) + 2 * M * H
+    assert w["attention"] == (4 * M * S * H, 2 * 4 * M * H + 4 * 256)
+    assert w["ln1"] == (0.0, 2 * 2 * M * H)
+    # Dense GEMM flops per token per layer 2H(3H + H + 2F): 14.16 MFLOP for BERT-Base.
+    per_token = sum(w[k][0] for k in ("qkv_gemm", "out_proj_gemm", "ffn1_gemm", "ffn2_gemm")) / M
+    assert per_token == 2 * H * (3 * H + H + 2 * F)
+    assert abs(per_token / 1e6 - 14.16) < 0.01
+
+
+def test_kernel_work_fp32_counts_four_byte_elements():
+    wl = bench.parse_workload("tiny-fp32:1")
+    M, H = 32, 128
+    assert bench.kernel_work(wl)["ln1"] == (0.0, 4 * 2 * M * H)
+
+
+def test_job_throughput_counts_every_rank():
+    assert bench.job_throughput(512, 1, 2.0) == pytest.approx(256000.0)
+    assert bench.job_throughput(512, 4, 2.0) == pytest.approx(4 * 256000.0)
+
+
+@pytest.mark.parametrize("spec,shape,layers,seq,batch", [
+    ("bert-base-s32:512", (12, 64, 3072), 12, 32, 512),
+    ("pruned-s32:1024", (4, 32, 512), 12, 32, 1024),
+    ("bert-base:256:128", (12, 64, 3072), 12, 128, 256),
+    ("bert-base:64:96", (12, 64, 3072), 12, 96, 64),
+    ("bert-large:32:512", (16, 64, 4096), 24, 512, 32),
+    ("tiny-fp32:1", (4, 32, 512), 1, 32, 1),
+])
+def test_named_workloads_have_the_config_shapes(spec, shape, layers, seq, batch):
+    wl = bench.parse_workload(spec)
+    sh = wl.shape
+    assert (sh.head_num, sh.size_per_head, sh.ffn_dim) == shape
+    assert sh.num_layers == layers and wl.seq == seq and wl.batch == batch
+    assert wl.dtype == ("fp32" if spec.startswith("tiny") else "fp16")
+
+
+def _write_table(path, kernel, workload, nbytes, digest):
+    with open(path, "w") as f:
+        f.write("| kernel | workload | bytes per launch | source digest | capture |\n|---|---|---:|---|---|\n")
+        f.write(f"| {kernel} | {workload} | {nbytes:,} | `{digest}` | x.md |\n")
+
+
+def test_traffic_is_reported_only_for_the_measured_sources(tmp_path, monkeypatch):
+    kernel, workload = "ffn2_ln_gemm", "bert-base-12L-h768-s32-b512-fp16"
+    digest = bench.source_digest(kernel)
+    assert len(digest) == 16
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # source_digest reads the sources under ROOT: keep reading the real ones.
+    monkeypatch.setattr(bench, "source_digest", lambda k: digest)
+    table = tmp_path / "profiles" / "traffic.md"
+    _write_table(table, kernel, workload, 142873856, digest)
+    assert bench.measured_traffic(kernel, workload) == 142873856.0
+    assert bench.measured_traffic(kernel, "another-workload") is None
+    assert bench.measured_traffic("qkv_gemm", workload) is None
+    _write_table(table, kernel, workload, 142873856, "0" * 16)         # sources changed since
+    assert bench.measured_traffic(kernel, workload) is None
+
+
+def test_source_digest_depends_on_every_listed_file():
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.exists(os.path.join(ROOT, "transformer_encoder_bert_b200", "csrc", f)), (kernel, f)
+    assert bench.source_digest("ln1") != bench.source_digest("qkv_gemm")
+    assert bench.source_digest("qkv_gemm") == bench.source_digest("ffn1_gemm")    # same sources
