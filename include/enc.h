@@ -86,7 +86,10 @@ typedef struct {
   const void* ln2_g; const void* ln2_b;   /* [H], [H] */
 } enc_layer_weights;
 
-/* enc_create - build a handle on the current CUDA device.
+/* enc_create - build a handle on the current CUDA device.  Every handle of a
+ * process lives on the device of the first one (kernel launch attributes are
+ * set once per process); on another device enc_create returns
+ * ENC_ERR_UNSUPPORTED.  Use one process per GPU.
  * [FT] "什么是 Faster Transformer": head_num and size_per_head are the two
  * structural parameters; ffn_dim and num_layers complete the stack.
  *   head_num, ffn_dim, num_layers > 0; size_per_head in {32, 64, 128}

@@ -15,6 +15,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <string>
@@ -25,6 +26,9 @@
 namespace {
 
 thread_local std::string g_last_error;
+// The device of the first handle: kernel launch attributes (dynamic shared
+// memory sizes, cluster occupancy) are set once per process, for that device.
+std::atomic<int> g_process_device{-1};
 
 enc_status fail(enc_status st, const char* fmt, ...) {
   char buf[512];
@@ -493,6 +497,13 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
     for (const void* p : ps)
       if (!p) return fail(ENC_ERR_INVALID_ARG, "layer %d has a null parameter pointer", l);
   }
+
+  int cur_dev = -1;
+  if (cudaGetDevice(&cur_dev) != cudaSuccess) return fail(ENC_ERR_CUDA, "no CUDA device");
+  int first = -1;
+  if (!g_process_device.compare_exchange_strong(first, cur_dev) && first != cur_dev)
+    return fail(ENC_ERR_UNSUPPORTED, "handles of one process share one CUDA device (%d); the current device is %d",
+                first, cur_dev);
 
   enc_handle* h = new enc_handle();
   h->nh = head_num; h->d = size_per_head; h->H = H; h->F = ffn_dim; h->L = num_layers;
