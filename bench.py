@@ -25,6 +25,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -149,7 +150,10 @@ class ClockSampler:
         vis = os.environ.get("CUDA_VISIBLE_DEVICES")
         self.index = vis.split(",")[local_rank] if vis else str(local_rank)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{local_rank}.csv")
+        # The raw samples go to BENCH_CLOCKS_DIR (default: the temp directory); the
+        # JSON line carries their summary.
+        out_dir = os.environ.get("BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"bench_clocks_rank{local_rank}_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -455,7 +459,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-sample", type=int, default=8, help="sequences per reference-arm step")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu DRAM bytes per launch of the dominant kernel, if captured for this build")
+                    help="ncu DRAM bytes per launch of the dominant kernel, if captured for the current sources")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
