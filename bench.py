@@ -14,8 +14,14 @@ host memory and its output back inside the timed region, consecutive steps
 overlapping their copies with the encoder.  The per-kernel breakdown and the
 roofline come from CUDA events the library records between its kernels on the
 launching stream: during the timed steps with --no-graph, else in as many traced
-enc_forward calls right after them (a recorded forward carries no events).  --impl reference times the float64 CPU oracle on a bounded sample.
-Default workload: 12-layer BERT-Base shape (12x64, FFN 3072), seq 32, batch 512.
+enc_forward calls right after them (a recorded forward carries no events).  The
+events break the overlap between kernels, so those times are upper bounds on the
+in-graph ones; the roofline divides by the measured burst tensor peak (kernels of
+microseconds inside millisecond steps).  --impl reference times the float64 CPU
+oracle on a bounded sample.
+Default workload: 12-layer BERT-Base shape (12x64, FFN 3072), seq 32, batch 512;
+the goal point (BERT-Base, seq 128, batch 256) is timed in the same run and
+reported under "secondary" (one GPU; --secondary '' skips it).
 """
 from __future__ import annotations
 
@@ -39,6 +45,8 @@ import encoder_inputs as EI  # noqa: E402
 METRIC = "BERT-Base FP16 encoder fwd sequences/s (seq 32/128); % tensor/HBM roofline"
 UNIT = "sequences/s"
 DEFAULT_WORKLOAD = "bert-base-s32:512"
+# The goal point: BERT-Base, seq 128, batch 256.
+SECONDARY_WORKLOAD = "bert-base:256:128"
 KERNEL_NAMES = ["qkv_gemm", "attention", "out_proj_gemm", "ln1", "ffn1_gemm", "ffn2_gemm", "ln2"]
 # when the output-projection and FFN2 GEMMs write the LayerNorm of their rows
 KERNEL_NAMES_FUSED = ["qkv_gemm", "attention", "out_proj_ln_gemm", "ffn1_gemm", "ffn2_ln_gemm"]
@@ -276,6 +284,118 @@ def workload_config(wl: EI.Workload, world: int, l2: str):
 
 
 # ------------------------------------------------------------------ our arm
+def kernel_names(nk: int, num_layers: int, packed: bool):
+    """Names of the nk kernels of one forward, in launch order."""
+    per_layer = (nk - (3 if packed else 0)) // num_layers
+    layer_names = {5: KERNEL_NAMES_FUSED, 6: KERNEL_NAMES_FFN2_LN}.get(per_layer, KERNEL_NAMES)
+    if packed:
+        return ["offsets", "pack"] + layer_names * num_layers + ["unpack"]
+    return layer_names * num_layers
+
+
+def time_forward(enc, x, vl, out, wl, args, flush, stream, barrier):
+    """Device time of args.steps forwards (graph replays by default) after
+    args.warmup untimed ones, the L2 flushed before each; then the per-kernel
+    breakdown from as many traced enc_forward calls (CUDA events recorded by the
+    library between its kernels on the launching stream).  The events break the
+    programmatic-dependent-launch overlap between kernels, so each traced kernel
+    time is an upper bound on its time inside the timed graph."""
+    import torch
+    graph = enc.record(x, vl, out) if args.graph else None
+    step = (lambda: graph.launch()) if graph is not None else (lambda: enc.forward(x, vl, out))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    nk = enc.kernels_per_forward(wl.batch, wl.seq)
+    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for evs in ev_sets:                                   # create the events before the timed region
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = enc.launch_count()
+    for i in range(args.steps):
+        flush.zero_()
+        if graph is None:
+            enc.set_trace_events(ev_sets[i], prepare=False)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = enc.launch_count() - launches0
+    if graph is not None:
+        for i in range(args.steps):
+            flush.zero_()
+            enc.set_trace_events(ev_sets[i], prepare=False)
+            enc.forward(x, vl, out)
+        torch.cuda.synchronize()
+        graph.close()
+    enc.set_trace_events(None)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    names = kernel_names(nk, wl.shape.num_layers, args.packed)
+    per_kernel = {k: [] for k in names}
+    traced = []
+    for evs in ev_sets:
+        for j in range(nk):
+            per_kernel[names[j]].append(evs[j].elapsed_time(evs[j + 1]))
+        traced.append(evs[0].elapsed_time(evs[nk]))
+    return {"ms": sum(step_ms) / len(step_ms), "per_kernel": per_kernel, "launches": launches,
+            "traced_ms": sum(traced) / len(traced), "nk": nk}
+
+
+def kernel_table(wl, inp, per_kernel, peaks, packed: bool):
+    """Per kernel: average traced time, share, TFLOP/s (GEMMs) and algorithmic GB/s,
+    each with its fraction of the measured peak (burst tensor peak: the kernels run
+    for microseconds inside steps of milliseconds)."""
+    sh = wl.shape
+    work = kernel_work(wl)
+    if packed:
+        # valid tokens only: the algorithmic work of the packed path
+        t_valid = int(np.clip(inp.valid_len, 0, wl.seq).sum())
+        work = kernel_work(wl.with_(batch=1, seq=t_valid), attn_seq=wl.seq, attn_tokens=t_valid)
+        work.update({"offsets": (0.0, 8.0 * wl.batch), "pack": (0.0, 4.0 * t_valid * sh.hidden),
+                     "unpack": (0.0, 4.0 * t_valid * sh.hidden)})
+    tc_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    kernels = {}
+    total = sum(sum(v) for v in per_kernel.values())
+    for k, vals in per_kernel.items():
+        avg_ms = sum(vals) / len(vals)
+        flops, nbytes = work[k]
+        entry = {"avg_us": avg_ms * 1e3, "share": sum(vals) / total}
+        if flops and k.endswith("gemm"):
+            entry["tflops"] = flops / (avg_ms * 1e-3) / 1e12
+            entry["tensor_frac"] = entry["tflops"] / tc_peak
+        entry["gbs"] = nbytes / (avg_ms * 1e-3) / 1e9
+        if not k.endswith("gemm"):
+            entry["hbm_frac"] = entry["gbs"] / hbm_peak
+        kernels[k] = entry
+    return kernels, work
+
+
+def roofline_of(kernels, work, dominant, peaks, peak_src, traffic):
+    d = kernels[dominant]
+    if dominant.endswith("gemm"):
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        return {"bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
+                "frac": d["tflops"] / peak, "traffic": traffic,
+                "kernel": dominant, "per_launch_flops": work[dominant][0],
+                "peak_source": f"{peak_src} burst bf16 matmul (FP16 dense rate = BF16 dense rate); "
+                               "the kernel runs for microseconds inside millisecond steps",
+                "time_source": "traced enc_forward calls (events between kernels): an upper bound on "
+                               "the kernel's time in the timed graph, so achieved is a lower bound"}
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {"bound": "hbm", "achieved": d["gbs"], "peak": peak, "unit": "GB/s", "frac": d["gbs"] / peak,
+            "traffic": traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
+            "peak_source": f"{peak_src} HBM copy bandwidth",
+            "time_source": "traced enc_forward calls (events between kernels): an upper bound on "
+                           "the kernel's time in the timed graph, so achieved is a lower bound"}
+
+
 def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -300,57 +420,11 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         if world > 1:
             dist.barrier()
 
-    graph = enc.record(x, vl, out) if args.graph else None
-    step = (lambda: graph.launch()) if graph is not None else (lambda: enc.forward(x, vl, out))
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
-    nk = enc.kernels_per_forward(wl.batch, wl.seq)
-    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for evs in ev_sets:                                   # create the events before the timed region
-        for e in evs:
-            e.record()
-    torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    launches0 = enc.launch_count()
-    for i in range(args.steps):
-        flush.zero_()
-        if graph is None:
-            enc.set_trace_events(ev_sets[i], prepare=False)
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    launches = enc.launch_count() - launches0
-    clk = clocks.stop()
-    if graph is not None:
-        # A recorded forward carries no per-kernel events: take the breakdown from
-        # the same number of traced (non-recorded) forwards after the timed region.
-        for i in range(args.steps):
-            flush.zero_()
-            enc.set_trace_events(ev_sets[i], prepare=False)
-            enc.forward(x, vl, out)
-        torch.cuda.synchronize()
-    enc.set_trace_events(None)
-
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(step_ms) / len(step_ms)
-    per_layer = (nk - (3 if args.packed else 0)) // sh.num_layers
-    layer_names = {5: KERNEL_NAMES_FUSED, 6: KERNEL_NAMES_FFN2_LN}.get(per_layer, KERNEL_NAMES)
-    names = (["offsets", "pack"] + layer_names * sh.num_layers + ["unpack"]) if args.packed \
-        else layer_names * sh.num_layers
-    per_kernel = {k: [] for k in names}
-    for evs in ev_sets:
-        for j in range(nk):
-            per_kernel[names[j]].append(evs[j].elapsed_time(evs[j + 1]))
+    main_t = time_forward(enc, x, vl, out, wl, args, flush, stream, barrier)
+    ms = main_t["ms"]
 
     # e2e through the pipelined host entry point (enc_forward_host_async): every
     # step copies its input from pinned host memory and its output back to host
@@ -374,46 +448,37 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     barrier()
     e2e_step = s.elapsed_time(e) / args.steps
     status = enc.device_status()
-    if graph is not None:
-        graph.close()
+    enc.close()
+
+    # The goal point (BERT-Base, seq 128, batch 256) in the same run, device-timed
+    # the same way, when it is not already the main workload (one GPU only).
+    secondary = None
+    sec_wl = parse_workload(args.secondary) if args.secondary else None
+    if world == 1 and sec_wl is not None and sec_wl.name != wl.name:
+        sec_inp = EI.make_inputs(sec_wl)
+        ssh = sec_wl.shape
+        enc2 = Encoder(ssh.head_num, ssh.size_per_head, ssh.ffn_dim, sec_inp.layers, sec_wl.dtype)
+        if args.packed:
+            enc2.set_packing(True)
+        enc2.reserve(sec_wl.batch, sec_wl.seq)
+        x2 = torch.from_numpy(sec_inp.x).to(dev)
+        vl2 = torch.from_numpy(sec_inp.valid_len).to(dev)
+        out2 = torch.empty_like(x2)
+        sec_t = time_forward(enc2, x2, vl2, out2, sec_wl, args, flush, stream, barrier)
+        sec_status = enc2.device_status()
+        enc2.close()
+        secondary = {"workload": sec_wl.name, "sec_t": sec_t, "inp": sec_inp, "wl": sec_wl, "status": sec_status}
+    clk = clocks.stop()
 
     ms, e2e_step = max_over_ranks([ms, e2e_step], device=dev)
     if rank != 0:
         return 0
 
     peaks, peak_src = load_peaks()
-    work = kernel_work(wl)
-    if args.packed:
-        # valid tokens only: the algorithmic work of the packed path
-        t_valid = int(np.clip(inp.valid_len, 0, wl.seq).sum())
-        work = kernel_work(wl.with_(batch=1, seq=t_valid), attn_seq=wl.seq, attn_tokens=t_valid)
-        work.update({"offsets": (0.0, 8.0 * wl.batch), "pack": (0.0, 4.0 * t_valid * sh.hidden),
-                     "unpack": (0.0, 4.0 * t_valid * sh.hidden)})
-    kernels = {}
-    total = sum(sum(v) for v in per_kernel.values())
-    for k in per_kernel:
-        vals = per_kernel[k]
-        avg_ms = sum(vals) / len(vals)
-        flops, nbytes = work[k]
-        entry = {"avg_us": avg_ms * 1e3, "share": sum(vals) / total}
-        if flops and k.endswith("gemm"):
-            entry["tflops"] = flops / (avg_ms * 1e-3) / 1e12
-        entry["gbs"] = nbytes / (avg_ms * 1e-3) / 1e9
-        kernels[k] = entry
+    kernels, work = kernel_table(wl, inp, main_t["per_kernel"], peaks, args.packed)
     dominant = max(kernels, key=lambda k: kernels[k]["share"])
-    d = kernels[dominant]
     traffic = args.traffic if args.traffic is not None else measured_traffic(dominant, wl.name)
-    if dominant.endswith("gemm"):
-        peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-        roof = {"bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
-                "frac": d["tflops"] / peak, "traffic": traffic,
-                "kernel": dominant, "per_launch_flops": work[dominant][0],
-                "peak_source": f"{peak_src} sustained bf16 matmul (FP16 dense rate = BF16 dense rate)"}
-    else:
-        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        roof = {"bound": "hbm", "achieved": d["gbs"], "peak": peak, "unit": "GB/s", "frac": d["gbs"] / peak,
-                "traffic": traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
-                "peak_source": f"{peak_src} HBM copy bandwidth"}
+    roof = roofline_of(kernels, work, dominant, peaks, peak_src, traffic)
 
     value = job_throughput(wl.batch, world, ms)
     line = {
@@ -428,11 +493,29 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         "e2e": {"value": job_throughput(wl.batch, world, e2e_step), "unit": UNIT,
                 "h2d_bytes_per_step": int(hx.numel() * hx.element_size() + hvl.numel() * 4),
                 "d2h_bytes_per_step": int(hout.numel() * hout.element_size())},
-        "gpu_launches": int(launches),
+        "gpu_launches": int(main_t["launches"]),
         "clocks": clk,
+        "traced_ms_per_forward": main_t["traced_ms"],
         "kernels": kernels,
         "device_status": status,
     }
+    if secondary is not None:
+        sw, st = secondary["wl"], secondary["sec_t"]
+        skern, swork = kernel_table(sw, secondary["inp"], st["per_kernel"], peaks, args.packed)
+        sdom = max(skern, key=lambda k: skern[k]["share"])
+        gemms = [k for k in skern if k.endswith("gemm")]
+        g_flops = sum(swork[k][0] * len(st["per_kernel"][k]) for k in gemms) / args.steps
+        g_ms = sum(sum(st["per_kernel"][k]) for k in gemms) / args.steps
+        tc_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        line["secondary"] = {
+            "workload": sw.name, "value": sw.batch / (st["ms"] * 1e-3), "unit": UNIT, "ms_per_step": st["ms"],
+            "traced_ms_per_forward": st["traced_ms"], "gpu_launches": int(st["launches"]),
+            "roofline": roofline_of(skern, swork, sdom, peaks, peak_src,
+                                    measured_traffic(sdom, sw.name)),
+            "gemms_aggregate": {"tflops": g_flops / (g_ms * 1e-3) / 1e12,
+                                "tensor_frac": g_flops / (g_ms * 1e-3) / 1e12 / tc_peak},
+            "kernels": skern, "device_status": secondary["status"],
+        }
     if world == 1 and not args.no_cpu_baseline:
         rate, n, dt = oracle_rate(inp, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -456,6 +539,8 @@ def main(argv=None):
                     help="time replays of a recorded forward (enc_graph_launch); the default")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time enc_forward calls instead of graph replays")
+    ap.add_argument("--secondary", default=SECONDARY_WORKLOAD,
+                    help="a second workload device-timed in the same run (one GPU; '' for none)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-sample", type=int, default=8, help="sequences per reference-arm step")
     ap.add_argument("--traffic", type=float, default=None,

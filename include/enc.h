@@ -109,6 +109,44 @@ ENC_API enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int 
  * (host-side setting; takes effect at the next launch). */
 ENC_API enc_status enc_set_gelu(enc_t h, enc_gelu form);
 
+/* Kernel-path switches.  Every choice computes the same result to rounding;
+ * the defaults are the measured-fastest paths, and the others exist so that
+ * each alternative kernel can be compared and checked on any shape. */
+typedef enum {
+  /* 1 (default): 2-CTA 256x256 GEMM tiles where they still give a quarter of
+   * the SMs a tile; 0: one-CTA 128-row tiles only. */
+  ENC_OPT_PAIR_TILES = 0,
+  /* 1 (default): GEMM epilogues store their output, and read the residual,
+   * through TMA; 0: plain 16-byte stores and loads (also turns off both
+   * LayerNorm fusions, which need TMA). */
+  ENC_OPT_TMA_STORE = 1,
+  /* 1 (default): tcgen05 attention for size-64 heads on sequences longer than
+   * 64; 0: the mma.sync attention kernels for every length. */
+  ENC_OPT_TC_ATTENTION = 2,
+  /* 1 (default): split-K thread-block clusters for GEMMs whose tiles would
+   * leave more than half the SMs idle; 0: never split K. */
+  ENC_OPT_SPLIT_K = 3,
+  /* 1 (default): the FFN2 GEMM writes LayerNorm 2 of its rows itself where the
+   * 2-CTA tiles run and the hidden size is 256, 512 or 768; 0: a separate
+   * LayerNorm kernel. */
+  ENC_OPT_LN_FUSE_FFN2 = 4,
+  /* 0 (default): a separate LayerNorm 1 kernel; 1: the output-projection GEMM
+   * writes LayerNorm 1 itself wherever the fused epilogue is supported. */
+  ENC_OPT_LN_FUSE_OUT_PROJ = 5,
+  /* 1 (default): kernels are launched with programmatic dependent launch, so
+   * each one's set-up overlaps its predecessor's tail; 0: plain stream order. */
+  ENC_OPT_PDL = 6
+} enc_option;
+
+/* enc_set_option - set one kernel-path switch of this handle (value 0 or 1;
+ * else ENC_ERR_INVALID_ARG).  Host-side; takes effect at the next launch.  A
+ * recorded forward (enc_graph_create) keeps the kernels it recorded.  Not part
+ * of the source pages' design: it exposes this library's own alternatives. */
+ENC_API enc_status enc_set_option(enc_t h, enc_option option, int value);
+
+/* enc_get_option - read one switch into *value. */
+ENC_API enc_status enc_get_option(enc_t h, enc_option option, int* value);
+
 /* enc_set_packing - padding removal for every later forward (FP16 mode, H <=
  * 1024; else ENC_ERR_UNSUPPORTED).  With it on, the valid tokens of the batch
  * are packed on the device into [T, H] (T = sum of the clamped valid lengths),

@@ -95,3 +95,26 @@ def test_source_digest_depends_on_every_listed_file():
             assert os.path.exists(os.path.join(ROOT, "transformer_encoder_bert_b200", "csrc", f)), (kernel, f)
     assert bench.source_digest("ln1") != bench.source_digest("qkv_gemm")
     assert bench.source_digest("qkv_gemm") == bench.source_digest("ffn1_gemm")    # same sources
+
+
+def test_kernel_names_follow_launch_order():
+    assert bench.kernel_names(7 * 2, 2, False) == bench.KERNEL_NAMES * 2
+    assert bench.kernel_names(6 * 12, 12, False) == bench.KERNEL_NAMES_FFN2_LN * 12
+    names = bench.kernel_names(6 * 12 + 3, 12, True)
+    assert names[:2] == ["offsets", "pack"] and names[-1] == "unpack" and len(names) == 75
+
+
+def test_roofline_divides_by_the_burst_tensor_peak():
+    """The GEMMs run for microseconds inside millisecond steps: the clock-burst
+    matmul peak is the denominator, and the fraction recomputes from the line."""
+    wl = bench.parse_workload("bert-base-s32:512")
+    peaks = {"hbm_gbs": 6558.4, "bf16_tflops": 1653.4, "bf16_tflops_sustained": 1397.7}
+    per_kernel = {k: [0.1, 0.1] for k in bench.KERNEL_NAMES_FFN2_LN}
+    per_kernel["ffn2_ln_gemm"] = [0.0736, 0.0736]
+    kernels, work = bench.kernel_table(wl, None, per_kernel, peaks, packed=False)
+    roof = bench.roofline_of(kernels, work, "ffn2_ln_gemm", peaks, "measured", None)
+    assert roof["peak"] == 1653.4
+    assert roof["achieved"] == pytest.approx(2 * 16384 * 3072 * 768 / 73.6e-6 / 1e12)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / 1653.4)
+    ln = bench.roofline_of(kernels, work, "ln1", peaks, "measured", None)
+    assert ln["bound"] == "hbm" and ln["frac"] == pytest.approx(2 * 2 * 16384 * 768 / 0.1e-3 / 1e9 / 6558.4)

@@ -170,6 +170,31 @@ def test_deterministic_and_host_entry_point_matches():
     assert enc.device_status() == 0
 
 
+def test_plain_stream_order_is_bit_identical():
+    """The pdl option off launches every kernel in plain stream order; the kernels
+    are the same, so the output is the same bit for bit, and switching it back
+    on restores the default."""
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 16))
+    enc, got = _run(inp)
+    assert enc.get_option("pdl")
+    enc.set_option("pdl", False)
+    assert not enc.get_option("pdl")
+    plain = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    assert np.array_equal(got, plain)
+    enc.set_option("pdl", True)
+    assert np.array_equal(got, to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len))))
+    assert enc.device_status() == 0
+
+
+def test_option_argument_checks():
+    inp = EI.make_inputs(EI.Workload("args", EI.EncoderShape(4, 32, 512, 1), 2, 8, "fp16", 1, 8))
+    enc = encoder_from_inputs(inp)
+    assert enc.lib.enc_set_option(enc.handle, 2, 2) == 1       # value not 0 or 1: ENC_ERR_INVALID_ARG
+    assert enc.lib.enc_set_option(enc.handle, 99, 1) == 1      # unknown option
+    assert enc.lib.enc_set_option(None, 2, 1) == 1             # null handle
+    assert enc.get_option("tc_attention") and not enc.get_option("ln_fuse_out_proj")
+
+
 def test_host_argument_checks():
     import torch
     from transformer_encoder_bert_b200 import EncError
@@ -273,6 +298,30 @@ def test_pipelined_host_entry_point_matches_device_forward():
     assert enc.device_status() == 0
 
 
+def test_pipelined_host_entry_point_alternating_shapes():
+    """enc_forward_host_async with calls of different sizes in flight together
+    (64, 16, 64, 16, 48 sequences): the smaller call's staging slot must lie
+    outside the larger call's, whose encoder run and copies may still be in
+    flight.  Every output equals the device forward bit for bit."""
+    import torch
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    wl = EI.named_workload("bert-base-s32", 64).with_(shape=sh)
+    sizes = [64, 16, 64, 16, 48]
+    batches = [EI.make_inputs(wl.with_(batch=b, seed=200 + i)) for i, b in enumerate(sizes)]
+    enc = encoder_from_inputs(batches[0])
+    refs = [to_host(enc.forward(to_dev(b.x), to_dev(b.valid_len))) for b in batches]
+    hx = [torch.from_numpy(b.x).pin_memory() for b in batches]
+    hvl = [torch.from_numpy(b.valid_len).pin_memory() for b in batches]
+    hout = [torch.zeros_like(t).pin_memory() for t in hx]
+    for i, b in enumerate(sizes):
+        enc.forward_host_async_ptr(hx[i].data_ptr(), hvl[i].data_ptr(), hout[i].data_ptr(), b, 32)
+    enc.host_join()
+    torch.cuda.current_stream().synchronize()
+    for i in range(len(sizes)):
+        assert np.array_equal(hout[i].numpy(), refs[i]), i
+    assert enc.device_status() == 0
+
+
 # ---------------------------------------------------------------- padding removal
 
 @pytest.mark.parametrize("seq,lo,hi,L", [(32, 1, 32, 12), (37, 0, 37, 2), (96, 64, 96, 2), (128, 64, 128, 2),
@@ -292,6 +341,38 @@ def test_packed_forward_matches_oracle_and_zeroes_padding(seq, lo, hi, L):
     tol = FP16_STACK_REL_L2 if L > 2 else L * FP16_LAYER_REL_L2
     _check(got, _oracle(inp), inp.valid_len, seq, tol)
     assert rel_l2(got, dense, m) < tol
+    assert enc.device_status() == 0
+
+
+PACKED_FULL_SIZE = [
+    ("bert-base-s32", 512, None, 4),
+    ("bert-base", 256, 128, 3),
+    ("bert-large", 256, 128, 3),
+]
+
+
+@pytest.mark.parametrize("kind,batch,seq,nsample", PACKED_FULL_SIZE, ids=lambda v: str(v))
+def test_packed_full_size_against_oracle(kind, batch, seq, nsample):
+    """Padding removal at the sizes the bench runs it: every GEMM takes the 2-CTA
+    tiles chosen from the padded token count and reads the real count T from the
+    device, and for hidden sizes up to 768 the FFN2 GEMM writes LayerNorm 2 itself
+    (6 launches per layer; 7 for BERT-Large), plus the offsets, pack and unpack
+    kernels.  A seeded sample of sequences (the first, the last and a shortest one
+    among them) against the oracle; every padded row is zero."""
+    wl = EI.named_workload(kind, batch, seq)
+    inp = EI.make_inputs(wl)
+    enc = encoder_from_inputs(inp)
+    enc.set_packing(True)
+    L = wl.shape.num_layers
+    per_layer = 6 if wl.shape.hidden <= 768 else 7
+    assert enc.kernels_per_forward(wl.batch, wl.seq) == per_layer * L + 3
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    m = valid_mask(inp.valid_len, wl.seq)
+    assert np.all(got[~m] == 0)
+    assert np.all(np.isfinite(got[m]))
+    seqs = EI.sample_sequences(wl.batch, nsample, inp.valid_len)
+    ref = _oracle(inp, seqs)
+    _check(got[seqs], ref, inp.valid_len[seqs], wl.seq, FP16_STACK_REL_L2)
     assert enc.device_status() == 0
 
 

@@ -104,17 +104,18 @@ def test_out_proj_ffn1_ffn2(shape, batch, seq):
 
 @pytest.mark.parametrize("shape,M", [((4, 64, 1024), 9300), ((12, 64, 3072), 4000), ((16, 64, 4096), 2600),
                                      ((12, 64, 3072), 16384)], ids=lambda v: str(v))
-def test_fused_layernorm_gemms(monkeypatch, shape, M):
+def test_fused_layernorm_gemms(shape, M):
     """Enough tokens for the 2-CTA tiles: the GEMMs write the LayerNorm of their rows
     (row statistics exchanged across the cluster that covers the row; clusters of
     2, 6 and 8 CTAs for H = 256, 768, 1024).  FFN2 is fused by default for H <= 768,
-    the output projection through ENC_LN_FUSE_OPROJ=1.  Against the oracle step,
-    and against the unfused path (GEMM writing bias + residual, then the LayerNorm
-    kernel; ENC_LN_NO_FUSE=1)."""
-    monkeypatch.setenv("ENC_LN_FUSE_OPROJ", "1")
+    the output projection through the ln_fuse_out_proj option.  Against the oracle
+    step, and against the unfused path (GEMM writing bias + residual, then the
+    LayerNorm kernel; both fusion options off)."""
     nh, d, F = shape
     H = nh * d
     wl, inp, enc, x64, vl, lw = _setup(shape, 1, M)
+    enc.set_option("ln_fuse_out_proj", True)
+    enc.set_option("ln_fuse_ffn2", True)
     ctx = EI.random_array((M, H), "fp16", seed=41)
     resid = EI.random_array((M, H), "fp16", seed=42, mean=0.2)
     uu = EI.random_array((M, F), "fp16", seed=43, std=0.5)
@@ -134,9 +135,9 @@ def test_fused_layernorm_gemms(monkeypatch, shape, M):
     for g, r in ((got_a, ref_a), (got_y, ref_y)):
         assert rel_l2(g, r) < GEMM_REL_L2 and max_abs(g, r) < LN_MAX_ABS
     assert enc.device_status() == 0
-    monkeypatch.setenv("ENC_LN_NO_FUSE", "1")
-    monkeypatch.delenv("ENC_LN_FUSE_OPROJ")
     wl, inp, enc1, x64, vl, lw = _setup(shape, 1, M)
+    enc1.set_option("ln_fuse_out_proj", False)
+    enc1.set_option("ln_fuse_ffn2", False)
     un_a, un_y = run(enc1)
     assert rel_l2(got_a, un_a) < GEMM_REL_L2 and rel_l2(got_y, un_y) < GEMM_REL_L2
 
@@ -227,17 +228,18 @@ def test_gelu_epilogue_against_exact_erf(hidden, batch, seq, form):
     assert np.all(np.abs(got - ref) <= 0.5 * ulp + 1e-6)
 
 
-@pytest.mark.parametrize("env", ["ENC_GEMM_NO_PAIR", "ENC_GEMM_NO_TMA_STORE"])
+@pytest.mark.parametrize("option", ["pair_tiles", "tma_store"])
 @pytest.mark.parametrize("batch,seq", [(2, 128), (5, 131)], ids=str)
-def test_alternative_gemm_paths(monkeypatch, env, batch, seq):
+def test_alternative_gemm_paths(option, batch, seq):
     """The one-CTA tile path (used for small M) and the direct-store epilogue (used when
     the output map cannot be built) on shapes that normally take the pair / TMA-store path."""
-    monkeypatch.setenv(env, "1")
     shape = (12, 64, 3072)
     nh, d, F = shape
     H = nh * d
     M = batch * seq
     wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    assert enc.get_option(option)
+    enc.set_option(option, False)
     h1 = EI.random_array((M, H), "fp16", seed=12)
     u = empty_dev((M, F), "fp16")
     enc.op_ffn1(0, to_dev(h1), u, M)
@@ -260,14 +262,14 @@ def test_alternative_gemm_paths(monkeypatch, env, batch, seq):
 
 
 @pytest.mark.parametrize("batch,seq", [(3, 128), (4, 96), (3, 65), (2, 200)], ids=str)
-def test_attention_mma_sync_path_for_long_sequences(monkeypatch, batch, seq):
+def test_attention_mma_sync_path_for_long_sequences(batch, seq):
     """Size-64 heads on sequences longer than 64 run on the tensor-core (tcgen05)
-    kernels; the mma.sync kernel for the same shapes stays checked through
-    ENC_ATTN_NO_TC."""
-    monkeypatch.setenv("ENC_ATTN_NO_TC", "1")
+    kernels; the mma.sync kernel for the same shapes stays checked through the
+    tc_attention option."""
     shape = (12, 64, 3072)
     nh, d, _ = shape
     wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    enc.set_option("tc_attention", False)
     qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=17)
     vlen = np.array([seq] + [max(1, seq // (i + 2)) for i in range(batch - 1)], np.int32)
     ctx = empty_dev((batch * seq, nh * d), "fp16")
@@ -308,13 +310,13 @@ def test_attention_long_sequences_tensor_core(batch, seq, lens, key_boost):
 
 
 @pytest.mark.parametrize("batch,seq", [(1, 32), (8, 32), (1, 7), (3, 37)], ids=str)
-def test_split_k_gemms(monkeypatch, batch, seq):
+def test_split_k_gemms(batch, seq):
     """At small M the GEMMs run split-K: a cluster of CTAs shares each 128x128 tile,
     each CTA one range of the k-blocks, and the partial tiles are summed in rank
     order through distributed shared memory.  Every epilogue (head split, plain,
     erf-GELU, tanh-GELU, bias + residual + LayerNorm) against its oracle step; a repeated call is bit-identical
     (the sum's order does not depend on timing); the unsplit kernel
-    (ENC_GEMM_NO_SPLITK=1) agrees within the GEMM bound."""
+    (split_k option off) agrees within the GEMM bound."""
     shape = (12, 64, 3072)
     nh, d, F = shape
     H = nh * d
@@ -355,7 +357,7 @@ def test_split_k_gemms(monkeypatch, batch, seq):
     for g, a in zip(got, again):
         assert np.array_equal(g, a)
     assert enc.device_status() == 0
-    monkeypatch.setenv("ENC_GEMM_NO_SPLITK", "1")
     wl, inp, enc1, x64, vl, lw = _setup(shape, batch, seq)
+    enc1.set_option("split_k", False)
     for g, r in zip(got, run(enc1)):
         assert rel_l2(g, r) < GEMM_REL_L2

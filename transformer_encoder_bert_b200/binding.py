@@ -20,6 +20,10 @@ STATUS_NAMES = {0: "ENC_OK", 1: "ENC_ERR_INVALID_ARG", 2: "ENC_ERR_UNSUPPORTED",
 DTYPE_CODES = {"fp32": 0, "fp16": 1}
 NP_DTYPES = {"fp32": np.float32, "fp16": np.float16}
 
+# enc_option codes (kernel-path switches; every choice computes the same result to rounding).
+OPTION_CODES = {"pair_tiles": 0, "tma_store": 1, "tc_attention": 2, "split_k": 3, "ln_fuse_ffn2": 4,
+                "ln_fuse_out_proj": 5, "pdl": 6}
+
 # Field order of enc_layer_weights.
 WEIGHT_FIELDS = ("w_qkv", "b_qkv", "w_o", "b_o", "ln1_g", "ln1_b",
                  "w_ff1", "b_ff1", "w_ff2", "b_ff2", "ln2_g", "ln2_b")
@@ -40,6 +44,8 @@ SIGNATURES = {
     "enc_set_gelu": (_i, [_vp, _i]),
     "enc_set_packing": (_i, [_vp, _i]),
     "enc_set_host_chunks": (_i, [_vp, _i]),
+    "enc_set_option": (_i, [_vp, _i, _i]),
+    "enc_get_option": (_i, [_vp, _i, ctypes.POINTER(_i)]),
     "enc_graph_create": (_i, [_vp, _vp, _vp, _vp, _i, _i, ctypes.POINTER(_vp)]),
     "enc_graph_launch": (_i, [_vp, _vp]),
     "enc_graph_destroy": (_i, [_vp]),
@@ -163,6 +169,15 @@ class Encoder:
     def set_packing(self, enable: bool):
         """Padding removal: compute valid tokens only; padded output rows become zeros."""
         _check(self.lib.enc_set_packing(self.handle, 1 if enable else 0))
+
+    def set_option(self, name: str, value: bool):
+        """One kernel-path switch (see OPTION_CODES and enc_option in include/enc.h)."""
+        _check(self.lib.enc_set_option(self.handle, OPTION_CODES[name], 1 if value else 0))
+
+    def get_option(self, name: str) -> bool:
+        v = ctypes.c_int(0)
+        _check(self.lib.enc_get_option(self.handle, OPTION_CODES[name], ctypes.byref(v)))
+        return bool(v.value)
 
     def set_host_chunks(self, chunks: int):
         _check(self.lib.enc_set_host_chunks(self.handle, chunks))

@@ -116,12 +116,14 @@ struct enc_handle {
   enc_gelu gelu = ENC_GELU_ERF;
   bool packed = false;              // padding removal (enc_set_packing)
   int host_chunks = 1;              // enc_forward_host: most chunks the batch is cut into (see enc.h)
-  bool no_pair = false;             // ENC_GEMM_NO_PAIR=1: one-CTA tiles only (comparison runs)
-  bool no_tma_store = false;        // ENC_GEMM_NO_TMA_STORE=1: epilogue stores without TMA
-  bool no_tc_attn = false;          // ENC_ATTN_NO_TC=1: mma.sync attention for every length
-  bool no_splitk = false;           // ENC_GEMM_NO_SPLITK=1: no split-K for small GEMMs (comparison runs)
-  bool no_ln_fuse = false;          // ENC_LN_NO_FUSE=1: LayerNorm as its own kernel (comparison runs)
-  bool ln_fuse_oproj = false;       // ENC_LN_FUSE_OPROJ=1: fuse LayerNorm 1 into the out-proj GEMM too
+  // Kernel-path switches (enc_set_option); the defaults are the fastest measured paths.
+  bool pair_tiles = true;           // ENC_OPT_PAIR_TILES: 2-CTA 256x256 GEMM tiles where they fill the GPU
+  bool tma_store = true;            // ENC_OPT_TMA_STORE: GEMM epilogues store (and read the residual) by TMA
+  bool tc_attn = true;              // ENC_OPT_TC_ATTENTION: tcgen05 attention for d = 64, seq > 64
+  bool splitk = true;               // ENC_OPT_SPLIT_K: split-K clusters for GEMMs that would idle most SMs
+  bool ln_fuse_ffn2 = true;         // ENC_OPT_LN_FUSE_FFN2: FFN2 writes LayerNorm 2 where supported
+  bool ln_fuse_oproj = false;       // ENC_OPT_LN_FUSE_OUT_PROJ: the output projection writes LayerNorm 1
+  bool pdl = true;                  // ENC_OPT_PDL: programmatic dependent launch between kernels
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -191,7 +193,7 @@ enc_status check_handle(const enc_handle* h) {
 // of the SMs a cluster each; else 128x256 one-CTA tiles when they fill the
 // GPU; else 128x128.
 int choose_bn(const enc_handle* h, int M, int N) {
-  if (N % 256 == 0 && M >= 256 && !h->no_pair) {
+  if (N % 256 == 0 && M >= 256 && h->pair_tiles) {
     const long pair_tiles = (long)((M + 255) / 256) * (N / 256);
     if (4 * pair_tiles >= h->num_sms) return enc::kPairTile;
   }
@@ -204,7 +206,7 @@ int choose_bn(const enc_handle* h, int M, int N) {
 // idle (small batches): the k-blocks of a tile are shared by a cluster of CTAs,
 // so that the weights are streamed by most SMs instead of a few.
 int choose_splits(const enc_handle* h, int M, int N, int K, int bn) {
-  if (bn != 128 || h->no_splitk) return 1;
+  if (bn != 128 || !h->splitk) return 1;
   const long tiles = (long)((M + 127) / 128) * ((N + 127) / 128);
   if (2 * tiles > h->num_sms) return 1;
   return enc::choose_gemm_splits((int)tiles, (K + 63) / 64, h->num_sms);
@@ -223,7 +225,7 @@ enc_status run_gemm(enc_handle* h, const void* A, int M, int K, void* W, const C
     // Output through TMA stores (32x32 boxes); the head split needs whole
     // 32-token chunks per sequence, otherwise its epilogue stores directly.
     CUtensorMap tc;
-    bool use_tc = !h->no_tma_store;
+    bool use_tc = h->tma_store;
     if (use_tc) {
       if (epi == enc::Epi::kBiasQkvSplit)
         use_tc = (sp.seq % 32 == 0) && enc::encode_output_map_split(&tc, C, sp);
@@ -276,7 +278,7 @@ enc_status step_qkv(enc_handle* h, int l, const void* x, void* qkv, int batch, i
 // 128, key blocks with a running maximum beyond); mma.sync otherwise (and for
 // every length under ENC_ATTN_NO_TC=1).
 bool use_tc_attention(const enc_handle* h, int seq) {
-  return enc::attention_tc_supported(h->d, seq) && !h->no_tc_attn;
+  return enc::attention_tc_supported(h->d, seq) && h->tc_attn;
 }
 
 enc_status step_attention(enc_handle* h, const void* qkv, const int32_t* vl, void* ctx, int batch, int seq,
@@ -314,10 +316,10 @@ enc_status step_out_proj(enc_handle* h, int l, const void* ctx, const void* resi
 // (H <= 768), and not behind the output projection's K = H main loop, nor with
 // 8-CTA clusters (H = 1024): those keep the separate LayerNorm kernel.
 bool ln_fused(const enc_handle* h, int tokens, int which) {
-  if (h->dtype != ENC_FP16 || h->no_ln_fuse || h->no_tma_store || !enc::gemm_ln_supported(tokens, h->H) ||
+  if (h->dtype != ENC_FP16 || !h->tma_store || !enc::gemm_ln_supported(tokens, h->H) ||
       choose_bn(h, tokens, h->H) != enc::kPairTile)
     return false;
-  return which == 2 ? h->H <= 768 : h->ln_fuse_oproj;
+  return which == 2 ? (h->ln_fuse_ffn2 && h->H <= 768) : h->ln_fuse_oproj;
 }
 
 int kernels_per_layer(const enc_handle* h, int tokens) {
@@ -457,13 +459,20 @@ enc_status host_setup(enc_handle* h, int batch, int seq) {
 
 }  // namespace
 
-bool enc::pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("ENC_NO_PDL");
-    return !(e && e[0] == '1');
-  }();
-  return on;
-}
+namespace {
+// Whether the launches of the entry point running on this thread use
+// programmatic dependent launch: the handle's ENC_OPT_PDL, set for the
+// duration of each entry point by a PdlScope.
+thread_local bool t_pdl = true;
+
+struct PdlScope {
+  bool prev;
+  explicit PdlScope(const enc_handle* h) : prev(t_pdl) { t_pdl = h ? h->pdl : true; }
+  ~PdlScope() { t_pdl = prev; }
+};
+}  // namespace
+
+bool enc::pdl_enabled() { return t_pdl; }
 
 int enc::device_sm_count() {
   int dev = 0, n = 0;
@@ -511,12 +520,6 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
   h->esize = dtype == ENC_FP16 ? 2 : 4;
   cudaGetDevice(&h->device);
   h->num_sms = enc::device_sm_count();
-  if (const char* e = getenv("ENC_GEMM_NO_PAIR")) h->no_pair = e[0] == '1';
-  if (const char* e = getenv("ENC_GEMM_NO_TMA_STORE")) h->no_tma_store = e[0] == '1';
-  if (const char* e = getenv("ENC_ATTN_NO_TC")) h->no_tc_attn = e[0] == '1';
-  if (const char* e = getenv("ENC_GEMM_NO_SPLITK")) h->no_splitk = e[0] == '1';
-  if (const char* e = getenv("ENC_LN_NO_FUSE")) h->no_ln_fuse = e[0] == '1';
-  if (const char* e = getenv("ENC_LN_FUSE_OPROJ")) h->ln_fuse_oproj = e[0] == '1';
   if (h->num_sms <= 0) { free_handle(h); return fail(ENC_ERR_CUDA, "no CUDA device"); }
   if (dtype == ENC_FP16) {
     cudaDeviceProp prop;
@@ -784,6 +787,7 @@ extern "C" {
 
 enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
                        enc_stream_t stream) {
+  PdlScope pdl(h);
   enc_status s = forward_impl(h, x, valid_len, out, batch, seq, reinterpret_cast<cudaStream_t>(stream), true);
   return s == ENC_OK ? ok() : s;
 }
@@ -796,6 +800,7 @@ enc_status enc_graph_create(enc_t h, const void* x, const int32_t* valid_len, vo
   if (s != ENC_OK) return s;
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if ((s = ensure_workspace(h, (size_t)batch * seq)) != ENC_OK) return s;   // no allocation while recording
+  PdlScope pdl(h);
   cudaStream_t st = nullptr;
   cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
@@ -854,6 +859,7 @@ enc_status enc_forward_host(enc_t h, const void* x, const int32_t* valid_len, vo
                             enc_stream_t stream) {
   enc_status s = check_handle(h);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if (!x || !valid_len || !out) return fail(ENC_ERR_INVALID_ARG, "null host buffer");
   const size_t seq_bytes = (size_t)seq * h->H * h->esize;
@@ -944,13 +950,21 @@ enc_status enc_forward_host_async(enc_t h, const void* x, const int32_t* valid_l
                                   enc_stream_t stream) {
   enc_status s = check_handle(h);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if (!x || !valid_len || !out) return fail(ENC_ERR_INVALID_ARG, "null host buffer");
   if ((s = host_setup(h, batch, seq)) != ENC_OK) return s;
   const int k = h->host_slot;
   const size_t act = (size_t)batch * seq * h->H * h->esize;
   const size_t act_al = align_up(act, 256);
-  char* base = static_cast<char*>(h->stage) + (size_t)k * host_slot_bytes(h, batch, seq);
+  // The two slots split the staging allocation in halves, whatever the shape of
+  // the call that allocated it: a call smaller than the previous one must not
+  // place its slot inside the other slot, whose run may still be in flight.
+  const size_t slot_stride = h->stage_bytes / 2;
+  if (host_slot_bytes(h, batch, seq) > slot_stride)
+    return fail(ENC_ERR_CUDA, "staging slot of %zu bytes is smaller than the %zu this call needs", slot_stride,
+                host_slot_bytes(h, batch, seq));
+  char* base = static_cast<char*>(h->stage) + (size_t)k * slot_stride;
   char* dx = base;
   char* dout = base + act_al;
   int32_t* dvl = reinterpret_cast<int32_t*>(base + 2 * act_al);
@@ -1016,6 +1030,41 @@ enc_status enc_set_packing(enc_t h, int enable) {
   return ok();
 }
 
+enc_status enc_set_option(enc_t h, enc_option option, int value) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  if (value != 0 && value != 1) return fail(ENC_ERR_INVALID_ARG, "option value %d is not 0 or 1", value);
+  const bool v = value != 0;
+  switch (option) {
+    case ENC_OPT_PAIR_TILES: h->pair_tiles = v; break;
+    case ENC_OPT_TMA_STORE: h->tma_store = v; break;
+    case ENC_OPT_TC_ATTENTION: h->tc_attn = v; break;
+    case ENC_OPT_SPLIT_K: h->splitk = v; break;
+    case ENC_OPT_LN_FUSE_FFN2: h->ln_fuse_ffn2 = v; break;
+    case ENC_OPT_LN_FUSE_OUT_PROJ: h->ln_fuse_oproj = v; break;
+    case ENC_OPT_PDL: h->pdl = v; break;
+    default: return fail(ENC_ERR_INVALID_ARG, "unknown option %d", (int)option);
+  }
+  return ok();
+}
+
+enc_status enc_get_option(enc_t h, enc_option option, int* value) {
+  if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
+  if (!value) return fail(ENC_ERR_INVALID_ARG, "value is null");
+  bool v;
+  switch (option) {
+    case ENC_OPT_PAIR_TILES: v = h->pair_tiles; break;
+    case ENC_OPT_TMA_STORE: v = h->tma_store; break;
+    case ENC_OPT_TC_ATTENTION: v = h->tc_attn; break;
+    case ENC_OPT_SPLIT_K: v = h->splitk; break;
+    case ENC_OPT_LN_FUSE_FFN2: v = h->ln_fuse_ffn2; break;
+    case ENC_OPT_LN_FUSE_OUT_PROJ: v = h->ln_fuse_oproj; break;
+    case ENC_OPT_PDL: v = h->pdl; break;
+    default: return fail(ENC_ERR_INVALID_ARG, "unknown option %d", (int)option);
+  }
+  *value = v ? 1 : 0;
+  return ok();
+}
+
 enc_status enc_set_host_chunks(enc_t h, int chunks) {
   if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
   if (chunks < 1 || chunks > enc_handle::kMaxChunks)
@@ -1058,6 +1107,7 @@ static enc_status op_prologue(enc_t h, int layer, bool needs_layer, int tokens) 
 enc_status enc_op_qkv(enc_t h, int layer, const void* x, void* qkv, int batch, int seq, enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, batch > 0 && seq > 0 ? batch * seq : 0);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if ((s = check_ptrs({x, qkv})) != ENC_OK) return s;
   if ((s = step_qkv(h, layer, x, qkv, batch, seq, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
@@ -1068,6 +1118,7 @@ enc_status enc_op_attention(enc_t h, const void* qkv, const int32_t* valid_len, 
                             enc_stream_t stream) {
   enc_status s = op_prologue(h, 0, false, batch > 0 && seq > 0 ? batch * seq : 0);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if ((s = check_ptrs({qkv, ctx})) != ENC_OK) return s;
   if (!valid_len) return fail(ENC_ERR_INVALID_ARG, "valid_len is null");
@@ -1080,6 +1131,7 @@ enc_status enc_op_out_proj_ln(enc_t h, int layer, const void* ctx, const void* r
                               enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_ptrs({ctx, resid, out})) != ENC_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (ln_fused(h, tokens, 1)) {
@@ -1096,6 +1148,7 @@ enc_status enc_op_out_proj_ln(enc_t h, int layer, const void* ctx, const void* r
 enc_status enc_op_ffn1(enc_t h, int layer, const void* h1, void* u, int tokens, enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_ptrs({h1, u})) != ENC_OK) return s;
   if ((s = step_ffn1(h, layer, h1, u, tokens, reinterpret_cast<cudaStream_t>(stream))) != ENC_OK) return s;
   return ok();
@@ -1105,6 +1158,7 @@ enc_status enc_op_ffn2_ln(enc_t h, int layer, const void* u, const void* resid, 
                           enc_stream_t stream) {
   enc_status s = op_prologue(h, layer, true, tokens);
   if (s != ENC_OK) return s;
+  PdlScope pdl(h);
   if ((s = check_ptrs({u, resid, out})) != ENC_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (ln_fused(h, tokens, 2)) {

@@ -964,7 +964,6 @@ int pair_max_clusters(cudaError_t& err) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, gemm_tc_pair_kernel<EPI, CL>, &cfg);
-    if (getenv("ENC_DEBUG")) fprintf(stderr, "[enc] pair GEMM (%d-CTA clusters): %d co-resident\n", CL, max_clusters);
   });
   err = attr_err;
   return max_clusters;

@@ -42,7 +42,8 @@ constexpr int kStatusWaitTimeout = 1;
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// False when ENC_NO_PDL=1 (plain stream order, for comparison runs).
+// The handle's ENC_OPT_PDL for the entry point running on this thread (plain
+// stream order when off, for comparison runs).
 bool pdl_enabled();
 
 // <<<grid, block, smem, stream>>> with programmatic stream serialization
