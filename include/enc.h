@@ -178,6 +178,35 @@ ENC_API enc_status enc_set_host_chunks(enc_t h, int chunks);
 ENC_API enc_status enc_forward(enc_t h, const void* x, const int32_t* valid_len, void* out,
                        int batch, int seq, enc_stream_t stream);
 
+/* Size of the fixed device array that enc_forward_noalloc uses as its scratch:
+ * 32 MiB.  Every GPU that loads this library holds it until the process exits. */
+#define ENC_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+/* enc_forward_noalloc - enc_forward without any device allocation.  The source
+ * pages have no counterpart: this serves callers that cannot call cudaMalloc
+ * when they run the encoder, such as a server whose device memory is all handed
+ * out by its own pool allocator (so a library allocation fails or takes memory
+ * the pool counts on), or a latency-bound loop that cannot afford cudaMalloc /
+ * cudaFree, which may synchronise the whole device.  The handle still comes
+ * from enc_create, which does allocate, at set-up time.
+ *   Same arguments, layout, results and kernels as enc_forward.  The
+ *   intermediates live in one fixed device array of ENC_STATIC_WORKSPACE_BYTES
+ *   compiled into the library instead of the handle's workspace, so the call
+ *   accepts a batch only when enc_workspace_bytes(h, batch, seq) <=
+ *   ENC_STATIC_WORKSPACE_BYTES (BERT-Base needs 18,432 bytes per token, so at
+ *   most 1,820 tokens, e.g. batch 14 at seq 128); larger ones return
+ *   ENC_ERR_UNSUPPORTED before anything is enqueued.
+ *   The first call on a device looks up the array's device address there
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Later calls only launch kernels.
+ *   The array is shared by every call on the device, from every handle and
+ *   stream, and keeps the last call's contents.  Nothing in it needs to start
+ *   at zero: each forward writes every intermediate before reading it.  Calls
+ *   that overlap on the GPU race on the array and corrupt each other's
+ *   results: order them, e.g. on one stream. */
+ENC_API enc_status enc_forward_noalloc(enc_t h, const void* x, const int32_t* valid_len, void* out,
+                                       int batch, int seq, enc_stream_t stream);
+
 /* enc_forward_host - enc_forward on HOST buffers: copies x and valid_len to
  * handle-owned device staging buffers, runs the stack and copies the result
  * back into out, then synchronises `stream`.  The copies run on two

@@ -33,6 +33,7 @@ _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
     "enc_create": (_i, [_i, _i, _i, _i, _i, _vp, ctypes.POINTER(_vp)]),
     "enc_forward": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
+    "enc_forward_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "enc_forward_host": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "enc_forward_host_async": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "enc_host_join": (_i, [_vp, _vp]),
@@ -196,6 +197,14 @@ class Encoder:
             out = torch.empty_like(x)
         _check(self.lib.enc_forward(self.handle, _dptr(x), _dptr(valid_len), _dptr(out), B, S,
                                     _current_stream(stream)))
+        return out
+
+    def forward_noalloc(self, x, valid_len, out, stream=None):
+        """enc_forward_noalloc: the forward with its scratch in the library's fixed
+        device array (no device allocation); out must be given."""
+        B, S, H = x.shape
+        _check(self.lib.enc_forward_noalloc(self.handle, _dptr(x), _dptr(valid_len), _dptr(out), B, S,
+                                            _current_stream(stream)))
         return out
 
     def forward_host(self, x: np.ndarray, valid_len: np.ndarray, out: Optional[np.ndarray] = None,

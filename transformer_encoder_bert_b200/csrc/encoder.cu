@@ -18,6 +18,7 @@
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -852,6 +853,97 @@ enc_status enc_graph_destroy(enc_graph_t graph) {
   if (graph->graph) cudaGraphDestroy(graph->graph);
   if (graph->h) --graph->h->graphs_alive;
   delete graph;
+  return ok();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------- forward without allocation
+
+// Scratch of enc_forward_noalloc: a fixed array in the library's own device
+// image, so that the entry point needs no cudaMalloc.  Every GPU that loads the
+// library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_static_workspace[ENC_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+// In host code g_static_workspace names a host-side stand-in, not device
+// memory; its device address is looked up once per device, with that device
+// current, and kept here.
+constexpr int kMaxStaticDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_addr[kMaxStaticDevices] = {};
+
+enc_status static_workspace_address(int device, void** ptr) {
+  if (device < 0 || device >= kMaxStaticDevices)
+    return fail(ENC_ERR_UNSUPPORTED, "device %d is beyond the %d the static workspace table holds", device,
+                kMaxStaticDevices);
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_addr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static workspace");
+    g_static_ws_addr[device] = p;
+  }
+  *ptr = g_static_ws_addr[device];
+  return ENC_OK;
+}
+
+// The workspace layout of carve(), laid out from `base` instead of the
+// handle's own allocation.
+Workspace carve_at(const enc_handle* h, void* base, size_t tokens) {
+  const size_t es = h->esize;
+  const size_t mh = align_up(tokens * h->H * es, 256);
+  const size_t mf = align_up(tokens * h->F * es, 256);
+  char* p = static_cast<char*>(base);
+  Workspace w;
+  w.qkv = p; p += 3 * mh;
+  w.ctx = p; p += mh;
+  w.a = p; p += mh;
+  w.h1 = p; p += mh;
+  w.u = p; p += mf;
+  w.x0 = p; p += mh;
+  w.x1 = p; p += mh;
+  w.offsets = reinterpret_cast<int32_t*>(p);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+enc_status enc_forward_noalloc(enc_t h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                               enc_stream_t stream) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
+  if ((s = check_ptrs({x, out})) != ENC_OK) return s;
+  if (!valid_len) return fail(ENC_ERR_INVALID_ARG, "valid_len is null");
+  const size_t M = (size_t)batch * seq;
+  const size_t bytes = M * h->H * h->esize;
+  const char* xb = static_cast<const char*>(x);
+  const char* ob = static_cast<const char*>(out);
+  if (xb < ob + bytes && ob < xb + bytes) return fail(ENC_ERR_INVALID_ARG, "out overlaps x");
+  const size_t need = workspace_bytes(h, M);
+  if (need > ENC_STATIC_WORKSPACE_BYTES)
+    return fail(ENC_ERR_UNSUPPORTED,
+                "batch %d x seq %d needs %zu bytes of scratch; the static workspace of enc_forward_noalloc holds %zu",
+                batch, seq, need, (size_t)ENC_STATIC_WORKSPACE_BYTES);
+  void* base = nullptr;
+  if ((s = static_workspace_address(h->device, &base)) != ENC_OK) return s;
+  PdlScope pdl(h);
+  const Workspace w = carve_at(h, base, M);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto no_mark = [] {};
+  if (h->packed) {
+    s = forward_packed(h, x, valid_len, out, batch, seq, st, w, no_mark);
+    return s == ENC_OK ? ok() : s;
+  }
+  for (int l = 0; l < h->L; ++l) {
+    const void* xin = l == 0 ? x : (((l - 1) & 1) ? w.x1 : w.x0);
+    void* xout = l == h->L - 1 ? out : ((l & 1) ? w.x1 : w.x0);
+    if ((s = run_layer(h, l, xin, xout, valid_len, batch, seq, w, st, no_mark)) != ENC_OK) return s;
+  }
   return ok();
 }
 
