@@ -82,6 +82,7 @@ KERNEL_SOURCES = {
     "attention": ["attention.cu", "attention_tc.cu", "sm100.cuh", "internal.h"],
     "ln1": ["layernorm.cu", "internal.h"],
     "ln2": ["layernorm.cu", "internal.h"],
+    "persistent": ["persistent.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
 }
 
 
@@ -135,7 +136,14 @@ def kernel_work(wl: EI.Workload, attn_seq=None, attn_tokens=None):
     es = 2 if wl.dtype == "fp16" else 4
     def gemm(n, k, extra_out=0):
         return 2.0 * M * n * k, es * (M * k + k * n + M * n) + extra_out
+    L = sh.num_layers
+    weight_bytes = es * L * (3 * H * H + H * H + 2 * H * F)
     return {
+        # the whole stack in one launch: every GEMM and attention flop; bytes =
+        # every weight once plus the input and output rows (the activations in
+        # between stay in L2 at these sizes)
+        "persistent": (L * (2.0 * M * H * (4 * H + 2 * F) + 4.0 * M * S * H),
+                       weight_bytes + es * 2.0 * M * H + 4 * wl.batch),
         "qkv_gemm": gemm(3 * H, H),
         "attention": (4.0 * M * S * H, es * 4.0 * M * H + 4 * wl.batch),
         "out_proj_gemm": gemm(H, H, extra_out=es * M * H),     # epilogue reads the residual
@@ -286,6 +294,8 @@ def workload_config(wl: EI.Workload, world: int, l2: str):
 # ------------------------------------------------------------------ our arm
 def kernel_names(nk: int, num_layers: int, packed: bool):
     """Names of the nk kernels of one forward, in launch order."""
+    if nk == 1:
+        return ["persistent"]                 # the single-launch forward of the whole stack
     per_layer = (nk - (3 if packed else 0)) // num_layers
     layer_names = {5: KERNEL_NAMES_FUSED, 6: KERNEL_NAMES_FFN2_LN}.get(per_layer, KERNEL_NAMES)
     if packed:
@@ -367,7 +377,7 @@ def kernel_table(wl, inp, per_kernel, peaks, packed: bool):
         avg_ms = sum(vals) / len(vals)
         flops, nbytes = work[k]
         entry = {"avg_us": avg_ms * 1e3, "share": sum(vals) / total}
-        if flops and k.endswith("gemm"):
+        if flops and (k.endswith("gemm") or k == "persistent"):
             entry["tflops"] = flops / (avg_ms * 1e-3) / 1e12
             entry["tensor_frac"] = entry["tflops"] / tc_peak
         entry["gbs"] = nbytes / (avg_ms * 1e-3) / 1e9
@@ -379,6 +389,13 @@ def kernel_table(wl, inp, per_kernel, peaks, packed: bool):
 
 def roofline_of(kernels, work, dominant, peaks, peak_src, traffic):
     d = kernels[dominant]
+    if dominant == "persistent":
+        # small batch: every weight byte is read once per forward, so HBM bounds it
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        return {"bound": "hbm", "achieved": d["gbs"], "peak": peak, "unit": "GB/s", "frac": d["gbs"] / peak,
+                "traffic": traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
+                "peak_source": f"{peak_src} HBM copy bandwidth",
+                "time_source": "the whole forward is this one launch (CUDA events around it)"}
     if dominant.endswith("gemm"):
         peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         return {"bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
@@ -409,6 +426,9 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     enc = Encoder(sh.head_num, sh.size_per_head, sh.ffn_dim, inp.layers, wl.dtype)
     if args.packed:
         enc.set_packing(True)
+    options = dict(o.split("=", 1) for o in args.option)
+    for name, v in options.items():
+        enc.set_option(name, int(v))
     enc.reserve(wl.batch, wl.seq)
     x = torch.from_numpy(inp.x).to(dev)
     vl = torch.from_numpy(inp.valid_len).to(dev)
@@ -460,6 +480,8 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         enc2 = Encoder(ssh.head_num, ssh.size_per_head, ssh.ffn_dim, sec_inp.layers, sec_wl.dtype)
         if args.packed:
             enc2.set_packing(True)
+        for name, v in options.items():
+            enc2.set_option(name, int(v))
         enc2.reserve(sec_wl.batch, sec_wl.seq)
         x2 = torch.from_numpy(sec_inp.x).to(dev)
         vl2 = torch.from_numpy(sec_inp.valid_len).to(dev)
@@ -488,7 +510,8 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         "config": dict(workload_config(wl, world, l2="flushed before every timed step (256 MiB write)"),
                        launch="one recorded CUDA graph per step" if args.graph else "enc_forward per step",
                        padding="removed (valid tokens only; padded outputs zero)" if args.packed
-                       else "computed (fixed length)"),
+                       else "computed (fixed length)",
+                       **({"options": options} if options else {})),
         "roofline": roof,
         "e2e": {"value": job_throughput(wl.batch, world, e2e_step), "unit": UNIT,
                 "h2d_bytes_per_step": int(hx.numel() * hx.element_size() + hvl.numel() * 4),
@@ -543,6 +566,8 @@ def main(argv=None):
                     help="a second workload device-timed in the same run (one GPU; '' for none)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-sample", type=int, default=8, help="sequences per reference-arm step")
+    ap.add_argument("--option", action="append", default=[], metavar="NAME=VALUE",
+                    help="a kernel-path switch of the handle (enc_set_option), e.g. persistent=0")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if captured for the current sources")
     args = ap.parse_args(argv)

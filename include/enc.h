@@ -126,20 +126,37 @@ typedef enum {
   /* 1 (default): split-K thread-block clusters for GEMMs whose tiles would
    * leave more than half the SMs idle; 0: never split K. */
   ENC_OPT_SPLIT_K = 3,
-  /* 1 (default): the FFN2 GEMM writes LayerNorm 2 of its rows itself where the
-   * 2-CTA tiles run and the hidden size is 256, 512 or 768; 0: a separate
-   * LayerNorm kernel. */
+  /* Whether the FFN2 GEMM writes LayerNorm 2 of its rows itself (row
+   * statistics exchanged across the thread-block cluster that covers a row;
+   * needs the 2-CTA tiles and a hidden size that is a multiple of 256, at most
+   * 1024): 0 never (a separate LayerNorm kernel), 1 (default) where it measured
+   * faster (hidden size <= 768, clusters of at most 6 CTAs), 2 wherever
+   * supported. */
   ENC_OPT_LN_FUSE_FFN2 = 4,
-  /* 0 (default): a separate LayerNorm 1 kernel; 1: the output-projection GEMM
-   * writes LayerNorm 1 itself wherever the fused epilogue is supported. */
+  /* The same for the output-projection GEMM and LayerNorm 1 (0, 1 = default, 2). */
   ENC_OPT_LN_FUSE_OUT_PROJ = 5,
   /* 1 (default): kernels are launched with programmatic dependent launch, so
    * each one's set-up overlaps its predecessor's tail; 0: plain stream order. */
-  ENC_OPT_PDL = 6
+  ENC_OPT_PDL = 6,
+  /* 0 (default): the per-step kernels; 1: FP16 forwards of at most 256 tokens
+   * (batch * seq) without padding removal run as ONE persistent kernel for the
+   * whole stack, with grid-wide barriers between the steps ([FT] "Faster
+   * Transformer 优化原理": at small batch the launches, not the arithmetic, set
+   * the time).  Needs hidden and ffn sizes that are multiples of 64, hidden <=
+   * 1024; other shapes keep the per-step kernels.  Off by default because the
+   * per-step kernels, replayed as a CUDA graph with programmatic dependent
+   * launch, measured faster at every batch size. */
+  ENC_OPT_PERSISTENT = 7,
+  /* Failure-detection test of that single-launch forward, 0 by default: with
+   * 1, one CTA waits on a flag that nothing sets instead of joining the first
+   * grid-wide barrier, every wait of the launch gives up after 20 ms, and the
+   * launch reports status 1 through enc_device_status; the outputs of that
+   * forward are undefined and the context stays usable. */
+  ENC_OPT_TEST_STALL = 8
 } enc_option;
 
-/* enc_set_option - set one kernel-path switch of this handle (value 0 or 1;
- * else ENC_ERR_INVALID_ARG).  Host-side; takes effect at the next launch.  A
+/* enc_set_option - set one kernel-path switch of this handle (0 or 1; 0, 1 or 2
+ * for the two LayerNorm fusions; else ENC_ERR_INVALID_ARG).  Host-side; takes effect at the next launch.  A
  * recorded forward (enc_graph_create) keeps the kernels it recorded.  Not part
  * of the source pages' design: it exposes this library's own alternatives. */
 ENC_API enc_status enc_set_option(enc_t h, enc_option option, int value);
@@ -277,7 +294,8 @@ ENC_API enc_status enc_graph_launch(enc_graph_t graph, enc_stream_t stream);
 ENC_API enc_status enc_graph_destroy(enc_graph_t graph);
 
 /* enc_kernels_per_forward - kernel launches one enc_forward of batch x seq
- * issues: per layer 7, less one for each of the output-projection and FFN2
+ * issues: 1 when the single-launch forward runs (ENC_OPT_PERSISTENT);
+ * otherwise per layer 7, less one for each of the output-projection and FFN2
  * GEMMs that writes the LayerNorm of its rows itself (FP16, enough tokens for
  * the 2-CTA tiles; by default FFN2 with hidden size 256, 512 or 768); plus 3
  * with padding removal.  0 for invalid arguments. */
@@ -288,8 +306,8 @@ ENC_API int enc_kernels_per_forward(enc_t h, int batch, int seq);
 ENC_API uint64_t enc_launch_count(enc_t h);
 
 /* enc_set_trace_events - optional per-kernel timing of enc_forward.  events
- * holds count CUDA events (cudaEvent_t, created by the caller; at least
- * 5 * num_layers + 1, and a forward needing more fails with ENC_ERR_INVALID_ARG);
+ * holds count CUDA events (cudaEvent_t, created by the caller; at least 2, and
+ * a forward needing more than count fails with ENC_ERR_INVALID_ARG);
  * with count >= enc_kernels_per_forward(h, batch, seq) + 1, each enc_forward records events[k] on its
  * stream just before its k-th kernel and events[kernels] after the last, so
  * cudaEventElapsedTime(events[k], events[k+1]) is kernel k's duration.

@@ -192,7 +192,9 @@ def test_option_argument_checks():
     assert enc.lib.enc_set_option(enc.handle, 2, 2) == 1       # value not 0 or 1: ENC_ERR_INVALID_ARG
     assert enc.lib.enc_set_option(enc.handle, 99, 1) == 1      # unknown option
     assert enc.lib.enc_set_option(None, 2, 1) == 1             # null handle
-    assert enc.get_option("tc_attention") and not enc.get_option("ln_fuse_out_proj")
+    assert enc.get_option("tc_attention") and enc.get_option("ln_fuse_out_proj") == 1
+    assert enc.lib.enc_set_option(enc.handle, 5, 3) == 1       # the fusion switches take 0..2
+    assert enc.lib.enc_set_option(enc.handle, 5, 2) == 0
 
 
 def test_host_argument_checks():
@@ -355,16 +357,16 @@ PACKED_FULL_SIZE = [
 def test_packed_full_size_against_oracle(kind, batch, seq, nsample):
     """Padding removal at the sizes the bench runs it: every GEMM takes the 2-CTA
     tiles chosen from the padded token count and reads the real count T from the
-    device, and for hidden sizes up to 768 the FFN2 GEMM writes LayerNorm 2 itself
-    (6 launches per layer; 7 for BERT-Large), plus the offsets, pack and unpack
-    kernels.  A seeded sample of sequences (the first, the last and a shortest one
+    device, and for hidden sizes up to 768 the output-projection and FFN2 GEMMs
+    write LayerNorms 1 and 2 themselves (5 launches per layer; 7 for BERT-Large),
+    plus the offsets, pack and unpack kernels.  A seeded sample of sequences (the first, the last and a shortest one
     among them) against the oracle; every padded row is zero."""
     wl = EI.named_workload(kind, batch, seq)
     inp = EI.make_inputs(wl)
     enc = encoder_from_inputs(inp)
     enc.set_packing(True)
     L = wl.shape.num_layers
-    per_layer = 6 if wl.shape.hidden <= 768 else 7
+    per_layer = 5 if wl.shape.hidden <= 768 else 7
     assert enc.kernels_per_forward(wl.batch, wl.seq) == per_layer * L + 3
     got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
     m = valid_mask(inp.valid_len, wl.seq)
@@ -399,3 +401,101 @@ def test_packed_mode_needs_fp16():
     with pytest.raises(EncError) as e:
         enc.set_packing(True)
     assert e.value.status == 2
+
+
+# ---------------------------------------------------------------- single-launch small-batch forward
+
+@pytest.mark.parametrize("batch", [1, 8])
+def test_single_launch_forward_bert_base_against_oracle(batch):
+    """BERT-Base, 12 layers, seq 32, batch 1 and 8: one persistent kernel runs the
+    whole stack (grid-wide barriers between the steps, LayerNorms applied as the
+    next GEMM loads its operand).  Against the oracle on every sequence, and
+    against the per-step kernels within the 12-layer bound."""
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", batch))
+    enc = encoder_from_inputs(inp)
+    assert not enc.get_option("persistent")       # off by default: the per-step graph measured faster
+    enc.set_option("persistent", True)
+    assert enc.kernels_per_forward(batch, 32) == 1
+    n0 = enc.launch_count()
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    assert enc.launch_count() - n0 == 1
+    _check(got, _oracle(inp), inp.valid_len, 32, FP16_STACK_REL_L2)
+    enc.set_option("persistent", False)
+    assert enc.kernels_per_forward(batch, 32) > 1
+    per_step = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    assert rel_l2(got, per_step, valid_mask(inp.valid_len, 32)) < FP16_STACK_REL_L2
+    assert enc.device_status() == 0
+
+
+@pytest.mark.parametrize("nh,d,F,L,batch,seq", [
+    (4, 32, 512, 2, 5, 37),        # pruned structure, ragged token count (185 rows)
+    (16, 64, 4096, 2, 2, 128),     # BERT-Large structure, 256 tokens (FFN2 in units of 8 features)
+    (8, 128, 2048, 2, 3, 21),      # size-128 heads
+    (12, 64, 3072, 1, 1, 1),       # one token
+    (12, 64, 3072, 2, 4, 64),      # 256 tokens, longer sequences
+], ids=str)
+def test_single_launch_forward_structures(nh, d, F, L, batch, seq):
+    sh = EI.EncoderShape(nh, d, F, L)
+    inp = EI.make_inputs(EI.Workload("single", sh, batch, seq, "fp16", 1, seq, seed=nh + seq,
+                                     ln_affine_random=True))
+    inp.valid_len[0] = seq
+    enc = encoder_from_inputs(inp)
+    enc.set_option("persistent", True)
+    assert enc.kernels_per_forward(batch, seq) == 1
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    _check(got, _oracle(inp), inp.valid_len, seq, L * FP16_LAYER_REL_L2)
+    assert enc.device_status() == 0
+
+
+def test_single_launch_forward_empty_sequence_and_tanh_gelu():
+    sh = EI.EncoderShape(12, 64, 3072, 2)
+    inp = EI.make_inputs(EI.Workload("single-empty", sh, 4, 33, "fp16", 1, 33, seed=8))
+    inp.valid_len[2] = 0                       # no valid key: ctx = 0 for that sequence
+    enc = encoder_from_inputs(inp)
+    enc.set_option("persistent", True)
+    enc.set_gelu("tanh")
+    assert enc.kernels_per_forward(4, 33) == 1
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    x64, vl, layers = inp.as_float64()
+    ref = O.encoder_forward(x64, vl, layers, 12, 64, gelu="tanh")
+    _check(got, ref, vl, 33, 2 * FP16_LAYER_REL_L2)
+    assert np.all(np.isfinite(got))
+    assert enc.device_status() == 0
+
+
+def test_single_launch_forward_replays_and_is_deterministic():
+    import torch
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 2))
+    enc = encoder_from_inputs(inp)
+    enc.set_option("persistent", True)
+    x, vl = to_dev(inp.x), to_dev(inp.valid_len)
+    ref = to_host(enc.forward(x, vl))
+    assert np.array_equal(ref, to_host(enc.forward(x, vl)))      # fixed summation order
+    out = torch.zeros_like(x)
+    g = enc.record(x, vl, out)
+    n0 = enc.launch_count()
+    for _ in range(3):
+        g.launch()
+    torch.cuda.synchronize()
+    assert enc.launch_count() - n0 == 3
+    assert np.array_equal(to_host(out), ref)
+    g.close()
+    assert enc.device_status() == 0
+
+
+def test_single_launch_forward_wait_timeout_sets_status():
+    """Failure detection without a GPU fault: with the test_stall option one CTA
+    waits on a flag that nothing sets instead of joining the first grid-wide
+    barrier; every wait of that launch gives up after 20 ms, the kernel returns
+    and reports status 1.  The context stays usable: the next forward is correct."""
+    inp = EI.make_inputs(EI.named_workload("bert-base-s32", 1).with_(shape=EI.EncoderShape(12, 64, 3072, 2)))
+    enc = encoder_from_inputs(inp)
+    enc.set_option("persistent", True)
+    x, vl = to_dev(inp.x), to_dev(inp.valid_len)
+    enc.set_option("test_stall", True)
+    enc.forward(x, vl)
+    assert enc.device_status() == 1
+    enc.set_option("test_stall", False)
+    got = to_host(enc.forward(x, vl))
+    _check(got, _oracle(inp), inp.valid_len, 32, 2 * FP16_LAYER_REL_L2)
+    assert enc.device_status() == 0

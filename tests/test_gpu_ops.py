@@ -107,15 +107,15 @@ def test_out_proj_ffn1_ffn2(shape, batch, seq):
 def test_fused_layernorm_gemms(shape, M):
     """Enough tokens for the 2-CTA tiles: the GEMMs write the LayerNorm of their rows
     (row statistics exchanged across the cluster that covers the row; clusters of
-    2, 6 and 8 CTAs for H = 256, 768, 1024).  FFN2 is fused by default for H <= 768,
-    the output projection through the ln_fuse_out_proj option.  Against the oracle
+    2, 6 and 8 CTAs for H = 256, 768, 1024).  Both GEMMs fuse by default for
+    H <= 768; the options' value 2 fuses wherever supported.  Against the oracle
     step, and against the unfused path (GEMM writing bias + residual, then the
-    LayerNorm kernel; both fusion options off)."""
+    LayerNorm kernel; both fusion options 0)."""
     nh, d, F = shape
     H = nh * d
     wl, inp, enc, x64, vl, lw = _setup(shape, 1, M)
-    enc.set_option("ln_fuse_out_proj", True)
-    enc.set_option("ln_fuse_ffn2", True)
+    enc.set_option("ln_fuse_out_proj", 2)         # wherever supported (H = 1024 too)
+    enc.set_option("ln_fuse_ffn2", 2)
     ctx = EI.random_array((M, H), "fp16", seed=41)
     resid = EI.random_array((M, H), "fp16", seed=42, mean=0.2)
     uu = EI.random_array((M, F), "fp16", seed=43, std=0.5)
@@ -140,6 +140,29 @@ def test_fused_layernorm_gemms(shape, M):
     enc1.set_option("ln_fuse_ffn2", False)
     un_a, un_y = run(enc1)
     assert rel_l2(got_a, un_a) < GEMM_REL_L2 and rel_l2(got_y, un_y) < GEMM_REL_L2
+
+
+@pytest.mark.parametrize("shape,M", [((4, 32, 512), 4100), ((8, 32, 1024), 2053), ((12, 64, 3072), 5000),
+                                     ((10, 64, 2560), 3001), ((16, 64, 4096), 2049), ((12, 64, 3072), 32768)],
+                         ids=lambda v: str(v))
+def test_layernorm_kernel_many_rows(shape, M):
+    """The LayerNorm kernel after a GEMM that wrote z = acc + bias + residual,
+    at thousands of rows (both fusions off so that it runs), hidden sizes 128
+    to 1024 and ragged row counts, against the oracle step."""
+    nh, d, F = shape
+    H = nh * d
+    wl, inp, enc, x64, vl, lw = _setup(shape, 1, M)
+    enc.set_option("ln_fuse_ffn2", False)
+    enc.set_option("ln_fuse_out_proj", False)
+    ctx = EI.random_array((M, H), "fp16", seed=51)
+    resid = EI.random_array((M, H), "fp16", seed=52, mean=0.3)
+    a = empty_dev((M, H), "fp16")
+    enc.op_out_proj_ln(0, to_dev(ctx), to_dev(resid), a, M)
+    ref = O.bias_residual_layernorm(ctx.astype(np.float64) @ lw["w_o"], lw["b_o"], resid.astype(np.float64),
+                                    lw["ln1_g"], lw["ln1_b"])
+    got = to_host(a)
+    assert rel_l2(got, ref) < GEMM_REL_L2 and max_abs(got, ref) < LN_MAX_ABS
+    assert enc.device_status() == 0
 
 
 @pytest.mark.parametrize("shape", [(4, 32, 512), (12, 64, 3072)], ids=lambda s: f"{s[0]}x{s[1]}")

@@ -22,7 +22,7 @@ NP_DTYPES = {"fp32": np.float32, "fp16": np.float16}
 
 # enc_option codes (kernel-path switches; every choice computes the same result to rounding).
 OPTION_CODES = {"pair_tiles": 0, "tma_store": 1, "tc_attention": 2, "split_k": 3, "ln_fuse_ffn2": 4,
-                "ln_fuse_out_proj": 5, "pdl": 6}
+                "ln_fuse_out_proj": 5, "pdl": 6, "persistent": 7, "test_stall": 8}
 
 # Field order of enc_layer_weights.
 WEIGHT_FIELDS = ("w_qkv", "b_qkv", "w_o", "b_o", "ln1_g", "ln1_b",
@@ -171,14 +171,15 @@ class Encoder:
         """Padding removal: compute valid tokens only; padded output rows become zeros."""
         _check(self.lib.enc_set_packing(self.handle, 1 if enable else 0))
 
-    def set_option(self, name: str, value: bool):
-        """One kernel-path switch (see OPTION_CODES and enc_option in include/enc.h)."""
-        _check(self.lib.enc_set_option(self.handle, OPTION_CODES[name], 1 if value else 0))
+    def set_option(self, name: str, value):
+        """One kernel-path switch (see OPTION_CODES and enc_option in include/enc.h):
+        a bool, or 0/1/2 for the two LayerNorm fusions."""
+        _check(self.lib.enc_set_option(self.handle, OPTION_CODES[name], int(value)))
 
-    def get_option(self, name: str) -> bool:
+    def get_option(self, name: str) -> int:
         v = ctypes.c_int(0)
         _check(self.lib.enc_get_option(self.handle, OPTION_CODES[name], ctypes.byref(v)))
-        return bool(v.value)
+        return int(v.value)
 
     def set_host_chunks(self, chunks: int):
         _check(self.lib.enc_set_host_chunks(self.handle, chunks))

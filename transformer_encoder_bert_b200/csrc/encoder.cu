@@ -122,9 +122,16 @@ struct enc_handle {
   bool tma_store = true;            // ENC_OPT_TMA_STORE: GEMM epilogues store (and read the residual) by TMA
   bool tc_attn = true;              // ENC_OPT_TC_ATTENTION: tcgen05 attention for d = 64, seq > 64
   bool splitk = true;               // ENC_OPT_SPLIT_K: split-K clusters for GEMMs that would idle most SMs
-  bool ln_fuse_ffn2 = true;         // ENC_OPT_LN_FUSE_FFN2: FFN2 writes LayerNorm 2 where supported
-  bool ln_fuse_oproj = false;       // ENC_OPT_LN_FUSE_OUT_PROJ: the output projection writes LayerNorm 1
+  // ENC_OPT_LN_FUSE_FFN2 / _OUT_PROJ: the GEMM writes the LayerNorm of its rows
+  // (0 never, 1 where measured faster: hidden size <= 768, 2 wherever supported)
+  int ln_fuse_ffn2 = 1;
+  int ln_fuse_oproj = 1;
   bool pdl = true;                  // ENC_OPT_PDL: programmatic dependent launch between kernels
+  bool persistent = false;          // ENC_OPT_PERSISTENT: single-launch forward for small batches
+  bool stall_test = false;          // ENC_OPT_TEST_STALL: failure-detection test of that forward
+  enc::PersistLayer* d_players = nullptr;   // device copy of every layer's pointers (FP16 mode)
+  CUtensorMap* d_wmaps = nullptr;           // device [L][4] weight maps of the single-launch forward
+  void* persist_partial = nullptr;          // its FFN2 partial tiles and tile counters
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
 };
 
@@ -320,7 +327,52 @@ bool ln_fused(const enc_handle* h, int tokens, int which) {
   if (h->dtype != ENC_FP16 || !h->tma_store || !enc::gemm_ln_supported(tokens, h->H) ||
       choose_bn(h, tokens, h->H) != enc::kPairTile)
     return false;
-  return which == 2 ? (h->ln_fuse_ffn2 && h->H <= 768) : h->ln_fuse_oproj;
+  const int mode = which == 2 ? h->ln_fuse_ffn2 : h->ln_fuse_oproj;
+  return mode == 2 || (mode == 1 && h->H <= 768);
+}
+
+// The single-launch forward (persistent.cu): FP16, padding kept, few enough
+// tokens that every GEMM is a weight stream.
+bool use_persistent(const enc_handle* h, int batch, int seq) {
+  return h->dtype == ENC_FP16 && !h->packed && h->persistent && h->persist_partial && h->d_wmaps &&
+         enc::persistent_supported(batch, seq, h->nh, h->d, h->F, h->num_sms);
+}
+
+enc_status run_persistent(enc_handle* h, const void* x, const int32_t* valid_len, void* out, int batch, int seq,
+                          const Workspace& w, cudaStream_t st) {
+  enc::PersistArgs a;
+  const int M = batch * seq;
+  const uint32_t box_rows = (uint32_t)(16 * ((M + 15) / 16));
+  const void* abase[5] = {x, w.x0, w.ctx, w.a, w.u};        // x, z2, ctx, z1, u
+  for (int i = 0; i < 5; ++i)
+    if (!enc::encode_kmajor_fp16_map(&a.amap[i], abase[i], (uint64_t)M, (uint64_t)(i == 4 ? h->F : h->H), box_rows))
+      return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation operand");
+  a.wmaps = h->d_wmaps;
+  a.layers = h->d_players;
+  a.L = h->L;
+  a.x = static_cast<const __half*>(x);
+  a.valid_len = valid_len;
+  a.out = static_cast<__half*>(out);
+  a.B = batch; a.S = seq; a.NH = h->nh; a.D = h->d; a.F = h->F;
+  a.qkv = static_cast<__half*>(w.qkv);
+  a.ctx = static_cast<__half*>(w.ctx);
+  a.z1 = static_cast<__half*>(w.a);
+  a.h1 = static_cast<__half*>(w.h1);
+  a.u = static_cast<__half*>(w.u);
+  a.z2 = static_cast<__half*>(w.x0);
+  a.xl = static_cast<__half*>(w.x1);
+  a.partial = static_cast<float*>(h->persist_partial);
+  a.tile_cnt = reinterpret_cast<unsigned*>(static_cast<char*>(h->persist_partial) +
+                                           (size_t)enc::kPersistMaxSplits * enc::kPersistMaxTokens * h->H * 4);
+  a.gelu_tanh = h->gelu == ENC_GELU_TANH ? 1 : 0;
+  a.bar = reinterpret_cast<unsigned*>(h->status + 4);
+  a.status = h->status;
+  a.stall_test = h->stall_test ? 1 : 0;
+  a.wait_ns = h->stall_test ? 20000000ull : 2000000000ull;   // 20 ms in the failure test, else 2 s
+  cudaError_t e = enc::launch_persistent(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "single-launch forward");
+  ++h->launches;
+  return ENC_OK;
 }
 
 int kernels_per_layer(const enc_handle* h, int tokens) {
@@ -413,6 +465,9 @@ void free_handle(enc_handle* h) {
   if (h->ws) cudaFree(h->ws);
   if (h->stage) cudaFree(h->stage);
   if (h->status) cudaFree(h->status);
+  if (h->d_players) cudaFree(h->d_players);
+  if (h->d_wmaps) cudaFree(h->d_wmaps);
+  if (h->persist_partial) cudaFree(h->persist_partial);
   delete h;
 }
 
@@ -529,7 +584,9 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
       return fail(ENC_ERR_UNSUPPORTED, "FP16 mode needs an sm_100 (B200-class) device");
     }
   }
-  if (cudaMalloc(&h->status, sizeof(int)) != cudaSuccess || cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) {
+  // The status word, then (16 bytes on) the four barrier words of the single-launch forward.
+  if (cudaMalloc(&h->status, 8 * sizeof(int)) != cudaSuccess ||
+      cudaMemset(h->status, 0, 8 * sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
     free_handle(h);
     return fail(ENC_ERR_OOM, "status word allocation failed");
@@ -618,6 +675,50 @@ enc_status enc_create(int head_num, int size_per_head, int ffn_dim, int num_laye
           free_handle(h);
           return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight operand");
         }
+      }
+    }
+  }
+  if (dtype == ENC_FP16) {
+    std::vector<enc::PersistLayer> pl(num_layers);
+    for (int l = 0; l < num_layers; ++l) {
+      const LayerDev& L = h->layers[l];
+      pl[l] = {static_cast<const __half*>(L.w_qkv), static_cast<const __half*>(L.w_o),
+               static_cast<const __half*>(L.w_ff1), static_cast<const __half*>(L.w_ff2),
+               L.b_qkv, L.b_o, L.b_ff1, L.b_ff2, L.ln1_g, L.ln1_b, L.ln2_g, L.ln2_b};
+    }
+    const size_t bytes = sizeof(enc::PersistLayer) * num_layers;
+    if (cudaMalloc(&h->d_players, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      free_handle(h);
+      return fail(ENC_ERR_OOM, "layer table allocation failed");
+    }
+    cudaError_t e = cudaMemcpy(h->d_players, pl.data(), bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "layer table upload"); }
+    // Weight maps of the single-launch forward: box of 64 columns x 32 rows.
+    std::vector<CUtensorMap> wm((size_t)num_layers * 4);
+    for (int l = 0; l < num_layers; ++l) {
+      const LayerDev& L = h->layers[l];
+      const struct { void* w; int n, k; } ws[4] = {
+          {L.w_qkv, 3 * H, H}, {L.w_o, H, H}, {L.w_ff1, ffn_dim, H}, {L.w_ff2, H, ffn_dim}};
+      for (int i = 0; i < 4; ++i)
+        if (!enc::encode_kmajor_fp16_map(&wm[(size_t)l * 4 + i], ws[i].w, ws[i].n, ws[i].k, 32)) {
+          free_handle(h);
+          return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight operand");
+        }
+    }
+    if (cudaMalloc(&h->d_wmaps, wm.size() * sizeof(CUtensorMap)) != cudaSuccess) {
+      cudaGetLastError();
+      free_handle(h);
+      return fail(ENC_ERR_OOM, "weight map allocation failed");
+    }
+    e = cudaMemcpy(h->d_wmaps, wm.data(), wm.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "weight map upload"); }
+    if (H % 32 == 0) {
+      const size_t pb = enc::persistent_partial_bytes(H, ffn_dim);
+      if (cudaMalloc(&h->persist_partial, pb) != cudaSuccess || cudaMemset(h->persist_partial, 0, pb) != cudaSuccess) {
+        cudaGetLastError();
+        free_handle(h);
+        return fail(ENC_ERR_OOM, "partial-tile allocation of %zu bytes failed", pb);
       }
     }
   }
@@ -765,6 +866,12 @@ enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, 
     if (tracing) cudaEventRecord(h->trace[k++], st);
   };
   if (h->packed) return forward_packed(h, x, valid_len, out, batch, seq, st, w, mark);
+  if (use_persistent(h, batch, seq)) {
+    mark();
+    if ((s = run_persistent(h, x, valid_len, out, batch, seq, w, st)) != ENC_OK) return s;
+    mark();
+    return ENC_OK;
+  }
   (void)tokens;
   for (int l = 0; l < h->L; ++l) {
     const void* xin = l == 0 ? x : (((l - 1) & 1) ? w.x1 : w.x0);
@@ -1111,6 +1218,7 @@ enc_status enc_device_status(enc_t h, int32_t* code) {
 
 int enc_kernels_per_forward(enc_t h, int batch, int seq) {
   if (!h || batch <= 0 || seq <= 0) return 0;
+  if (use_persistent(h, batch, seq)) return 1;
   return kernels_per_layer(h, batch * seq) * h->L + (h->packed ? 3 : 0);
 }
 
@@ -1124,16 +1232,20 @@ enc_status enc_set_packing(enc_t h, int enable) {
 
 enc_status enc_set_option(enc_t h, enc_option option, int value) {
   if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
-  if (value != 0 && value != 1) return fail(ENC_ERR_INVALID_ARG, "option value %d is not 0 or 1", value);
+  const bool three = option == ENC_OPT_LN_FUSE_FFN2 || option == ENC_OPT_LN_FUSE_OUT_PROJ;
+  if (value < 0 || value > (three ? 2 : 1))
+    return fail(ENC_ERR_INVALID_ARG, "option %d takes 0..%d, not %d", (int)option, three ? 2 : 1, value);
   const bool v = value != 0;
   switch (option) {
     case ENC_OPT_PAIR_TILES: h->pair_tiles = v; break;
     case ENC_OPT_TMA_STORE: h->tma_store = v; break;
     case ENC_OPT_TC_ATTENTION: h->tc_attn = v; break;
     case ENC_OPT_SPLIT_K: h->splitk = v; break;
-    case ENC_OPT_LN_FUSE_FFN2: h->ln_fuse_ffn2 = v; break;
-    case ENC_OPT_LN_FUSE_OUT_PROJ: h->ln_fuse_oproj = v; break;
+    case ENC_OPT_LN_FUSE_FFN2: h->ln_fuse_ffn2 = value; break;
+    case ENC_OPT_LN_FUSE_OUT_PROJ: h->ln_fuse_oproj = value; break;
     case ENC_OPT_PDL: h->pdl = v; break;
+    case ENC_OPT_PERSISTENT: h->persistent = v; break;
+    case ENC_OPT_TEST_STALL: h->stall_test = v; break;
     default: return fail(ENC_ERR_INVALID_ARG, "unknown option %d", (int)option);
   }
   return ok();
@@ -1142,7 +1254,7 @@ enc_status enc_set_option(enc_t h, enc_option option, int value) {
 enc_status enc_get_option(enc_t h, enc_option option, int* value) {
   if (!h) return fail(ENC_ERR_INVALID_ARG, "null handle");
   if (!value) return fail(ENC_ERR_INVALID_ARG, "value is null");
-  bool v;
+  int v;
   switch (option) {
     case ENC_OPT_PAIR_TILES: v = h->pair_tiles; break;
     case ENC_OPT_TMA_STORE: v = h->tma_store; break;
@@ -1151,9 +1263,11 @@ enc_status enc_get_option(enc_t h, enc_option option, int* value) {
     case ENC_OPT_LN_FUSE_FFN2: v = h->ln_fuse_ffn2; break;
     case ENC_OPT_LN_FUSE_OUT_PROJ: v = h->ln_fuse_oproj; break;
     case ENC_OPT_PDL: v = h->pdl; break;
+    case ENC_OPT_PERSISTENT: v = h->persistent; break;
+    case ENC_OPT_TEST_STALL: v = h->stall_test; break;
     default: return fail(ENC_ERR_INVALID_ARG, "unknown option %d", (int)option);
   }
-  *value = v ? 1 : 0;
+  *value = v;
   return ok();
 }
 
@@ -1180,8 +1294,7 @@ enc_status enc_set_trace_events(enc_t h, void* const* events, int count) {
     h->trace.clear();
     return ok();
   }
-  if (count < 5 * h->L + 1)
-    return fail(ENC_ERR_INVALID_ARG, "need at least %d trace events, got %d", 5 * h->L + 1, count);
+  if (count < 2) return fail(ENC_ERR_INVALID_ARG, "need at least 2 trace events, got %d", count);
   h->trace.assign(reinterpret_cast<cudaEvent_t const*>(events), reinterpret_cast<cudaEvent_t const*>(events) + count);
   return ok();
 }

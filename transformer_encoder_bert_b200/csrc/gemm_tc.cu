@@ -27,6 +27,7 @@
 
 #include <cudaTypedefs.h>
 
+#include "gelu.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -66,60 +67,6 @@ struct Cfg {
   static constexpr int kStoreOffset = (kBiasOffset + kEpiWarps * (BN / kEpiSlices) * 4 + 1023) / 1024 * 1024;
   static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * 2 * (32 * 32 * 2);   // two staging buffers per warp
 };
-
-// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), with erf from the
-// rational approximation of Abramowitz & Stegun, Handbook of Mathematical
-// Functions, formula 7.1.28: for z >= 0,
-//   erf(z) = 1 - 1 / (1 + a1 z + a2 z^2 + a3 z^3 + a4 z^4 + a5 z^5 + a6 z^6)^16,
-// |error| <= 3e-7, and erf(-z) = -erf(z).  The 16th power is four squarings, so
-// an element costs one reciprocal (special-function unit) and a dozen FMA-pipe
-// operations, which keeps the FFN1 epilogue behind its MMAs.  For large z the
-// power overflows to +inf and the reciprocal gives 0, i.e. erf = 1.  The error
-// is far below the FP16 rounding of the stored result.
-// Two elements are evaluated at once with the packed FP32 instructions of
-// sm_100 (fma/mul .f32x2): the polynomial, the squarings and the final
-// scaling cost one instruction per pair; the reciprocal and the sign stay per
-// element.
-__device__ __forceinline__ void gelu_erf_pair(float& v0, float& v1) {
-  const uint64_t v = f2_pack(v0, v1);
-  const uint64_t z = f2_mul(f2_pack(fabsf(v0), fabsf(v1)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
-  uint64_t q = f2_fma(z, f2_pack(0.0000430638f, 0.0000430638f), f2_pack(0.0002765672f, 0.0002765672f));
-  q = f2_fma(z, q, f2_pack(0.0001520143f, 0.0001520143f));
-  q = f2_fma(z, q, f2_pack(0.0092705272f, 0.0092705272f));
-  q = f2_fma(z, q, f2_pack(0.0422820123f, 0.0422820123f));
-  q = f2_fma(z, q, f2_pack(0.0705230784f, 0.0705230784f));
-  q = f2_fma(z, q, f2_pack(1.0f, 1.0f));
-  q = f2_mul(q, q);
-  q = f2_mul(q, q);
-  q = f2_mul(q, q);
-  q = f2_mul(q, q);
-  float q0, q1, r0, r1;
-  f2_unpack(q, q0, q1);
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(q0));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(q1));
-  // erf(|z|) = 1 - r >= 0; give it the sign of v
-  const uint64_t e = f2_fma(f2_pack(r0, r1), f2_pack(-1.0f, -1.0f), f2_pack(1.0f, 1.0f));
-  float e0, e1;
-  f2_unpack(e, e0, e1);
-  e0 = copysignf(e0, v0);
-  e1 = copysignf(e1, v1);
-  const uint64_t hv = f2_mul(v, f2_pack(0.5f, 0.5f));
-  f2_unpack(f2_fma(hv, f2_pack(e0, e1), hv), v0, v1);
-}
-
-// tanh form of GELU: 0.5 v (1 + tanh(u)), u = sqrt(2/pi) (v + 0.044715 v^3), with
-// tanh(u) = 1 - 2 / (exp(2u) + 1) (one exponential and one reciprocal on the
-// special-function unit; exp overflowing to +inf gives tanh = 1, underflowing
-// to 0 gives -1).
-__device__ __forceinline__ float gelu_tanh(float v) {
-  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
-  float e, r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(u * 2.8853900817779268f));   // exp(2u) = 2^(2u log2 e)
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(e + 1.0f));
-  const float th = fmaf(-2.0f, r, 1.0f);
-  const float hv = 0.5f * v;
-  return fmaf(hv, th, hv);
-}
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -171,11 +118,11 @@ __device__ __forceinline__ void epilogue_values(const uint32_t (&r)[32], const f
   }
   if constexpr (EPI == Epi::kBiasGelu) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) gelu_erf_pair(v[i], v[i + 1]);
+    for (int i = 0; i < 32; i += 2) act::gelu_erf_pair(v[i], v[i + 1]);
   }
   if constexpr (EPI == Epi::kBiasGeluTanh) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+    for (int i = 0; i < 32; ++i) v[i] = act::gelu_tanh(v[i]);
   }
 }
 
@@ -224,7 +171,7 @@ struct EpiWarpState {
 // brought into the chunk's staging buffer by a TMA load (the next chunk's
 // while this one is processed) and added in place; otherwise each lane loads
 // its row's halves.
-template <Epi EPI, int CHUNKS, typename WaitFull, typename Release>
+template <Epi EPI, int CHUNKS, int NBUF = 2, typename WaitFull, typename Release>
 __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, int col_begin, int M, int N,
                                                    const float* __restrict__ bias, float* bias_s,
                                                    __half* __restrict__ C, const SplitShape& sp,
@@ -247,16 +194,30 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
   const int s0 = EPI == Epi::kBiasQkvSplit ? row0 - b0 * sp.seq : 0;
   constexpr bool kResid = EPI == Epi::kBiasResidStore;
   const bool tma_resid = kResid && tm_c != nullptr && ws.tm_r != nullptr;
-  auto buf_of = [&](uint32_t seq) { return ws.stage + (seq & 1u) * kStageChunkBytes; };
+  // With a buffer per chunk (NBUF >= CHUNKS) every residual chunk of the tile
+  // is requested before the accumulator is awaited, chunk j into buffer j;
+  // otherwise two buffers alternate and the residual runs one chunk ahead.
+  constexpr bool kAllAhead = NBUF >= CHUNKS;
+  auto buf_of = [&](uint32_t seq) {
+    return ws.stage + (kAllAhead ? (seq % (uint32_t)NBUF) : (seq & 1u)) * kStageChunkBytes;
+  };
   // Lane 0: residual chunk j into the buffer of chunk number `seq`, once every
   // store this thread issued has read its buffer.
   auto issue_res = [&](uint32_t seq, int j) {
-    sm100::bulk_wait_group_read<0>();
-    const uint32_t bar = ws.res_bar + 8u * (seq & 1u);
+    if (!kAllAhead) sm100::bulk_wait_group_read<0>();
+    const uint32_t bar = ws.res_bar + 8u * (kAllAhead ? (seq % (uint32_t)NBUF) : (seq & 1u));
     sm100::mbar_arrive_expect_tx(bar, kStageChunkBytes);
     sm100::tma_load_2d(ws.tm_r, sm100::smem_u32(buf_of(seq)), bar, col_begin + 32 * j, row0);
   };
-  if (tma_resid && lane == 0 && col_begin < N) issue_res(ws.seq, 0);
+  if (tma_resid && lane == 0) {
+    if constexpr (kAllAhead) {
+      sm100::bulk_wait_group_read<0>();        // the previous tile's stores have read every buffer
+      for (int j = 0; j < CHUNKS; ++j)
+        if (col_begin + 32 * j < N) issue_res(ws.seq + j, j);
+    } else if (col_begin < N) {
+      issue_res(ws.seq, 0);
+    }
+  }
   // Per-lane residual path: chunk 0 before the accumulator is awaited, chunk
   // j+1 while chunk j is processed.
   uint4 res_a[4] = {}, res_b[kResid ? 4 : 1] = {};
@@ -301,12 +262,12 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
     const int col0 = col_begin + 32 * j;
     if (col0 >= N) continue;
     if (kResid && !tma_resid && j + 1 < CHUNKS) load_res(j + 1, (j & 1) ? res_a : res_b);
-    if (tma_resid && lane == 0 && j + 1 < CHUNKS && col0 + 32 < N) issue_res(ws.seq + 1, j + 1);
+    if (!kAllAhead && tma_resid && lane == 0 && j + 1 < CHUNKS && col0 + 32 < N) issue_res(ws.seq + 1, j + 1);
     float v[32];
     epilogue_values<EPI>(cur, bias_s + 32 * j, v);
     uint8_t* buf = buf_of(ws.seq);
     if (tma_resid) {
-      const uint32_t k = ws.seq & 1u;
+      const uint32_t k = kAllAhead ? (ws.seq % (uint32_t)NBUF) : (ws.seq & 1u);
       int ok = 0;
       if (lane == 0) ok = mbar_wait<kSleepNs>(ws.res_bar + 8u * k, (ws.res_phase >> k) & 1u, kWaitLimitNs) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -719,14 +680,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   - Both CTAs' epilogue warps release an accumulator on the leader's
 //     accumulator-empty barrier (count 2 x kEpiWarps).
 // ---------------------------------------------------------------------------
-struct PairCfg {
-  static constexpr int kStages = 5;
+// The bias + residual epilogue (output projection, FFN2 without the fused
+// LayerNorm) keeps four staging buffers per warp instead of two, so that the
+// residual of all four of a warp's 32-column chunks is fetched while the
+// tile's MMAs run; one operand stage fewer pays for them.
+template <Epi EPI>
+struct PairCfgT {
+  static constexpr bool kResAll = EPI == Epi::kBiasResidStore;
+  static constexpr int kStoreBufs = kResAll ? 4 : 2;          // staging buffers per epilogue warp
+  static constexpr int kStages = kResAll ? 4 : 5;
   static constexpr int kABytes = 128 * kBK * 2;
   static constexpr int kBBytes = 128 * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;             // two 256-column accumulators
   static constexpr int kResBar0 = 2 * kStages + 5;
-  static constexpr int kLnBar0 = kResBar0 + 2 * kEpiWarps;   // LayerNorm: local, ready[2]
+  static constexpr int kLnBar0 = kResBar0 + kStoreBufs * kEpiWarps;   // LayerNorm: local, ready[2]
   static constexpr int kNumBars = kLnBar0 + 3;
   static constexpr int kBiasOffset = (kStages * kStageBytes + kNumBars * 8 + 16 + 15) / 16 * 16;
   // Per epilogue warp: bias (and, for the fused LayerNorm, gamma and beta) of its columns.
@@ -734,7 +702,8 @@ struct PairCfg {
   static constexpr int kStatsOffset = (kBiasOffset + kEpiWarps * kParamFloats * 4 + 15) / 16 * 16;
   static constexpr int kStatsBytes = 2 * 2 * 128 * 8;       // LayerNorm statistics, [2][2][128] float2
   static constexpr int kStoreOffset = (kStatsOffset + kStatsBytes + 1023) / 1024 * 1024;
-  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * 2 * (32 * 32 * 2);
+  static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * kStoreBufs * (32 * 32 * 2);
+  static_assert(kSmem <= 227 * 1024, "dynamic shared memory of one CTA");
 };
 
 // CL = CTAs per cluster: 2 (one pair) for every epilogue but the fused
@@ -750,7 +719,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
                         int* __restrict__ status, const int* __restrict__ m_dev, const __half* __restrict__ resid,
                         const float* __restrict__ ln_gamma, const float* __restrict__ ln_beta) {
   constexpr bool kLn = EPI == Epi::kBiasResidLN;
-  using G = PairCfg;
+  using G = PairCfgT<EPI>;
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -788,7 +757,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(tempty_bar(a), 2 * kEpiWarps);
     }
     mbar_init(drain_bar, 1);
-    for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(bar0 + 8u * (G::kResBar0 + i), 1);
+    for (int i = 0; i < G::kStoreBufs * kEpiWarps; ++i) mbar_init(bar0 + 8u * (G::kResBar0 + i), 1);
     mbar_init(bar0 + 8u * G::kLnBar0, kEpiWarps);
     for (int i = 1; i <= 2; ++i) mbar_init(bar0 + 8u * (G::kLnBar0 + i), CL > 2 ? CL / 2 - 1 : 1);
     fence_barrier_init();
@@ -890,9 +859,9 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
     float* bias_s = bias_smem + (warp - 2) * kCols;
     const CUtensorMap* tmc = (use_tma_store & 1) ? &tm_c : nullptr;
     EpiWarpState ws;
-    ws.stage = store_smem + (warp - 2) * 2 * kStageChunkBytes;
+    ws.stage = store_smem + (warp - 2) * G::kStoreBufs * kStageChunkBytes;
     ws.tm_r = (use_tma_store & 2) ? &tm_r : nullptr;     // residual through TMA (kBiasResidStore)
-    ws.res_bar = bar0 + 8u * (G::kResBar0 + 2 * (warp - 2));
+    ws.res_bar = bar0 + 8u * (G::kResBar0 + G::kStoreBufs * (warp - 2));
     const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), lead);
     const uint32_t leader_tempty1 = mapa_shared(tempty_bar(1), lead);
     LnCtx ln;
@@ -918,8 +887,8 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
         got = epilogue_ln_tile(t_cols, row0, n_blk * BN + slice * kCols, N, bias, ln_gamma, ln_beta, par_s, tmc,
                                ws, ln, slice, quad * 32 + lane, warp == 2, local, wait_full, release);
       else
-        got = epilogue_warp_tile<EPI, kChunks>(t_cols, row0, n_blk * BN + slice * kCols, M, N, bias, bias_s, C, sp,
-                                              tmc, ws, resid, wait_full, release);
+        got = epilogue_warp_tile<EPI, kChunks, G::kStoreBufs>(t_cols, row0, n_blk * BN + slice * kCols, M, N, bias,
+                                                              bias_s, C, sp, tmc, ws, resid, wait_full, release);
       if (!got) { ok = false; break; }
     }
     if (lane == 0) bulk_wait_group_all();      // every TMA store of this warp has completed
@@ -944,7 +913,7 @@ int store_flags(const TcGemmArgs& a) { return (a.tmap_c ? 1 : 0) | (a.tmap_c && 
 // grid larger than that would run its last clusters as a second wave).
 template <Epi EPI, int CL>
 int pair_max_clusters(cudaError_t& err) {
-  using G = PairCfg;
+  using G = PairCfgT<EPI>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;
@@ -971,7 +940,7 @@ int pair_max_clusters(cudaError_t& err) {
 
 template <Epi EPI, int CL>
 cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
-  using G = PairCfg;
+  using G = PairCfgT<EPI>;
   cudaError_t err;
   const int max_clusters = pair_max_clusters<EPI, CL>(err);
   if (err != cudaSuccess) return err;
@@ -1037,12 +1006,12 @@ __device__ __forceinline__ void epilogue4(float (&v)[4], const float* __restrict
     v[0] += lo.x; v[1] += lo.y; v[2] += hi.x; v[3] += hi.y;
   }
   if constexpr (EPI == Epi::kBiasGelu) {
-    gelu_erf_pair(v[0], v[1]);
-    gelu_erf_pair(v[2], v[3]);
+    act::gelu_erf_pair(v[0], v[1]);
+    act::gelu_erf_pair(v[2], v[3]);
   }
   if constexpr (EPI == Epi::kBiasGeluTanh) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = gelu_tanh(v[i]);
+    for (int i = 0; i < 4; ++i) v[i] = act::gelu_tanh(v[i]);
   }
 }
 

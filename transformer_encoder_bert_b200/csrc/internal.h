@@ -160,6 +160,42 @@ cudaError_t launch_layernorm_f16h(const __half* z, const __half* gamma, const __
 cudaError_t launch_layernorm_f32(const float* z, const float* gamma, const float* beta, float* out, int rows,
                                  int hidden, cudaStream_t stream);
 
+// ---- single-launch forward for small batches, persistent.cu ----
+constexpr int kPersistMaxTokens = 256;   // batch * seq
+constexpr int kPersistMaxSplits = 4;     // K splits of FFN2
+// One layer's parameters as the handle stores them: FP16 weights transposed to
+// [out, in] (K-major), FP32 biases and LayerNorm parameters.
+struct PersistLayer {
+  const __half *w_qkv, *w_o, *w_ff1, *w_ff2;
+  const float *b_qkv, *b_o, *b_ff1, *b_ff2, *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+};
+struct PersistArgs {
+  // A operands, FP16 [M, K] with a box of 64 columns x 16 ceil(M / 16) rows and
+  // 128-byte swizzle: x, z2, ctx, z1 ([M, H]) and u ([M, F]).
+  alignas(64) CUtensorMap amap[5];
+  const CUtensorMap* wmaps;     // device [L][4]: Wqkv^T, Wo^T, W1^T, W2^T ([N, K], box 64 x 32, 128-byte swizzle)
+  const PersistLayer* layers;   // device array [L]
+  int L;
+  const __half* x;              // [B*S, H]
+  const int32_t* valid_len;     // [B]
+  __half* out;                  // [B*S, H]
+  int B, S, NH, D, F;
+  // Workspace [B*S, ...]: qkv [M, 3H] (Q | K | V per token), ctx, z1, h1 [M, H],
+  // u [M, F], z2 [M, H], xl [M, H] (the LayerNorm-2 output of the previous layer).
+  __half *qkv, *ctx, *z1, *h1, *u, *z2, *xl;
+  float* partial;               // FFN2 split-K partial tiles, FP32 [splits][M][H]
+  unsigned* tile_cnt;           // FFN2 per-tile counters [H / 32]
+  int gelu_tanh;
+  unsigned* bar;                // 4 words, zero between launches: arrivals, epoch, exits, a flag never set
+  int* status;
+  unsigned long long wait_ns;   // limit of every wait
+  int stall_test;               // failure-detection test: CTA 0 never joins the first barrier
+};
+bool persistent_supported(int B, int S, int NH, int D, int F, int num_sms);
+// Device bytes of the FFN2 partial tiles and tile counters for hidden size H.
+size_t persistent_partial_bytes(int H, int F);
+cudaError_t launch_persistent(const PersistArgs& args, cudaStream_t stream);
+
 // ---- weight repack, encoder.cu ----
 int device_sm_count();
 

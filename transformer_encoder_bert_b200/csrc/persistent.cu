@@ -1,0 +1,854 @@
+// Single-launch forward of the whole encoder stack for small batches.
+//
+// The source page ("Faster Transformer 优化原理") notes that at small batch
+// sizes, such as question answering with one sequence, the cost of a layer is
+// its kernel launches rather than its arithmetic.  With a handful of tokens
+// every GEMM is a weight stream (BERT-Base: 14.2 MB per layer), and a layer of
+// separate kernels spends most of its time in launch, ramp-up and drain.  Here
+// one persistent kernel runs every layer:
+//   - one CTA per SM (cooperative launch: all CTAs are resident at once), 8
+//     warps;
+//   - per layer five phases separated by a grid-wide barrier:
+//       QKV    qkv = A Wqkv + bqkv               (A = x, or LN2 of the previous
+//                                                layer's z2, normalised on load)
+//       ATTN   ctx = softmax(Q K^T / sqrt(d), keys j < n) V
+//       OPROJ  z1 = ctx Wo + bo + x_l
+//       FFN1   u = GELU(LN1(z1) W1 + b1)       (LN1 normalised on load)
+//       FFN2   z2 = u W2 + b2 + h1,  h1 = LN1(z1)
+//     and after the last layer, out = LN2(z2);
+//   - a GEMM phase is split into units of NU = 8, 16 or 32 output features
+//     over the whole K, at most one unit of a phase per CTA.  A unit's weight
+//     tile (NU rows of the [N, K] weight, one contiguous block) is brought into
+//     shared memory by bulk copies; every weight is read from HBM once per
+//     forward, and the tile of a CTA's next unit is loaded while it works on
+//     the current one (weights do not depend on the activations), so the
+//     weight stream overlaps the phases and barriers;
+//   - the MMAs are mma.sync m16n8k16 (FP16 in, FP32 accumulate): with at most
+//     256 tokens a unit is a thin GEMM whose time is its operand traffic, and
+//     the register-level MMA needs no tensor-memory set-up per unit;
+//   - the LayerNorms run where their output is consumed: each FFN1 unit takes
+//     the row statistics of z1 and normalises its A operand as it loads it
+//     (and writes its share of the rows of h1 for the FFN2 residual); each
+//     QKV unit does the same with z2 (and writes its share of x_l for the
+//     output-projection residual).  LayerNorm statistics and normalisation
+//     are the same FP32 arithmetic as the LayerNorm kernels, rounded to FP16
+//     at the same points, so the results match the per-kernel forward up to
+//     the order of the FP32 accumulation.
+// Every wait (grid barrier, weight tile) is bounded in time; a wait that
+// gives up writes kStatusWaitTimeout to the status word and the CTA leaves
+// after its copies in flight have landed.
+#include <mutex>
+
+#include "gelu.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace enc {
+namespace {
+
+using namespace sm100;
+
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kNU = 32;                          // output features per GEMM unit (four n8 tiles)
+constexpr int kMaxKU = 1024;                     // K columns per unit
+// Shared memory (offsets from a 1024-byte-aligned base; TMA's 128-byte swizzle
+// repeats every 1024 bytes).  A weight tile is KU / 64 boxes of 32 rows x 64
+// columns (4 KB each); an A chunk is boxes of 16 mt rows x 64 columns.
+constexpr int kBoxBytes = kNU * 128;
+constexpr int kSlotBytes = (kMaxKU / 64) * kBoxBytes;      // 64 KB
+constexpr int kStageOffset = 2 * kSlotBytes;
+constexpr int kStageBytes = 64 * 1024;           // A chunk of a unit, or K and V of one (sequence, head)
+constexpr int kScratchOffset = kStageOffset + kStageBytes;
+constexpr int kScratchBytes = kWarps * 16 * kNU * 4;   // k-split partial tiles; gamma and beta before them
+constexpr int kStatsOffset = kScratchOffset + kScratchBytes;
+constexpr int kBarOffset = kStatsOffset + kPersistMaxTokens * 8;
+constexpr int kSmem = 1024 + kBarOffset + 64;
+static_assert(kSmem + 5 * 1024 <= 227 * 1024, "one CTA's shared memory");
+
+enum Phase { kQkv = 0, kOproj = 1, kFfn1 = 2, kFfn2 = 3, kNumGemm = 4 };
+enum AMap { kAx = 0, kAz2 = 1, kActx = 2, kAz1 = 3, kAu = 4 };   // PersistArgs::amap
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// Grid-wide barrier over a monotone arrival count: the e-th barrier of a
+// launch completes when the count reaches e * nblocks; its last arriver
+// publishes e (release), the others wait for it (acquire), for at most
+// limit_ns.  Returns false, uniformly across the CTA, when the wait gave up.
+// Data written before the barrier by other SMs is read after it only through
+// L2 (bulk copies, or loads that bypass L1), never from a stale L1 line.
+__device__ bool grid_sync(unsigned* bar, unsigned nblocks, unsigned& epoch, uint64_t limit_ns, int* flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ++epoch;
+    int ok = 1;
+    __threadfence();
+    const unsigned prev = atomicAdd(bar, 1u);
+    if (prev + 1 == epoch * nblocks) {
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(bar + 1), "r"(epoch) : "memory");
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      for (uint32_t i = 1;; ++i) {
+        unsigned g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(bar + 1) : "memory");
+        if (static_cast<int>(g - epoch) >= 0) break;
+        if ((i & 31u) == 0u && globaltimer_ns() - t0 > limit_ns) {
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    *flag = ok;
+  }
+  __syncthreads();
+  return *flag != 0;
+}
+
+// K splits of FFN2 (K = F): the fewest whose K range is a multiple of 64 of at
+// most kMaxKU columns (0: none).
+__host__ __device__ inline int ffn2_splits(int F) {
+  for (int s = 1; s <= 8; ++s)
+    if (F % s == 0 && (F / s) % 64 == 0 && F / s <= kMaxKU) return s;
+  return 0;
+}
+
+// Columns of A staged per chunk for mt 16-row tiles: whole 64-column boxes of
+// 16 mt rows that fit the staging area.
+__device__ __forceinline__ int chunk_cols(int mt) {
+  return (kStageBytes / (16 * mt * 128)) * 64;
+}
+
+struct Ctx {
+  const PersistArgs* a;
+  uint8_t* smem;
+  uint32_t sbase;
+  int M;                  // tokens
+  int G;                  // CTAs
+  int nsplit[kNumGemm];   // K splits
+  int KU[kNumGemm];       // K columns of a unit
+  int K[kNumGemm];        // K of the GEMM
+  int nunits[kNumGemm];   // (N / 32) * nsplit
+  int off[kNumGemm];      // CTA of unit 0 of the phase
+  int mine[kNumGemm];     // this CTA's unit of the phase, or -1
+  int order[kNumGemm];    // this CTA's phases with a unit, in phase order
+  int cnt;                // units of this CTA per layer
+  uint32_t a_phase;       // A-chunk loads so far (parity of the staging barrier)
+};
+
+__device__ __forceinline__ const __half* weight_of(const PersistLayer& L, int p) {
+  return p == kQkv ? L.w_qkv : p == kOproj ? L.w_o : p == kFfn1 ? L.w_ff1 : L.w_ff2;
+}
+
+// Warp 0: the weight tile of this CTA's k-th unit of the forward into slot
+// k & 1: rows n0 .. n0 + 31 of the [N, K] weight, columns k0 .. k0 + KU - 1,
+// as KU / 64 TMA boxes (one per lane, 128-byte swizzle).
+__device__ void load_unit(const Ctx& c, int k) {
+  const int lane = threadIdx.x & 31;
+  const int layer = k / c.cnt;
+  const int p = c.order[k % c.cnt];
+  const int u = c.mine[p];
+  const int KU = c.KU[p];
+  const int n0 = (u / c.nsplit[p]) * kNU, k0 = (u % c.nsplit[p]) * KU;
+  const uint32_t slot = c.sbase + (k & 1) * kSlotBytes;
+  const uint32_t bar = c.sbase + kBarOffset + 8 * (k & 1);
+  if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(kNU * KU * 2));
+  __syncwarp();
+  if (lane < KU / 64) tma_load_2d(c.a->wmaps + layer * kNumGemm + p, slot + lane * kBoxBytes, bar, k0 + lane * 64, n0);
+}
+
+// Row statistics (mean, rstd) of the M rows of z (FP16, [M, H]) into shared
+// memory: warp w takes rows w, w + 8, ..., four rows' loads in flight at once;
+// two passes over the row in registers (mean, then the variance of the
+// deviations), FP32, as the LayerNorm kernels.  Rows r with r % nwrite ==
+// wpart are also written normalised to dst (the unit's share of the
+// materialised LayerNorm output).
+__device__ __noinline__ void ln_stats(const Ctx& c, const __half* __restrict__ z, int H, const float* __restrict__ g,
+                                      const float* __restrict__ b, __half* __restrict__ dst, int nwrite, int wpart) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float2* stats = reinterpret_cast<float2*>(c.smem + kStatsOffset);
+  const int nvec = H / 8;
+  constexpr int RB = 4;
+  for (int rb = warp; rb < c.M; rb += RB * kWarps) {
+    uint4 v[RB][4];
+#pragma unroll
+    for (int q = 0; q < RB; ++q) {
+      const int r = rb + q * kWarps;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = lane + 32 * i;
+        if (r < c.M && col < nvec) v[q][i] = __ldcg(reinterpret_cast<const uint4*>(z + (size_t)r * H + col * 8));
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < RB; ++q) {
+      const int r = rb + q * kWarps;
+      if (r >= c.M) break;
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (lane + 32 * i < nvec) {
+          const __half2* hh = reinterpret_cast<const __half2*>(&v[q][i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(hh[j]);
+            sum += f.x + f.y;
+          }
+        }
+      }
+      const float mean = warp_sum(sum) / (float)H;
+      float sq = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (lane + 32 * i < nvec) {
+          const __half2* hh = reinterpret_cast<const __half2*>(&v[q][i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(hh[j]);
+            const float d0 = f.x - mean, d1 = f.y - mean;
+            sq = fmaf(d0, d0, sq);
+            sq = fmaf(d1, d1, sq);
+          }
+        }
+      }
+      const float rstd = rsqrtf(warp_sum(sq) / (float)H + kLnEps);
+      if (lane == 0) stats[r] = make_float2(mean, rstd);
+      if (r % nwrite == wpart) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int col = lane + 32 * i;
+          if (col < nvec) {
+            const __half2* hh = reinterpret_cast<const __half2*>(&v[q][i]);
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __half22float2(hh[j]);
+              const int k = col * 8 + 2 * j;
+              o[j] = pack_h2(fmaf((f.x - mean) * rstd, g[k], b[k]), fmaf((f.y - mean) * rstd, g[k + 1], b[k + 1]));
+            }
+            *reinterpret_cast<uint4*>(dst + (size_t)r * H + col * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// A operand of a unit: the tensor map of an FP16 [M, K] matrix (box 64
+// columns x 16 ceil(M / 16) rows), optionally normalised once staged, with the
+// row statistics in shared memory and gamma, beta.
+struct AOp {
+  const CUtensorMap* map;
+  const float* g = nullptr;    // LayerNorm on load when non-null
+  const float* b = nullptr;
+};
+
+enum class UEpi { kBias, kBiasGelu, kBiasGeluTanh, kBiasResid, kPartial };
+
+// Byte offset of row r, column k (a multiple of 8) in a region of 64-column
+// boxes of `rows` rows with TMA's 128-byte swizzle (16-byte unit u of row r
+// stored at unit u ^ (r & 7)).
+__device__ __forceinline__ uint32_t swz(int r, int k, int rows) {
+  return (uint32_t)((k >> 6) * rows * 128 + r * 128 + ((((k >> 3) & 7) ^ (r & 7)) << 4));
+}
+
+// One GEMM unit: columns n0 .. n0 + 31 of epi(A[:, k0 .. k0 + KU) W[n0 ..
+// n0 + 31, k0 .. k0 + KU)^T), the weight tile in `slot`.  A is staged in
+// chunks of 64-column TMA boxes (one per lane of warp 0) and, for LayerNorm
+// on load, normalised there; the MMAs read both operands with ldmatrix.  Work
+// split: 16-row m-tiles; with fewer than 8 m-tiles the k-steps of a chunk are
+// split over the warps of an m-tile and the partial tiles are summed in warp
+// order through shared memory (a fixed order: the result does not depend on
+// timing).  The bias and residual of the epilogue are requested before the
+// first chunk.  kPartial writes the FP32 sum (no bias) to `partial` for a
+// later cross-unit reduction.  Returns false when a wait gave up (uniformly
+// across the CTA).
+__device__ __noinline__ bool gemm_unit(Ctx& c, const AOp& A, int k0, int KU, uint32_t slot, int n0, int ldo,
+                                       UEpi epi, const float* __restrict__ bias, const __half* __restrict__ resid,
+                                       __half* __restrict__ out, float* __restrict__ partial, uint64_t wait_ns,
+                                       int* flag) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, cq = lane & 3;
+  const int M = c.M;
+  const int mt = (M + 15) >> 4;
+  const int rows = 16 * mt;                      // rows of an A box
+  const int ksplit = mt >= kWarps ? 1 : kWarps / mt;
+  const float2* stats = reinterpret_cast<const float2*>(c.smem + kStatsOffset);
+  const int nch = (KU + chunk_cols(mt) - 1) / chunk_cols(mt);     // equal chunks of whole boxes
+  const int KC = ((KU / 64 + nch - 1) / nch) * 64;
+  uint8_t* stage = c.smem + kStageOffset;
+  const uint32_t sstage = c.sbase + kStageOffset;
+  const uint32_t abar = c.sbase + kBarOffset + 16;
+  float* gs = reinterpret_cast<float*>(c.smem + kScratchOffset);      // gamma, then beta (LayerNorm on load)
+  const int Kfull = c.K[0];                      // = H: gamma and beta have H entries
+  if (A.g) {
+    for (int i = threadIdx.x; i < Kfull; i += kThreads) {
+      gs[i] = A.g[i];
+      gs[Kfull + i] = A.b[i];
+    }
+  }
+  float acc[2][4][4];
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[t][j][e] = 0.f;
+  int mtile[2] = {-1, -1};
+  int kpart = 0;
+  if (ksplit == 1) {
+    mtile[0] = warp < mt ? warp : -1;
+    mtile[1] = warp + kWarps < mt ? warp + kWarps : -1;
+  } else {
+    kpart = warp % ksplit;
+    mtile[0] = warp / ksplit < mt ? warp / ksplit : -1;
+  }
+  // Epilogue operands, requested now: bias of the thread's 8 columns and the
+  // residual of its (up to) 16 output pairs.
+  float bv[4][2];
+  uint32_t rv[2][4][2];
+  if (epi != UEpi::kPartial) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + j * 8 + 2 * cq;
+      bv[j][0] = bias[n];
+      bv[j][1] = bias[n + 1];
+    }
+  }
+  if (epi == UEpi::kBiasResid) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int row = (mtile[t] < 0 ? 0 : mtile[t] * 16) + g + 8 * hr;
+          const int n = n0 + j * 8 + 2 * cq;
+          rv[t][j][hr] = (mtile[t] >= 0 && row < M)
+                             ? __ldcg(reinterpret_cast<const unsigned int*>(resid + (size_t)row * ldo + n))
+                             : 0u;
+        }
+  }
+
+  for (int c0 = 0; c0 < KU; c0 += KC) {
+    const int kcc = min(KC, KU - c0);
+    const int nbox = kcc / 64;
+    if (warp == 0) {
+      if (lane == 0) mbar_arrive_expect_tx(abar, (uint32_t)(nbox * rows * 128));
+      __syncwarp();
+      if (lane < nbox) tma_load_2d(A.map, sstage + lane * rows * 128, abar, k0 + c0 + lane * 64, 0);
+      if (lane == 0) flag[0] = mbar_wait(abar, c.a_phase & 1u, wait_ns) ? 1 : 0;
+    }
+    ++c.a_phase;
+    __syncthreads();
+    if (!flag[0]) return false;
+    if (A.g) {                                   // LayerNorm on load, in place: (z - mean) * rstd * gamma + beta
+      for (int i = threadIdx.x; i < nbox * M * 8; i += kThreads) {
+        const int bx = i / (M * 8), rem = i - bx * (M * 8);
+        const int r = rem >> 3, pu = rem & 7;    // physical 16-byte unit of row r
+        const int col = k0 + c0 + bx * 64 + ((pu ^ (r & 7)) << 3);
+        uint4* pv = reinterpret_cast<uint4*>(stage + bx * rows * 128 + r * 128 + pu * 16);
+        const uint4 raw = *pv;
+        const __half2* hh = reinterpret_cast<const __half2*>(&raw);
+        const float2 st = stats[r];
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __half22float2(hh[j]);
+          o[j] = pack_h2(fmaf((f.x - st.x) * st.y, gs[col + 2 * j], gs[Kfull + col + 2 * j]),
+                         fmaf((f.y - st.x) * st.y, gs[col + 2 * j + 1], gs[Kfull + col + 2 * j + 1]));
+        }
+        *pv = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      __syncthreads();
+    }
+    const int nks = kcc >> 4;
+    const int ks0 = ksplit > 1 ? kpart * nks / ksplit : 0;
+    const int ks1 = ksplit > 1 ? (kpart + 1) * nks / ksplit : nks;
+    if (mtile[0] >= 0) {
+      for (int ks = ks0; ks < ks1; ++ks) {
+        const int kl = ks * 16;                  // column within the chunk
+        uint32_t bf[4][2];
+#pragma unroll
+        for (int jp = 0; jp < 2; ++jp) {         // n8 tiles 2jp, 2jp + 1
+          const int row = jp * 16 + (lane >> 4) * 8 + (lane & 7);
+          ldsm_x4(slot + swz(row, c0 + kl + 8 * ((lane >> 3) & 1), kNU), bf[2 * jp][0], bf[2 * jp][1],
+                  bf[2 * jp + 1][0], bf[2 * jp + 1][1]);
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (mtile[t] < 0) continue;
+          const int arow = mtile[t] * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+          uint32_t af[4];
+          ldsm_x4(sstage + swz(arow, kl + 8 * (lane >> 4), rows), af[0], af[1], af[2], af[3]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma16816(acc[t][j], af, bf[j][0], bf[j][1]);
+        }
+      }
+    }
+    __syncthreads();                             // the chunk has been read before the next one lands
+  }
+
+  if (ksplit > 1) {
+    float* scratch = reinterpret_cast<float*>(c.smem + kScratchOffset);
+    if (mtile[0] >= 0 && kpart > 0) {
+      float* dst = scratch + (size_t)warp * (16 * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[(j * 4 + e) * 32 + lane] = acc[0][j][e];
+    }
+    __syncthreads();
+    if (mtile[0] >= 0 && kpart == 0) {
+      for (int q = 1; q < ksplit; ++q) {
+        const float* src = scratch + (size_t)(warp + q) * (16 * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[0][j][e] += src[(j * 4 + e) * 32 + lane];
+      }
+    } else {
+      mtile[0] = -1;                             // partial already handed over
+    }
+    __syncthreads();                             // scratch is free for the next unit
+  }
+
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (mtile[t] < 0) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + j * 8 + 2 * cq;
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = mtile[t] * 16 + g + 8 * hr;
+        if (row >= M) continue;
+        float v0 = acc[t][j][2 * hr], v1 = acc[t][j][2 * hr + 1];
+        if (epi == UEpi::kPartial) {
+          *reinterpret_cast<float2*>(partial + (size_t)row * ldo + n) = make_float2(v0, v1);
+          continue;
+        }
+        v0 += bv[j][0];
+        v1 += bv[j][1];
+        if (epi == UEpi::kBiasGelu) {
+          act::gelu_erf_pair(v0, v1);
+        } else if (epi == UEpi::kBiasGeluTanh) {
+          v0 = act::gelu_tanh(v0);
+          v1 = act::gelu_tanh(v1);
+        } else if (epi == UEpi::kBiasResid) {
+          const float2 rf = __half22float2(*reinterpret_cast<const __half2*>(&rv[t][j][hr]));
+          v0 += rf.x;
+          v1 += rf.y;
+        }
+        *reinterpret_cast<uint32_t*>(out + (size_t)row * ldo + n) = pack_h2(v0, v1);
+      }
+    }
+  }
+  return true;
+}
+
+template <int DL>   // head dimensions per lane: d / 32
+__device__ __noinline__ void attention_phase(const PersistArgs& a, uint8_t* kv_smem, float* qs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int d = 32 * DL;
+  constexpr int kRowB = 2 * d + 16;             // staged row (bytes)
+  const int H = a.NH * d;
+  const int ld = 3 * H;
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+  const int nblk = (a.S + 7) / 8;
+  const int items = a.B * a.NH * nblk;
+  uint8_t* ks = kv_smem;
+  uint8_t* vs = kv_smem + (size_t)a.S * kRowB;
+  float* q = qs + warp * d;
+  for (int it = blockIdx.x; it < items; it += gridDim.x) {
+    const int blk = it % nblk;
+    const int h = (it / nblk) % a.NH;
+    const int b = it / (nblk * a.NH);
+    int n = a.valid_len[b];
+    n = n < 0 ? 0 : (n > a.S ? a.S : n);
+    const __half* kbase = a.qkv + (size_t)b * a.S * ld + H + h * d;
+    const __half* vbase = kbase + H;
+    // Stage K and V of the n valid keys: 16-byte pieces, all requested at once.
+    const int pieces = n * (d / 8);
+    __syncthreads();                            // the previous item's rows have been read
+    for (int pc = threadIdx.x; pc < 2 * pieces; pc += kThreads) {
+      const int which = pc >= pieces;           // 0: K, 1: V
+      const int idx = pc - which * pieces;
+      const int j = idx / (d / 8), u = idx % (d / 8);
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>((which ? vbase : kbase) + (size_t)j * ld + u * 8));
+      *reinterpret_cast<uint4*>((which ? vs : ks) + j * kRowB + u * 16) = v;
+    }
+    __syncthreads();
+    const int i = blk * 8 + warp;
+    if (i >= a.S) continue;
+    const int row = b * a.S + i;
+    __half* dst = a.ctx + (size_t)row * H + h * d;
+    if (n == 0) {
+#pragma unroll
+      for (int t = 0; t < DL; ++t) dst[lane + 32 * t] = __float2half(0.f);
+      continue;
+    }
+    const __half* qrow = a.qkv + (size_t)row * ld + h * d;
+#pragma unroll
+    for (int t = 0; t < DL; ++t) q[lane + 32 * t] = __half2float(__ldcg(qrow + lane + 32 * t));
+    __syncwarp();
+    float m = -INFINITY, l = 0.f;
+    float o[DL];
+#pragma unroll
+    for (int t = 0; t < DL; ++t) o[t] = 0.f;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      float s = -INFINITY;
+      if (j < n) {
+        const uint4* kr = reinterpret_cast<const uint4*>(ks + j * kRowB);
+        float acc = 0.f;
+#pragma unroll
+        for (int v = 0; v < DL * 4; ++v) {
+          const uint4 u = kr[v];
+          const __half2* hh = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hh[e]);
+            acc = fmaf(q[8 * v + 2 * e], f.x, acc);
+            acc = fmaf(q[8 * v + 2 * e + 1], f.y, acc);
+          }
+        }
+        s = acc * scale_log2;                    // log2 domain
+      }
+      const float bm = warp_max(s);
+      const float m_new = fmaxf(m, bm);
+      const float alpha = exp2f(m - m_new);      // 0 on the first block (m = -inf)
+      const float p = j < n ? exp2f(s - m_new) : 0.f;
+      l = l * alpha + warp_sum(p);
+#pragma unroll
+      for (int t = 0; t < DL; ++t) o[t] *= alpha;
+      const int jn = min(32, n - j0);
+      for (int jj = 0; jj < jn; ++jj) {
+        const float pj = __shfl_sync(0xffffffffu, p, jj);
+        const __half* vr = reinterpret_cast<const __half*>(vs + (j0 + jj) * kRowB);
+#pragma unroll
+        for (int t = 0; t < DL; ++t) o[t] = fmaf(pj, __half2float(vr[lane + 32 * t]), o[t]);
+      }
+      m = m_new;
+    }
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int t = 0; t < DL; ++t) dst[lane + 32 * t] = __float2half(o[t] * inv);
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) encoder_persistent_kernel(const __grid_constant__ PersistArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ int flag[2];
+  __shared__ float qs[kWarps * 128];
+  Ctx c;
+  c.a = &a;
+  c.smem = smem;
+  c.sbase = smem_u32(smem);
+  c.M = a.B * a.S;
+  c.G = gridDim.x;
+  c.a_phase = 0;
+  const int H = a.NH * a.D;
+  const int Ks[kNumGemm] = {H, H, H, a.F};
+  const int Ns[kNumGemm] = {3 * H, H, a.F, H};
+  int total = 0;
+  c.cnt = 0;
+  for (int p = 0; p < kNumGemm; ++p) {
+    c.K[p] = Ks[p];
+    c.nsplit[p] = p == kFfn2 ? ffn2_splits(a.F) : 1;
+    c.KU[p] = Ks[p] / c.nsplit[p];
+    c.nunits[p] = (Ns[p] / kNU) * c.nsplit[p];
+    c.off[p] = total % c.G;
+    total += c.nunits[p];
+    const int u = ((int)blockIdx.x - c.off[p] + c.G) % c.G;
+    c.mine[p] = u < c.nunits[p] ? u : -1;
+    if (c.mine[p] >= 0) c.order[c.cnt++] = p;
+  }
+  const int units_total = c.cnt * a.L;
+  const uint32_t bar0 = c.sbase + kBarOffset;   // weight slot barriers [2], A staging barrier
+  unsigned epoch = 0;
+  bool ok = true;
+  const unsigned nblocks = gridDim.x;
+  unsigned* gbar = a.bar;                       // [0] arrivals, [1] published epoch, [2] exits, [3] never set
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    mbar_init(bar0 + 16, 1);
+    fence_barrier_init();
+  }
+  if (blockIdx.x == 0)                          // FFN2 tile counters: first used after four barriers
+    for (int i = threadIdx.x; i < H / kNU; i += kThreads) a.tile_cnt[i] = 0u;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    for (int k = 0; k < 2 && k < units_total; ++k) load_unit(c, k);
+  }
+
+  if (a.stall_test && blockIdx.x == 0) {
+    // Failure-detection test: this CTA waits on a flag that nothing sets
+    // instead of joining the first barrier; every other CTA's barrier wait then
+    // runs out, and this one's too.
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (*reinterpret_cast<volatile unsigned*>(gbar + 3) == 0u && globaltimer_ns() - t0 < a.wait_ns)
+        __nanosleep(1000);
+    }
+    ok = false;
+  }
+
+  int k = 0;                                    // this CTA's units so far
+  auto unit_begin = [&]() -> uint32_t {         // wait for the unit's weight tile
+    if (threadIdx.x == 0) flag[0] = mbar_wait(bar0 + 8 * (k & 1), (uint32_t)(k >> 1) & 1u, a.wait_ns) ? 1 : 0;
+    __syncthreads();
+    const bool r = flag[0] != 0;
+    __syncthreads();
+    return r ? c.sbase + (k & 1) * kSlotBytes : 0u;
+  };
+  auto unit_end = [&]() {                       // the slot is read: refill it with unit k + 2
+    __syncthreads();
+    if (threadIdx.x < 32 && k + 2 < units_total) load_unit(c, k + 2);
+    ++k;
+  };
+  auto run = [&](int p, const AOp& A, int ldo, UEpi epi, const float* bias, const __half* resid, __half* out,
+                 float* partial) -> bool {
+    const uint32_t slot = unit_begin();
+    if (!slot) return false;
+    const int u = c.mine[p];
+    const bool r = gemm_unit(c, A, (u % c.nsplit[p]) * c.KU[p], c.KU[p], slot, (u / c.nsplit[p]) * kNU, ldo, epi,
+                             bias, resid, out, partial, a.wait_ns, flag);
+    if (!r) return false;
+    unit_end();
+    return true;
+  };
+
+  for (int l = 0; l < a.L && ok; ++l) {
+    const PersistLayer& L = a.layers[l];
+    const PersistLayer* Lp = l > 0 ? &a.layers[l - 1] : nullptr;
+    // ---- QKV: qkv = A Wqkv + bqkv, A = x or LN2(z2) of the previous layer
+    if (c.mine[kQkv] >= 0) {
+      AOp A;
+      A.map = &a.amap[l == 0 ? kAx : kAz2];
+      if (l > 0) {
+        ln_stats(c, a.z2, H, Lp->ln2_g, Lp->ln2_b, a.xl, c.nunits[kQkv], c.mine[kQkv]);
+        A.g = Lp->ln2_g;
+        A.b = Lp->ln2_b;
+      }
+      if (!(ok = run(kQkv, A, 3 * H, UEpi::kBias, L.b_qkv, nullptr, a.qkv, nullptr))) break;
+    }
+    if (!(ok = grid_sync(gbar, nblocks, epoch, a.wait_ns, flag))) break;
+    // ---- ATTN (K and V of one (sequence, head) in the staging area)
+    if (a.D == 32)
+      attention_phase<1>(a, smem + kStageOffset, qs);
+    else if (a.D == 64)
+      attention_phase<2>(a, smem + kStageOffset, qs);
+    else
+      attention_phase<4>(a, smem + kStageOffset, qs);
+    if (!(ok = grid_sync(gbar, nblocks, epoch, a.wait_ns, flag))) break;
+    // ---- OPROJ: z1 = ctx Wo + bo + x_l
+    if (c.mine[kOproj] >= 0) {
+      AOp A;
+      A.map = &a.amap[kActx];
+      if (!(ok = run(kOproj, A, H, UEpi::kBiasResid, L.b_o, l == 0 ? a.x : a.xl, a.z1, nullptr))) break;
+    }
+    if (!(ok = grid_sync(gbar, nblocks, epoch, a.wait_ns, flag))) break;
+    // ---- FFN1: u = GELU(LN1(z1) W1 + b1); this unit's share of the rows of h1
+    if (c.mine[kFfn1] >= 0) {
+      ln_stats(c, a.z1, H, L.ln1_g, L.ln1_b, a.h1, c.nunits[kFfn1], c.mine[kFfn1]);
+      AOp A;
+      A.map = &a.amap[kAz1];
+      A.g = L.ln1_g;
+      A.b = L.ln1_b;
+      if (!(ok = run(kFfn1, A, a.F, a.gelu_tanh ? UEpi::kBiasGeluTanh : UEpi::kBiasGelu, L.b_ff1, nullptr, a.u,
+                     nullptr)))
+        break;
+    }
+    if (!(ok = grid_sync(gbar, nblocks, epoch, a.wait_ns, flag))) break;
+    // ---- FFN2, split over K: each unit writes its FP32 partial tile; the last
+    // of an N tile's units to finish sums the partials in split order (fixed,
+    // so the result does not depend on which unit finishes last) and writes
+    // z2 = sum + b2 + h1.
+    if (c.mine[kFfn2] >= 0) {
+      const int u = c.mine[kFfn2];
+      const int ns = c.nsplit[kFfn2];
+      const int tile = u / ns, q = u % ns;
+      AOp A;
+      A.map = &a.amap[kAu];
+      if (!(ok = run(kFfn2, A, H, UEpi::kPartial, nullptr, nullptr, nullptr, a.partial + (size_t)q * c.M * H)))
+        break;
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const unsigned prev = atomicAdd(a.tile_cnt + tile, 1u);
+        flag[1] = prev + 1 == (unsigned)ns;
+        if (flag[1]) {
+          __threadfence();
+          a.tile_cnt[tile] = 0u;                 // ready for the next layer
+        }
+      }
+      __syncthreads();
+      if (flag[1]) {
+        const int n0 = tile * kNU;
+        for (int i = threadIdx.x; i < c.M * (kNU / 2); i += kThreads) {
+          const int row = i / (kNU / 2), n = n0 + 2 * (i % (kNU / 2));
+          float v0 = L.b_ff2[n], v1 = L.b_ff2[n + 1];
+          for (int qq = 0; qq < ns; ++qq) {
+            const float2 pv = __ldcg(reinterpret_cast<const float2*>(a.partial + ((size_t)qq * c.M + row) * H + n));
+            v0 += pv.x;
+            v1 += pv.y;
+          }
+          const uint32_t rr = __ldcg(reinterpret_cast<const unsigned int*>(a.h1 + (size_t)row * H + n));
+          const float2 rf = __half22float2(*reinterpret_cast<const __half2*>(&rr));
+          *reinterpret_cast<uint32_t*>(a.z2 + (size_t)row * H + n) = pack_h2(v0 + rf.x, v1 + rf.y);
+        }
+      }
+    }
+    if (!(ok = grid_sync(gbar, nblocks, epoch, a.wait_ns, flag))) break;
+  }
+
+  if (ok) {
+    // out = LN2(z2) of the last layer: one warp per row.
+    const PersistLayer& L = a.layers[a.L - 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nvec = H / 8;
+    for (int r = blockIdx.x * kWarps + warp; r < c.M; r += gridDim.x * kWarps) {
+      uint4 v[4];
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = lane + 32 * i;
+        if (col < nvec) {
+          v[i] = __ldcg(reinterpret_cast<const uint4*>(a.z2 + (size_t)r * H + col * 8));
+          const __half2* hh = reinterpret_cast<const __half2*>(&v[i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(hh[j]);
+            sum += f.x + f.y;
+          }
+        }
+      }
+      const float mean = warp_sum(sum) / (float)H;
+      float sq = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (lane + 32 * i < nvec) {
+          const __half2* hh = reinterpret_cast<const __half2*>(&v[i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(hh[j]);
+            const float d0 = f.x - mean, d1 = f.y - mean;
+            sq = fmaf(d0, d0, sq);
+            sq = fmaf(d1, d1, sq);
+          }
+        }
+      }
+      const float rstd = rsqrtf(warp_sum(sq) / (float)H + kLnEps);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = lane + 32 * i;
+        if (col < nvec) {
+          const __half2* hh = reinterpret_cast<const __half2*>(&v[i]);
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(hh[j]);
+            const int kk = col * 8 + 2 * j;
+            o[j] = pack_h2(fmaf((f.x - mean) * rstd, L.ln2_g[kk], L.ln2_b[kk]),
+                           fmaf((f.y - mean) * rstd, L.ln2_g[kk + 1], L.ln2_b[kk + 1]));
+          }
+          *reinterpret_cast<uint4*>(a.out + (size_t)r * H + col * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+  }
+
+  // Leave only after this CTA's copies in flight have landed; the last CTA out
+  // resets the barrier words for the next launch.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int kk = k; kk < k + 2 && kk < units_total; ++kk)
+      mbar_wait(bar0 + 8 * (kk & 1), (uint32_t)(kk >> 1) & 1u, a.wait_ns);
+    if (c.a_phase > 0) mbar_wait(bar0 + 16, (c.a_phase - 1) & 1u, a.wait_ns);
+    if (!ok) atomicCAS(a.status, 0, kStatusWaitTimeout);
+    __threadfence();
+    if (atomicAdd(gbar + 2, 1u) + 1 == nblocks) {
+      gbar[0] = 0u;
+      gbar[1] = 0u;
+      gbar[2] = 0u;
+      __threadfence();
+    }
+  }
+}
+
+}  // namespace
+
+bool persistent_supported(int B, int S, int NH, int D, int F, int num_sms) {
+  const int H = NH * D;
+  if (D != 32 && D != 64 && D != 128) return false;
+  if (H % 64 != 0 || F % 64 != 0 || H > kMaxKU) return false;
+  if ((long)B * S > kPersistMaxTokens) return false;
+  if (2 * S * (2 * D + 16) > kStageBytes) return false;   // K and V of one (sequence, head) in shared memory
+  const int s = ffn2_splits(F);
+  if (s == 0 || s > kPersistMaxSplits) return false;
+  // At most one unit of a phase per CTA.
+  if (3 * H / kNU > num_sms || F / kNU > num_sms || (H / kNU) * s > num_sms) return false;
+  return true;
+}
+
+size_t persistent_partial_bytes(int H, int F) {
+  return (size_t)kPersistMaxSplits * kPersistMaxTokens * H * sizeof(float) + (size_t)(H / kNU) * sizeof(unsigned);
+}
+
+cudaError_t launch_persistent(const PersistArgs& args, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(encoder_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  });
+  if (attr != cudaSuccess) return attr;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(device_sm_count());
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, encoder_persistent_kernel, args);
+}
+
+}  // namespace enc
