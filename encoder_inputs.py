@@ -169,3 +169,81 @@ def sample_sequences(batch: int, count: int, valid_len: np.ndarray, seed: int = 
     rest = [i for i in rng.permutation(batch).tolist() if i not in must]
     picked = sorted(must) + rest[: max(0, count - len(must))]
     return np.array(sorted(set(picked)), dtype=np.int64)
+
+
+# ------------------------------------------------------------------ decoder inputs
+DECODER_LAYER_KEYS = ("w_qkv", "b_qkv", "w_o", "b_o", "ln1_g", "ln1_b",
+                      "w_q2", "b_q2", "w_kv2", "b_kv2", "w_o2", "b_o2", "ln2_g", "ln2_b",
+                      "w_ff1", "b_ff1", "w_ff2", "b_ff2", "ln3_g", "ln3_b")
+
+
+@dataclass(frozen=True)
+class DecoderWorkload:
+    """One synthetic decoder workload: target tokens y [B, T, H] attending to a
+    memory (an encoder output) mem [B, S, H]."""
+    name: str
+    shape: EncoderShape
+    batch: int
+    tgt_seq: int
+    mem_seq: int
+    dtype: str
+    tgt_lo: int
+    tgt_hi: int
+    mem_lo: int
+    mem_hi: int
+    ln_affine_random: bool = False
+    seed: int = 0
+    weight_std: float = 0.02
+
+    def with_(self, **kw) -> "DecoderWorkload":
+        return replace(self, **kw)
+
+
+@dataclass
+class DecoderInputs:
+    workload: DecoderWorkload
+    y: np.ndarray                               # [B, T, H]
+    mem: np.ndarray                             # [B, S, H]
+    tgt_len: np.ndarray                         # [B] int32
+    mem_len: np.ndarray                         # [B] int32
+    layers: List[Dict[str, np.ndarray]] = field(default_factory=list)
+
+    def as_float64(self):
+        return (self.y.astype(np.float64), self.tgt_len.copy(), self.mem.astype(np.float64), self.mem_len.copy(),
+                [{k: v.astype(np.float64) for k, v in lw.items()} for lw in self.layers])
+
+
+def make_decoder_inputs(wl: DecoderWorkload) -> DecoderInputs:
+    """Draw order (PCG64, seed): y, mem, then per layer w_qkv, b_qkv, w_o, b_o,
+    w_q2, b_q2, w_kv2, b_kv2, w_o2, b_o2, w_ff1, b_ff1, w_ff2, b_ff2 (weights and
+    biases ~ N(0, weight_std)), then (ln_affine_random) gamma ~ N(1, 0.1) and
+    beta ~ N(0, 0.1) of LayerNorms 1, 2, 3 (else 1 and 0), then tgt_len ~
+    U{tgt_lo..tgt_hi} and mem_len ~ U{mem_lo..mem_hi}.  y, mem ~ N(0, 1)."""
+    dt = DTYPES[wl.dtype]
+    sh = wl.shape
+    H, F = sh.hidden, sh.ffn_dim
+    std = wl.weight_std
+    rng = np.random.Generator(np.random.PCG64(wl.seed))
+    y = rng.standard_normal((wl.batch, wl.tgt_seq, H)).astype(dt)
+    mem = rng.standard_normal((wl.batch, wl.mem_seq, H)).astype(dt)
+    layers = []
+    for _ in range(sh.num_layers):
+        lw = {}
+        for name, shp in (("w_qkv", (H, 3 * H)), ("b_qkv", (3 * H,)), ("w_o", (H, H)), ("b_o", (H,)),
+                          ("w_q2", (H, H)), ("b_q2", (H,)), ("w_kv2", (H, 2 * H)), ("b_kv2", (2 * H,)),
+                          ("w_o2", (H, H)), ("b_o2", (H,)), ("w_ff1", (H, F)), ("b_ff1", (F,)),
+                          ("w_ff2", (F, H)), ("b_ff2", (H,))):
+            lw[name] = rng.normal(0.0, std, shp).astype(dt)
+        for i in (1, 2, 3):
+            if wl.ln_affine_random:
+                lw[f"ln{i}_g"] = rng.normal(1.0, 0.1, H).astype(dt)
+                lw[f"ln{i}_b"] = rng.normal(0.0, 0.1, H).astype(dt)
+            else:
+                lw[f"ln{i}_g"] = np.ones(H, dt)
+                lw[f"ln{i}_b"] = np.zeros(H, dt)
+        layers.append(lw)
+    tlo = max(0, min(wl.tgt_lo, wl.tgt_seq)); thi = max(tlo, min(wl.tgt_hi, wl.tgt_seq))
+    mlo = max(0, min(wl.mem_lo, wl.mem_seq)); mhi = max(mlo, min(wl.mem_hi, wl.mem_seq))
+    tgt_len = rng.integers(tlo, thi + 1, size=wl.batch).astype(np.int32)
+    mem_len = rng.integers(mlo, mhi + 1, size=wl.batch).astype(np.int32)
+    return DecoderInputs(wl, np.ascontiguousarray(y), np.ascontiguousarray(mem), tgt_len, mem_len, layers)
