@@ -320,6 +320,63 @@ ENC_API uint64_t enc_launch_count(enc_t h);
 ENC_API enc_status enc_set_trace_events(enc_t h, void* const* events, int count);
 
 /* ------------------------------------------------------------------------------
+ * Decoder forward.  [FT] "什么是 Faster Transformer" says a decoder follows the
+ * encoder in a later release and gives no design.  The layer here is the
+ * post-LN Transformer decoder layer run over a whole target sequence (every
+ * target token at once), with the encoder's conventions (LN eps 1e-12,
+ * biased variance, scale 1/sqrt(d), masked keys weigh exactly 0, erf GELU
+ * unless enc_set_gelu chooses tanh):
+ *   QKV = y Wqkv + bqkv;  per head: A1 = softmax(Q K^T / sqrt(d)) V over keys
+ *     j <= i and j < nt = clamp(tgt_len[b], 0, T)  (causal self-attention);
+ *   H1 = LN1(y + A1 Wo + bo);
+ *   Q2 = H1 Wq2 + bq2,  [K2 | V2] = mem Wkv2 + bkv2;  A2 = softmax(Q2 K2^T /
+ *     sqrt(d)) V2 over memory keys j < nm = clamp(mem_len[b], 0, S);
+ *   H2 = LN2(H1 + A2 Wo2 + bo2);
+ *   out = LN3(H2 + GELU(H2 W1 + b1) W2 + b2).
+ * Every layer attends to the same memory (e.g. the encoder output).  A query
+ * row with no valid key gets a zero attention context.
+ * ---------------------------------------------------------------------------- */
+
+/* One decoder layer's parameters, IEEE half, matrices [in, out] row-major.
+ * Wqkv's columns are Q | K | V and Wkv2's are K | V, head h at columns
+ * h*d .. h*d+d-1 inside each block.  Host or device pointers, read only
+ * during enc_decoder_create. */
+typedef struct {
+  const void* w_qkv; const void* b_qkv;   /* [H, 3H], [3H]  self-attention */
+  const void* w_o;   const void* b_o;     /* [H, H],  [H]   */
+  const void* ln1_g; const void* ln1_b;   /* [H], [H] */
+  const void* w_q2;  const void* b_q2;    /* [H, H],  [H]   cross-attention query */
+  const void* w_kv2; const void* b_kv2;   /* [H, 2H], [2H]  cross-attention keys | values, from the memory */
+  const void* w_o2;  const void* b_o2;    /* [H, H],  [H]   */
+  const void* ln2_g; const void* ln2_b;   /* [H], [H] */
+  const void* w_ff1; const void* b_ff1;   /* [H, F],  [F]   */
+  const void* w_ff2; const void* b_ff2;   /* [F, H],  [H]   */
+  const void* ln3_g; const void* ln3_b;   /* [H], [H] */
+} enc_decoder_layer_weights;
+
+/* enc_decoder_create - a decoder handle (FP16 only: ENC_FP32 gives
+ * ENC_ERR_UNSUPPORTED; size_per_head in {32, 64, 128}, hidden size <= 1024,
+ * ffn_dim a multiple of 8).  Copies and repacks every parameter like
+ * enc_create; release it with enc_destroy.  Synchronous.  enc_set_gelu and
+ * enc_set_option apply to it; the encoder-only calls (enc_forward and the
+ * enc_op_* steps) return ENC_ERR_INVALID_ARG on it. */
+ENC_API enc_status enc_decoder_create(int head_num, int size_per_head, int ffn_dim, int num_layers,
+                                      enc_dtype dtype, const enc_decoder_layer_weights* weights, enc_t* out);
+
+/* enc_decoder_forward - the decoder stack on `stream`.
+ *   y:        device [batch, tgt_seq, H] target hidden states;
+ *   tgt_len:  device int32 [batch], clamped to [0, tgt_seq] on device;
+ *   mem:      device [batch, mem_seq, H] memory (e.g. the encoder output);
+ *   mem_len:  device int32 [batch], clamped to [0, mem_seq] on device;
+ *   out:      device [batch, tgt_seq, H]; must not overlap y.
+ * 16-byte-aligned buffers; the workspace grows like enc_forward's.  12 kernel
+ * launches per layer.  Asynchronous; host checks fail before anything is
+ * enqueued. */
+ENC_API enc_status enc_decoder_forward(enc_t h, const void* y, const int32_t* tgt_len, const void* mem,
+                                       const int32_t* mem_len, void* out, int batch, int tgt_seq, int mem_seq,
+                                       enc_stream_t stream);
+
+/* ------------------------------------------------------------------------------
  * Single steps of one layer, for checking each kernel alone.  Each runs exactly
  * the kernel enc_forward runs for that step, with layer `layer`'s parameters,
  * on caller-owned device buffers (same dtype as the handle, 16-byte aligned,

@@ -3,6 +3,6 @@
 The product is the C-ABI library lib/libbertenc.so (include/enc.h); this
 package builds it (``build``) and binds it (``Encoder``).
 """
-from .binding import Encoder, EncError, load_library, LIB_PATH  # noqa: F401
+from .binding import Decoder, Encoder, EncError, load_library, LIB_PATH  # noqa: F401
 
-__all__ = ["Encoder", "EncError", "load_library", "LIB_PATH"]
+__all__ = ["Decoder", "Encoder", "EncError", "load_library", "LIB_PATH"]

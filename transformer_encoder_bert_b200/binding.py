@@ -53,6 +53,8 @@ SIGNATURES = {
     "enc_kernels_per_forward": (_i, [_vp, _i, _i]),
     "enc_launch_count": (ctypes.c_uint64, [_vp]),
     "enc_set_trace_events": (_i, [_vp, _vp, _i]),
+    "enc_decoder_create": (_i, [_i, _i, _i, _i, _i, _vp, ctypes.POINTER(_vp)]),
+    "enc_decoder_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "enc_op_qkv": (_i, [_vp, _i, _vp, _vp, _i, _i, _vp]),
     "enc_op_attention": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "enc_op_out_proj_ln": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp]),
@@ -63,6 +65,15 @@ SIGNATURES = {
 
 class EncLayerWeights(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in WEIGHT_FIELDS]
+
+
+# Field order of enc_decoder_layer_weights.
+DECODER_WEIGHT_FIELDS = ("w_qkv", "b_qkv", "w_o", "b_o", "ln1_g", "ln1_b", "w_q2", "b_q2", "w_kv2", "b_kv2",
+                         "w_o2", "b_o2", "ln2_g", "ln2_b", "w_ff1", "b_ff1", "w_ff2", "b_ff2", "ln3_g", "ln3_b")
+
+
+class EncDecoderLayerWeights(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in DECODER_WEIGHT_FIELDS]
 
 
 class EncError(RuntimeError):
@@ -295,6 +306,60 @@ class Encoder:
         """out = LN2(u W2 + b2 + resid)."""
         _check(self.lib.enc_op_ffn2_ln(self.handle, layer, _dptr(u), _dptr(resid), _dptr(out), tokens,
                                        _current_stream(stream)))
+
+
+class Decoder:
+    """The decoder stack behind the C ABI (enc_decoder_create / enc_decoder_forward).
+
+    layers: per-layer dicts with the keys of DECODER_WEIGHT_FIELDS (numpy FP16
+    arrays, [in, out] row-major)."""
+
+    def __init__(self, head_num: int, size_per_head: int, ffn_dim: int, layers: Sequence[Dict]):
+        self.lib = load_library()
+        self.hidden = head_num * size_per_head
+        arr = (EncDecoderLayerWeights * max(1, len(layers)))()
+        keep = []
+        for i, lw in enumerate(layers):
+            for name in DECODER_WEIGHT_FIELDS:
+                v = np.ascontiguousarray(lw[name], dtype=np.float16)
+                keep.append(v)
+                setattr(arr[i], name, v.ctypes.data)
+        h = ctypes.c_void_p()
+        _check(self.lib.enc_decoder_create(head_num, size_per_head, ffn_dim, len(layers), DTYPE_CODES["fp16"],
+                                           ctypes.cast(arr, ctypes.c_void_p), ctypes.byref(h)))
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            _check(self.lib.enc_destroy(self.handle))
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_gelu(self, form: str):
+        _check(self.lib.enc_set_gelu(self.handle, {"erf": 0, "tanh": 1}[form]))
+
+    def forward(self, y, tgt_len, mem, mem_len, out=None, stream=None):
+        """y: CUDA [B, T, H] FP16; mem: CUDA [B, S, H] FP16; lengths: CUDA int32 [B]."""
+        import torch
+        B, T, _ = y.shape
+        S = mem.shape[1]
+        if out is None:
+            out = torch.empty_like(y)
+        _check(self.lib.enc_decoder_forward(self.handle, _dptr(y), _dptr(tgt_len), _dptr(mem), _dptr(mem_len),
+                                            _dptr(out), B, T, S, _current_stream(stream)))
+        return out
+
+    def device_status(self) -> int:
+        code = ctypes.c_int32(0)
+        st = self.lib.enc_device_status(self.handle, ctypes.byref(code))
+        if st not in (ENC_OK, 5):
+            _check(st)
+        return int(code.value)
 
 
 class RecordedForward:

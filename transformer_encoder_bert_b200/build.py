@@ -23,7 +23,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libbertenc.so")
 SOURCES = ["gemm_tc.cu", "gemm_f32.cu", "attention.cu", "attention_tc.cu", "layernorm.cu", "pack.cu",
-           "persistent.cu", "encoder.cu"]
+           "persistent.cu", "decoder_attention.cu", "encoder.cu"]
 
 
 def nvcc_path() -> str:

@@ -89,6 +89,16 @@ struct LayerDev {
   CUtensorMap tm_qkv[2], tm_o[2], tm_ff1[2], tm_ff2[2];   // [0]: 128-row box, [1]: 256-row box
 };
 
+// One decoder layer on the device: FP16 weights transposed to [out, in] with
+// their tensor maps (128- and 256-row boxes), FP32 biases and LayerNorm
+// parameters, FP16 copies of the LayerNorm parameters for the LayerNorm kernel.
+struct DecLayerDev {
+  void *w_qkv, *w_o, *w_q2, *w_kv2, *w_o2, *w_ff1, *w_ff2;
+  float *b_qkv, *b_o, *b_q2, *b_kv2, *b_o2, *b_ff1, *b_ff2;
+  __half *ln_g[3], *ln_b[3];
+  CUtensorMap tm_qkv[2], tm_o[2], tm_q2[2], tm_kv2[2], tm_o2[2], tm_ff1[2], tm_ff2[2];
+};
+
 }  // namespace
 
 struct enc_handle {
@@ -133,6 +143,8 @@ struct enc_handle {
   CUtensorMap* d_wmaps = nullptr;           // device [L][4] weight maps of the single-launch forward
   void* persist_partial = nullptr;          // its FFN2 partial tiles and tile counters
   std::vector<cudaEvent_t> trace;   // optional per-kernel events for enc_forward
+  bool decoder = false;             // created by enc_decoder_create (its layers in dlayers)
+  std::vector<struct DecLayerDev> dlayers;
 };
 
 namespace {
@@ -846,6 +858,7 @@ enc_status forward_impl(enc_handle* h, const void* x, const int32_t* valid_len, 
                         cudaStream_t st, bool tracing) {
   enc_status s = check_handle(h);
   if (s != ENC_OK) return s;
+  if (h->decoder) return fail(ENC_ERR_INVALID_ARG, "a decoder handle runs enc_decoder_forward");
   if ((s = check_tokens(batch, seq)) != ENC_OK) return s;
   if ((s = check_ptrs({x, out})) != ENC_OK) return s;
   if (!valid_len) return fail(ENC_ERR_INVALID_ARG, "valid_len is null");
@@ -1304,6 +1317,7 @@ enc_status enc_set_trace_events(enc_t h, void* const* events, int count) {
 static enc_status op_prologue(enc_t h, int layer, bool needs_layer, int tokens) {
   enc_status s = check_handle(h);
   if (s != ENC_OK) return s;
+  if (h->decoder) return fail(ENC_ERR_INVALID_ARG, "single encoder steps need an encoder handle");
   if (needs_layer && (layer < 0 || layer >= h->L)) return fail(ENC_ERR_INVALID_ARG, "layer %d out of range", layer);
   if (tokens <= 0) return fail(ENC_ERR_INVALID_ARG, "token count must be >= 1");
   return ENC_OK;
@@ -1374,6 +1388,270 @@ enc_status enc_op_ffn2_ln(enc_t h, int layer, const void* u, const void* resid, 
   const Workspace w = carve(h, (size_t)tokens);
   if ((s = step_ffn2(h, layer, u, resid, w.a, tokens, st)) != ENC_OK) return s;
   if ((s = step_ln(h, layer, 2, w.a, out, tokens, st)) != ENC_OK) return s;
+  return ok();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ decoder forward
+//
+// [FT] "什么是 Faster Transformer" plans a decoder without describing it.  The
+// layer here is the post-LN Transformer decoder layer over a whole target
+// sequence, with the encoder's conventions (see enc.h), run as 12 launches:
+//   1 GEMM   y Wqkv + bqkv, head split [3, B, nh, T, d]
+//   2 attention (causal, keys j < tgt_len)
+//   3 GEMM   ctx Wo + bo + y           4 LayerNorm 1 -> h1
+//   5 GEMM   h1 Wq2 + bq2, head split [1, B, nh, T, d]
+//   6 GEMM   mem Wkv2 + bkv2, head split [2, B, nh, S, d]
+//   7 attention (cross, keys j < mem_len)
+//   8 GEMM   ctx2 Wo2 + bo2 + h1       9 LayerNorm 2 -> h2
+//  10 GEMM   GELU(h2 W1 + b1)         11 GEMM u W2 + b2 + h2     12 LayerNorm 3
+
+namespace {
+
+// Workspace of a decoder forward: qkv 3Mt H, ctx, z, h1, h2, q2 (Mt H each),
+// kv2 2 Ms H, u Mt F, two ping-pong layer outputs (Mt H each).
+struct DecWorkspace {
+  void *qkv, *ctx, *z, *h1, *h2, *q2, *kv2, *u, *x0, *x1;
+};
+
+size_t dec_workspace_bytes(const enc_handle* h, size_t mt, size_t ms) {
+  const size_t mh = align_up(mt * h->H * 2, 256), sh = align_up(ms * h->H * 2, 256);
+  const size_t mf = align_up(mt * h->F * 2, 256);
+  return 3 * mh + 5 * mh + 2 * sh + mf + 2 * mh;
+}
+
+DecWorkspace dec_carve(const enc_handle* h, size_t mt, size_t ms) {
+  const size_t mh = align_up(mt * h->H * 2, 256), sh = align_up(ms * h->H * 2, 256);
+  const size_t mf = align_up(mt * h->F * 2, 256);
+  char* p = static_cast<char*>(h->ws);
+  DecWorkspace w;
+  w.qkv = p; p += 3 * mh;
+  w.ctx = p; p += mh;
+  w.z = p; p += mh;
+  w.h1 = p; p += mh;
+  w.h2 = p; p += mh;
+  w.q2 = p; p += mh;
+  w.kv2 = p; p += 2 * sh;
+  w.u = p; p += mf;
+  w.x0 = p; p += mh;
+  w.x1 = p;
+  return w;
+}
+
+enc_status ensure_bytes(enc_handle* h, size_t need) {
+  if (need <= h->ws_bytes) return ENC_OK;
+  if (h->graphs_alive > 0)
+    return fail(ENC_ERR_INVALID_ARG, "workspace of %zu bytes needed but %d recorded graph(s) pin the current one",
+                need, h->graphs_alive);
+  if (h->ws) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize before workspace growth");
+    cudaFree(h->ws);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+  }
+  void* p = nullptr;
+  if (cudaMalloc(&p, need) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ENC_ERR_OOM, "workspace allocation of %zu bytes failed", need);
+  }
+  h->ws = p;
+  h->ws_bytes = need;
+  return ENC_OK;
+}
+
+enc_status dec_ln(enc_handle* h, const void* z, const __half* g, const __half* b, void* out, int rows,
+                  cudaStream_t st) {
+  cudaError_t e = enc::launch_layernorm_f16h(static_cast<const __half*>(z), g, b, static_cast<__half*>(out), rows,
+                                             h->H, st);
+  if (e != cudaSuccess) return cuda_fail(e, "LayerNorm launch");
+  ++h->launches;
+  return ENC_OK;
+}
+
+enc_status dec_attention(enc_handle* h, const void* q, const void* k, const void* v, const int32_t* kv_len, void* ctx,
+                         int batch, int tgt_seq, int kv_seq, bool causal, cudaStream_t st) {
+  cudaError_t e = enc::launch_decoder_attention(static_cast<const __half*>(q), static_cast<const __half*>(k),
+                                                static_cast<const __half*>(v), kv_len, static_cast<__half*>(ctx),
+                                                batch, h->nh, h->d, tgt_seq, kv_seq, causal, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decoder attention launch");
+  ++h->launches;
+  return ENC_OK;
+}
+
+enc_status dec_layer(enc_handle* h, int l, const void* yin, void* yout, const int32_t* tgt_len, const void* mem,
+                     const int32_t* mem_len, int B, int T, int S, const DecWorkspace& w, cudaStream_t st) {
+  DecLayerDev& L = h->dlayers[l];
+  const int H = h->H, Mt = B * T, Ms = B * S;
+  const size_t hd = (size_t)B * h->nh * h->d;   // elements of one [B, nh, ., d] block per token
+  enc_status s;
+  const enc::SplitShape spt{B, T, h->nh, h->d}, sps{B, S, h->nh, h->d};
+  if ((s = run_gemm(h, yin, Mt, H, L.w_qkv, L.tm_qkv, 3 * H, enc::Epi::kBiasQkvSplit, L.b_qkv, w.qkv, spt, st)) !=
+      ENC_OK)
+    return s;
+  const __half* qkv = static_cast<const __half*>(w.qkv);
+  if ((s = dec_attention(h, qkv, qkv + hd * T, qkv + 2 * hd * T, tgt_len, w.ctx, B, T, T, true, st)) != ENC_OK)
+    return s;
+  if ((s = run_gemm(h, w.ctx, Mt, H, L.w_o, L.tm_o, H, enc::Epi::kBiasResidStore, L.b_o, w.z, {}, st, nullptr,
+                    yin)) != ENC_OK)
+    return s;
+  if ((s = dec_ln(h, w.z, L.ln_g[0], L.ln_b[0], w.h1, Mt, st)) != ENC_OK) return s;
+  if ((s = run_gemm(h, w.h1, Mt, H, L.w_q2, L.tm_q2, H, enc::Epi::kBiasQkvSplit, L.b_q2, w.q2, spt, st)) != ENC_OK)
+    return s;
+  if ((s = run_gemm(h, mem, Ms, H, L.w_kv2, L.tm_kv2, 2 * H, enc::Epi::kBiasQkvSplit, L.b_kv2, w.kv2, sps, st)) !=
+      ENC_OK)
+    return s;
+  const __half* kv2 = static_cast<const __half*>(w.kv2);
+  if ((s = dec_attention(h, w.q2, kv2, kv2 + hd * S, mem_len, w.ctx, B, T, S, false, st)) != ENC_OK) return s;
+  if ((s = run_gemm(h, w.ctx, Mt, H, L.w_o2, L.tm_o2, H, enc::Epi::kBiasResidStore, L.b_o2, w.z, {}, st, nullptr,
+                    w.h1)) != ENC_OK)
+    return s;
+  if ((s = dec_ln(h, w.z, L.ln_g[1], L.ln_b[1], w.h2, Mt, st)) != ENC_OK) return s;
+  const enc::Epi gelu = h->gelu == ENC_GELU_TANH ? enc::Epi::kBiasGeluTanh : enc::Epi::kBiasGelu;
+  if ((s = run_gemm(h, w.h2, Mt, H, L.w_ff1, L.tm_ff1, h->F, gelu, L.b_ff1, w.u, {}, st)) != ENC_OK) return s;
+  if ((s = run_gemm(h, w.u, Mt, h->F, L.w_ff2, L.tm_ff2, H, enc::Epi::kBiasResidStore, L.b_ff2, w.z, {}, st, nullptr,
+                    w.h2)) != ENC_OK)
+    return s;
+  return dec_ln(h, w.z, L.ln_g[2], L.ln_b[2], yout, Mt, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+enc_status enc_decoder_create(int head_num, int size_per_head, int ffn_dim, int num_layers, enc_dtype dtype,
+                              const enc_decoder_layer_weights* weights, enc_t* out) {
+  if (!out) return fail(ENC_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  if (head_num <= 0 || size_per_head <= 0 || ffn_dim <= 0 || num_layers <= 0)
+    return fail(ENC_ERR_INVALID_ARG, "head_num, size_per_head, ffn_dim and num_layers must be > 0");
+  if (size_per_head != 32 && size_per_head != 64 && size_per_head != 128)
+    return fail(ENC_ERR_UNSUPPORTED, "size_per_head %d not in {32, 64, 128}", size_per_head);
+  if (dtype != ENC_FP16) return fail(ENC_ERR_UNSUPPORTED, "the decoder runs in FP16 mode only");
+  if (ffn_dim % 8 != 0) return fail(ENC_ERR_INVALID_ARG, "ffn_dim %d is not a multiple of 8", ffn_dim);
+  const int H = head_num * size_per_head;
+  if (H > 1024) return fail(ENC_ERR_UNSUPPORTED, "hidden size %d exceeds 1024", H);
+  if (!weights) return fail(ENC_ERR_INVALID_ARG, "weights is null");
+  for (int l = 0; l < num_layers; ++l) {
+    const void* const* ps = reinterpret_cast<const void* const*>(&weights[l]);
+    for (size_t i = 0; i < sizeof(enc_decoder_layer_weights) / sizeof(void*); ++i)
+      if (!ps[i]) return fail(ENC_ERR_INVALID_ARG, "decoder layer %d has a null parameter pointer", l);
+  }
+  int cur_dev = -1;
+  if (cudaGetDevice(&cur_dev) != cudaSuccess) return fail(ENC_ERR_CUDA, "no CUDA device");
+  int first = -1;
+  if (!g_process_device.compare_exchange_strong(first, cur_dev) && first != cur_dev)
+    return fail(ENC_ERR_UNSUPPORTED, "handles of one process share one CUDA device (%d); the current device is %d",
+                first, cur_dev);
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, cur_dev) != cudaSuccess || prop.major != 10)
+    return fail(ENC_ERR_UNSUPPORTED, "FP16 mode needs an sm_100 (B200-class) device");
+
+  enc_handle* h = new enc_handle();
+  h->decoder = true;
+  h->nh = head_num; h->d = size_per_head; h->H = H; h->F = ffn_dim; h->L = num_layers;
+  h->dtype = ENC_FP16;
+  h->esize = 2;
+  h->device = cur_dev;
+  h->num_sms = enc::device_sm_count();
+  if (cudaMalloc(&h->status, 8 * sizeof(int)) != cudaSuccess ||
+      cudaMemset(h->status, 0, 8 * sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    free_handle(h);
+    return fail(ENC_ERR_OOM, "status word allocation failed");
+  }
+  const size_t F = ffn_dim;
+  // Matrices [in, out]: Wqkv [H,3H], Wo [H,H], Wq2 [H,H], Wkv2 [H,2H], Wo2 [H,H], W1 [H,F], W2 [F,H].
+  const size_t mrows[7] = {(size_t)H, (size_t)H, (size_t)H, (size_t)H, (size_t)H, (size_t)H, F};
+  const size_t mcols[7] = {3 * (size_t)H, (size_t)H, (size_t)H, 2 * (size_t)H, (size_t)H, F, (size_t)H};
+  const size_t vlen[7] = {3 * (size_t)H, (size_t)H, (size_t)H, 2 * (size_t)H, (size_t)H, F, (size_t)H};
+  size_t per_layer = 6 * align_up((size_t)H * 2, 256), staging = 0;
+  for (int i = 0; i < 7; ++i) {
+    per_layer += align_up(mrows[i] * mcols[i] * 2, 256) + align_up(vlen[i] * 4, 256);
+    staging = std::max(staging, align_up(mrows[i] * mcols[i] * 2, 256));
+  }
+  if (cudaMalloc(&h->param_block, per_layer * num_layers + staging) != cudaSuccess) {
+    cudaGetLastError();
+    free_handle(h);
+    return fail(ENC_ERR_OOM, "parameter allocation failed");
+  }
+  char* p = static_cast<char*>(h->param_block);
+  char* stage = p + per_layer * num_layers;
+  h->dlayers.resize(num_layers);
+  for (int l = 0; l < num_layers; ++l) {
+    const enc_decoder_layer_weights& wsrc = weights[l];
+    DecLayerDev& L = h->dlayers[l];
+    const void* msrc[7] = {wsrc.w_qkv, wsrc.w_o, wsrc.w_q2, wsrc.w_kv2, wsrc.w_o2, wsrc.w_ff1, wsrc.w_ff2};
+    void** mdst[7] = {&L.w_qkv, &L.w_o, &L.w_q2, &L.w_kv2, &L.w_o2, &L.w_ff1, &L.w_ff2};
+    CUtensorMap* maps[7] = {L.tm_qkv, L.tm_o, L.tm_q2, L.tm_kv2, L.tm_o2, L.tm_ff1, L.tm_ff2};
+    const void* vsrc[7] = {wsrc.b_qkv, wsrc.b_o, wsrc.b_q2, wsrc.b_kv2, wsrc.b_o2, wsrc.b_ff1, wsrc.b_ff2};
+    float** vdst[7] = {&L.b_qkv, &L.b_o, &L.b_q2, &L.b_kv2, &L.b_o2, &L.b_ff1, &L.b_ff2};
+    for (int i = 0; i < 7; ++i) {
+      *mdst[i] = p;
+      const size_t bytes = mrows[i] * mcols[i] * 2;
+      cudaError_t e = cudaMemcpy(stage, msrc[i], bytes, cudaMemcpyDefault);
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder weight upload"); }
+      const dim3 grid((unsigned)((mcols[i] + 31) / 32), (unsigned)((mrows[i] + 31) / 32));
+      transpose_f16_kernel<<<grid, dim3(32, 8)>>>(reinterpret_cast<const __half*>(stage), reinterpret_cast<__half*>(p),
+                                                  (int)mrows[i], (int)mcols[i]);
+      e = cudaDeviceSynchronize();
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder weight repack"); }
+      // B operand [N = out, K = in]
+      if (!enc::encode_kmajor_fp16_map(&maps[i][0], p, mcols[i], mrows[i], 128) ||
+          !enc::encode_kmajor_fp16_map(&maps[i][1], p, mcols[i], mrows[i], 256)) {
+        free_handle(h);
+        return fail(ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed for a decoder weight");
+      }
+      p += align_up(bytes, 256);
+      *vdst[i] = reinterpret_cast<float*>(p);
+      e = cudaMemcpy(stage, vsrc[i], vlen[i] * 2, cudaMemcpyDefault);
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder bias upload"); }
+      widen_to_f32_kernel<__half><<<(unsigned)((vlen[i] + 255) / 256), 256>>>(reinterpret_cast<const __half*>(stage),
+                                                                              *vdst[i], (int)vlen[i]);
+      e = cudaDeviceSynchronize();
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder bias widen"); }
+      p += align_up(vlen[i] * 4, 256);
+    }
+    const void* lsrc[6] = {wsrc.ln1_g, wsrc.ln1_b, wsrc.ln2_g, wsrc.ln2_b, wsrc.ln3_g, wsrc.ln3_b};
+    for (int i = 0; i < 6; ++i) {
+      __half* dst = reinterpret_cast<__half*>(p);
+      cudaError_t e = cudaMemcpy(dst, lsrc[i], (size_t)H * 2, cudaMemcpyDefault);
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder LayerNorm upload"); }
+      if (i % 2 == 0) L.ln_g[i / 2] = dst; else L.ln_b[i / 2] = dst;
+      p += align_up((size_t)H * 2, 256);
+    }
+  }
+  *out = h;
+  return ok();
+}
+
+enc_status enc_decoder_forward(enc_t h, const void* y, const int32_t* tgt_len, const void* mem,
+                               const int32_t* mem_len, void* out, int batch, int tgt_seq, int mem_seq,
+                               enc_stream_t stream) {
+  enc_status s = check_handle(h);
+  if (s != ENC_OK) return s;
+  if (!h->decoder) return fail(ENC_ERR_INVALID_ARG, "an encoder handle runs enc_forward");
+  if ((s = check_tokens(batch, tgt_seq)) != ENC_OK) return s;
+  if ((s = check_tokens(batch, mem_seq)) != ENC_OK) return s;
+  if ((s = check_ptrs({y, mem, out})) != ENC_OK) return s;
+  if (!tgt_len || !mem_len) return fail(ENC_ERR_INVALID_ARG, "tgt_len and mem_len must not be null");
+  const size_t mt = (size_t)batch * tgt_seq, ms = (size_t)batch * mem_seq;
+  const size_t bytes = mt * h->H * 2;
+  const char* yb = static_cast<const char*>(y);
+  const char* ob = static_cast<const char*>(out);
+  if (yb < ob + bytes && ob < yb + bytes) return fail(ENC_ERR_INVALID_ARG, "out overlaps y");
+  if ((s = ensure_bytes(h, dec_workspace_bytes(h, mt, ms))) != ENC_OK) return s;
+  const DecWorkspace w = dec_carve(h, mt, ms);
+  PdlScope pdl(h);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int l = 0; l < h->L; ++l) {
+    const void* yin = l == 0 ? y : ((l - 1) & 1 ? w.x1 : w.x0);
+    void* yout = l == h->L - 1 ? out : (l & 1 ? w.x1 : w.x0);
+    if ((s = dec_layer(h, l, yin, yout, tgt_len, mem, mem_len, batch, tgt_seq, mem_seq, w, st)) != ENC_OK) return s;
+  }
   return ok();
 }
 

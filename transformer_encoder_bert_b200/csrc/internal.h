@@ -160,6 +160,13 @@ cudaError_t launch_layernorm_f16h(const __half* z, const __half* gamma, const __
 cudaError_t launch_layernorm_f32(const float* z, const float* gamma, const float* beta, float* out, int rows,
                                  int hidden, cudaStream_t stream);
 
+// ---- decoder attention, decoder_attention.cu ----
+// q [B, nh, T, d], k and v [B, nh, Skv, d] (head-split); keys j < clamp(kv_len[b],
+// 0, Skv), and with `causal` j <= i for query i; ctx [B*T, nh*d].
+cudaError_t launch_decoder_attention(const __half* q, const __half* k, const __half* v, const int32_t* kv_len,
+                                     __half* ctx, int batch, int head_num, int size_per_head, int tgt_seq, int kv_seq,
+                                     bool causal, cudaStream_t stream);
+
 // ---- single-launch forward for small batches, persistent.cu ----
 constexpr int kPersistMaxTokens = 256;   // batch * seq
 constexpr int kPersistMaxSplits = 4;     // K splits of FFN2
