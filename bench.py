@@ -18,7 +18,8 @@ enc_forward calls right after them (a recorded forward carries no events).  The
 events break the overlap between kernels, so those times are upper bounds on the
 in-graph ones; the roofline divides by the measured burst tensor peak (kernels of
 microseconds inside millisecond steps).  --impl reference times the float64 CPU
-oracle on a bounded sample.
+oracle on a bounded sample.  Rates use each kernel's in-graph time, estimated as
+its share of the traced forward times the graph's step (graph_us).
 Default workload: 12-layer BERT-Base shape (12x64, FFN 3072), seq 32, batch 512;
 the goal point (BERT-Base, seq 128, batch 256) is timed in the same run and
 reported under "secondary" (one GPU; --secondary '' skips it).
@@ -73,12 +74,12 @@ def load_peaks():
 # Sources each timed kernel is built from: a DRAM-traffic figure measured by
 # ncu holds only while these files are unchanged.
 KERNEL_SOURCES = {
-    "qkv_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
-    "out_proj_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
-    "ffn1_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
-    "ffn2_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
-    "out_proj_ln_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
-    "ffn2_ln_gemm": ["gemm_tc.cu", "sm100.cuh", "internal.h"],
+    "qkv_gemm": ["gemm_tc.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
+    "out_proj_gemm": ["gemm_tc.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
+    "ffn1_gemm": ["gemm_tc.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
+    "ffn2_gemm": ["gemm_tc.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
+    "out_proj_ln_gemm": ["gemm_tc.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
+    "ffn2_ln_gemm": ["gemm_tc.cu", "gelu.cuh", "sm100.cuh", "internal.h"],
     "attention": ["attention.cu", "attention_tc.cu", "sm100.cuh", "internal.h"],
     "ln1": ["layernorm.cu", "internal.h"],
     "ln2": ["layernorm.cu", "internal.h"],
@@ -357,10 +358,15 @@ def time_forward(enc, x, vl, out, wl, args, flush, stream, barrier):
             "traced_ms": sum(traced) / len(traced), "nk": nk}
 
 
-def kernel_table(wl, inp, per_kernel, peaks, packed: bool):
+def kernel_table(wl, inp, per_kernel, peaks, packed: bool, graph_ms=None, forwards=None):
     """Per kernel: average traced time, share, TFLOP/s (GEMMs) and algorithmic GB/s,
     each with its fraction of the measured peak (burst tensor peak: the kernels run
-    for microseconds inside steps of milliseconds)."""
+    for microseconds inside steps of milliseconds).  With graph_ms (the timed
+    graph's step) and the number of traced forwards, the rates come from the
+    kernel's in-graph time, estimated as its share of the traced forward times
+    graph_ms per launch (graph_us); avg_us, the traced per-launch time, is an
+    upper bound (events between kernels break the overlap of programmatic
+    dependent launch)."""
     sh = wl.shape
     work = kernel_work(wl)
     if packed:
@@ -374,9 +380,14 @@ def kernel_table(wl, inp, per_kernel, peaks, packed: bool):
     kernels = {}
     total = sum(sum(v) for v in per_kernel.values())
     for k, vals in per_kernel.items():
+        share = sum(vals) / total
         avg_ms = sum(vals) / len(vals)
+        entry = {"avg_us": avg_ms * 1e3, "share": share}
+        if graph_ms is not None and forwards:
+            launches_per_step = len(vals) / forwards
+            avg_ms = share * graph_ms / launches_per_step
+            entry["graph_us"] = avg_ms * 1e3
         flops, nbytes = work[k]
-        entry = {"avg_us": avg_ms * 1e3, "share": sum(vals) / total}
         if flops and (k.endswith("gemm") or k == "persistent"):
             entry["tflops"] = flops / (avg_ms * 1e-3) / 1e12
             entry["tensor_frac"] = entry["tflops"] / tc_peak
@@ -389,6 +400,11 @@ def kernel_table(wl, inp, per_kernel, peaks, packed: bool):
 
 def roofline_of(kernels, work, dominant, peaks, peak_src, traffic):
     d = kernels[dominant]
+    in_graph = "graph_us" in d
+    time_source = ("the kernel's share of the traced forward times the timed graph's step, per launch (the traced "
+                   "per-launch time, an upper bound, is avg_us)" if in_graph else
+                   "traced enc_forward calls (events between kernels): an upper bound on the kernel's time in "
+                   "the timed graph, so achieved is a lower bound")
     if dominant == "persistent":
         # small batch: every weight byte is read once per forward, so HBM bounds it
         peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -403,14 +419,12 @@ def roofline_of(kernels, work, dominant, peaks, peak_src, traffic):
                 "kernel": dominant, "per_launch_flops": work[dominant][0],
                 "peak_source": f"{peak_src} burst bf16 matmul (FP16 dense rate = BF16 dense rate); "
                                "the kernel runs for microseconds inside millisecond steps",
-                "time_source": "traced enc_forward calls (events between kernels): an upper bound on "
-                               "the kernel's time in the timed graph, so achieved is a lower bound"}
+                "time_source": time_source}
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     return {"bound": "hbm", "achieved": d["gbs"], "peak": peak, "unit": "GB/s", "frac": d["gbs"] / peak,
             "traffic": traffic, "kernel": dominant, "per_launch_bytes": work[dominant][1],
             "peak_source": f"{peak_src} HBM copy bandwidth",
-            "time_source": "traced enc_forward calls (events between kernels): an upper bound on "
-                           "the kernel's time in the timed graph, so achieved is a lower bound"}
+            "time_source": time_source}
 
 
 def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
@@ -497,7 +511,8 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         return 0
 
     peaks, peak_src = load_peaks()
-    kernels, work = kernel_table(wl, inp, main_t["per_kernel"], peaks, args.packed)
+    kernels, work = kernel_table(wl, inp, main_t["per_kernel"], peaks, args.packed,
+                                 graph_ms=ms if args.graph else None, forwards=args.steps)
     dominant = max(kernels, key=lambda k: kernels[k]["share"])
     traffic = args.traffic if args.traffic is not None else measured_traffic(dominant, wl.name)
     roof = roofline_of(kernels, work, dominant, peaks, peak_src, traffic)
@@ -524,11 +539,13 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     }
     if secondary is not None:
         sw, st = secondary["wl"], secondary["sec_t"]
-        skern, swork = kernel_table(sw, secondary["inp"], st["per_kernel"], peaks, args.packed)
+        skern, swork = kernel_table(sw, secondary["inp"], st["per_kernel"], peaks, args.packed,
+                                    graph_ms=st["ms"] if args.graph else None, forwards=args.steps)
         sdom = max(skern, key=lambda k: skern[k]["share"])
         gemms = [k for k in skern if k.endswith("gemm")]
         g_flops = sum(swork[k][0] * len(st["per_kernel"][k]) for k in gemms) / args.steps
-        g_ms = sum(sum(st["per_kernel"][k]) for k in gemms) / args.steps
+        g_ms = sum(skern[k].get("graph_us", skern[k]["avg_us"]) * 1e-3 * len(st["per_kernel"][k]) for k in gemms) \
+            / args.steps
         tc_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         line["secondary"] = {
             "workload": sw.name, "value": sw.batch / (st["ms"] * 1e-3), "unit": UNIT, "ms_per_step": st["ms"],
@@ -544,6 +561,75 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"first {n} of the {wl.batch} sequences of this workload, "
                                           f"float64 numpy oracle, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ decoder leg
+def decoder_workload(spec: str) -> "EI.DecoderWorkload":
+    """decoder-base:B:T:S (BERT-Base structure, 12 layers) or decoder-large:B:T:S
+    (BERT-Large structure, 24 layers): target lengths U[T/2, T], memory lengths U[S/2, S]."""
+    kind, b, t, sm = spec.split(":")
+    shape = {"decoder-base": EI.BERT_BASE, "decoder-large": EI.BERT_LARGE}[kind]
+    b, t, sm = int(b), int(t), int(sm)
+    return EI.DecoderWorkload(f"{kind}-{shape.num_layers}L-h{shape.hidden}-t{t}-s{sm}-b{b}-fp16", shape, b, t, sm,
+                              "fp16", t // 2, t, sm // 2, sm)
+
+
+def decoder_flops(wl) -> float:
+    """GEMM and attention flops of one decoder forward over the padded lengths."""
+    sh = wl.shape
+    H, F, L = sh.hidden, sh.ffn_dim, sh.num_layers
+    mt, ms = wl.batch * wl.tgt_seq, wl.batch * wl.mem_seq
+    gemm = 2.0 * mt * H * (3 * H + H + H + H + 2 * F) + 2.0 * ms * H * 2 * H
+    attn = 4.0 * mt * wl.tgt_seq * H / 2 + 4.0 * mt * wl.mem_seq * H      # causal half + cross
+    return L * (gemm + attn)
+
+
+def run_decoder(args, rank: int, world: int, local_rank: int):
+    """Device time of the decoder stack (enc_decoder_forward per step, L2 flushed
+    before each); the roofline is the whole forward's flops at the burst peak."""
+    import torch
+    from transformer_encoder_bert_b200 import Decoder
+    torch.cuda.set_device(local_rank)
+    wl = decoder_workload(args.workload).with_(seed=rank)
+    inp = EI.make_decoder_inputs(wl)
+    sh = wl.shape
+    dec = Decoder(sh.head_num, sh.size_per_head, sh.ffn_dim, inp.layers)
+    dev = torch.device("cuda", local_rank)
+    y, mem = torch.from_numpy(inp.y).to(dev), torch.from_numpy(inp.mem).to(dev)
+    tl, ml = torch.from_numpy(inp.tgt_len).to(dev), torch.from_numpy(inp.mem_len).to(dev)
+    out = torch.empty_like(y)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        dec.forward(y, tl, mem, ml, out)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        dec.forward(y, tl, mem, ml, out)
+        e.record()
+        e.synchronize()
+        ts.append(s.elapsed_time(e))
+    status = dec.device_status()
+    ms = max_over_ranks([sum(ts) / len(ts)], device=dev)[0]
+    if rank != 0:
+        return 0
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tf = decoder_flops(wl) / (ms * 1e-3) / 1e12
+    line = {"metric": "decoder fwd sequences/s", "value": job_throughput(wl.batch, world, ms), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "tgt_seq": wl.tgt_seq, "mem_seq": wl.mem_seq,
+                       "layers": sh.num_layers, "l2": "flushed before every timed step (256 MiB write)",
+                       "launch": "enc_decoder_forward per step (12 launches per layer)"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "traffic": None, "kernel": "whole decoder forward",
+                         "peak_source": f"{peak_src} burst bf16 matmul"},
+            "device_status": status}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -579,6 +665,10 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.workload.startswith("decoder-"):
+        if args.impl == "reference" or world > 1:
+            ap.error("the decoder leg runs our implementation on one GPU")
+        return run_decoder(args, rank, world, local_rank)
     wl = parse_workload(args.workload)
 
     if args.impl == "reference":

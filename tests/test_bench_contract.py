@@ -115,6 +115,23 @@ def test_roofline_divides_by_the_burst_tensor_peak():
     roof = bench.roofline_of(kernels, work, "ffn2_ln_gemm", peaks, "measured", None)
     assert roof["peak"] == 1653.4
     assert roof["achieved"] == pytest.approx(2 * 16384 * 3072 * 768 / 73.6e-6 / 1e12)
+    # in-graph time: the kernel's share of the traced forward times the graph step,
+    # per launch (two traced forwards of one launch each per kernel here)
+    kg, _ = bench.kernel_table(wl, None, per_kernel, peaks, packed=False, graph_ms=0.5, forwards=2)
+    share = 0.0736 / (0.0736 + 5 * 0.1)
+    assert kg["ffn2_ln_gemm"]["graph_us"] == pytest.approx(share * 0.5 * 1e3)
+    rg = bench.roofline_of(kg, work, "ffn2_ln_gemm", peaks, "measured", None)
+    assert rg["achieved"] == pytest.approx(2 * 16384 * 3072 * 768 / (share * 0.5e-3) / 1e12)
     assert roof["frac"] == pytest.approx(roof["achieved"] / 1653.4)
     ln = bench.roofline_of(kernels, work, "ln1", peaks, "measured", None)
     assert ln["bound"] == "hbm" and ln["frac"] == pytest.approx(2 * 2 * 16384 * 768 / 0.1e-3 / 1e9 / 6558.4)
+
+
+def test_decoder_workload_and_flops():
+    wl = bench.decoder_workload("decoder-base:8:64:128")
+    assert (wl.batch, wl.tgt_seq, wl.mem_seq, wl.shape.num_layers) == (8, 64, 128, 12)
+    H, F = 768, 3072
+    mt, ms = 8 * 64, 8 * 128
+    gemm = 2 * mt * H * (6 * H + 2 * F) + 2 * ms * H * 2 * H
+    attn = 4 * mt * 64 * H / 2 + 4 * mt * 128 * H
+    assert bench.decoder_flops(wl) == pytest.approx(12 * (gemm + attn))
