@@ -6,27 +6,31 @@
 //
 // The source page ("Faster Transformer 优化原理") runs attention as two batched
 // GEMMs around a SoftMax kernel.  Here both products run on tcgen05 and the
-// score tile never leaves the SM: one CTA per (sequence, head), 160 threads:
+// score tile never leaves the SM.  The one-block kernel is persistent: about
+// four CTAs per SM, each taking (sequence, head) items in turn, 160 threads:
 //   warps 0..3  softmax: thread r owns query row r = TMEM lane r.  It reads its
 //               row of S from TMEM, takes the row max over the valid keys (the
 //               row is in one thread: no shuffles), forms
 //               P = exp(S/sqrt(d) - max) in FP32, sums it, and writes P as FP16
-//               in the 128-byte-swizzled K-major layout the next MMA reads.
-//               After P V it scales its row of O by 1/sum and stores it.
+//               back into TMEM over the scores it has read.  After P V it
+//               scales its row of O by 1/sum and stores it.
 //   warp 4      one thread issues the TMA loads of Q, K and V and the MMAs
-//                 S = Q K^T   M=128, N=128, K=64  (A, B K-major)
-//                 O = P V     M=128, N=64,  K=128 (A K-major; B = V read
-//                             MN-major straight from its token-major tile)
-// The valid length n is the same for every row of the CTA, so every masking
+//                 S = Q K^T   M=128, N=128, K=64  (A, B K-major, both in smem)
+//                 O = P V     M=128, N=64,  K=16 per valid 16-key group (A = P
+//                             read from TMEM; B = V read MN-major straight from
+//                             its token-major tile)
+// The valid length n is the same for every row of an item, so every masking
 // decision is a warp-uniform branch: 32-key chunks wholly past n are skipped,
 // chunks wholly inside n run unmasked, and at most one chunk is masked per
 // element.  Keys j >= n get weight exactly 0.
 //
-// Footprint, so that four CTAs share an SM (their loads, MMAs and softmax
-// overlap one another): P (32 KB) overwrites the Q and K tiles once S = Q K^T
-// has completed, the output rows are staged in the V tile once O = P V has
-// completed, and O takes S's TMEM columns [0, 64) (128 columns per CTA).
-// Every mbarrier wait is bounded in time.
+// P in TMEM frees the Q and K tiles as soon as S = Q K^T has completed, so the
+// next item's Q and K load while this item's softmax, P V and output run; its
+// V loads once the output rows staged in the V tile have been read by their
+// TMA stores.  TMEM:
+// S in columns [0, 128), P (two halves per column) over [0, 64), O in
+// [64, 128); the next S waits until O has been read.  Footprint per CTA: 48 KB
+// of tiles and 128 TMEM columns.  Every mbarrier wait is bounded in time.
 //
 // Q, K and V are read through one 2-D tensor map with rows of 64 halves:
 // the split layout [3, B, nh, S, 64] (rows = ((t*B + b)*nh + h)*S + s) or the
@@ -52,16 +56,18 @@ constexpr int kTileBytes = kRows * kD * 2;        // 16 KB: 128 rows x 64 halves
 constexpr int kTmemCols = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared memory (offsets from a 1024-byte-aligned base).
-constexpr int kQ = 0;                             // Q tile, then P keys 0..63
-constexpr int kK = kTileBytes;                    // K tile, then P keys 64..127
-constexpr int kP = 0;                             // P: two 64-key K-major atoms
+// Shared memory of the one-block kernel (offsets from a 1024-byte-aligned base).
+constexpr int kQ = 0;                             // Q tile
+constexpr int kK = kTileBytes;                    // K tile
 constexpr int kV = 2 * kTileBytes;                // V tile, then the output rows
 constexpr int kBars = 3 * kTileBytes;
-// qk_full, v_full, s_full, p_full, o_full, drain
-constexpr int kNumBars = 6;
+// qk_full, v_full, s_full, p_full, o_full, o_free, v_free, drain
+constexpr int kNumBars = 8;
 constexpr int kSlot = kBars + kNumBars * 8;
 constexpr int kSmemTotal = 1024 + kSlot + 16;
+constexpr int kOCol = 64;                         // O's TMEM columns [64, 128)
+constexpr int kCtasPerSm = 4;                     // TMEM 4 x 128 columns, shared memory 4 x 50 KB
+static_assert(kCtasPerSm * (kSmemTotal + 1024) <= 228 * 1024, "four CTAs per SM");
 
 // MN-major operand, 128-byte swizzle: 64 contiguous MN elements (128 bytes) per
 // row, K rows 128 bytes apart in groups of 8 that are 1 KB apart (stride byte
@@ -128,36 +134,51 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&sv)[32], int lim, uint6
     store_p_unit(prow, 4 * c + u, r, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
 }
 
+// P of 32 keys (chunk c of the row) from 32 raw scores: p = 2^(s*c2 - m*c2)
+// for the first `lim` keys, 0 for the rest; adds to the pair sum and writes
+// the FP16 values into TMEM as 16 columns (two keys per column) of this lane.
+template <bool MASKED>
+__device__ __forceinline__ void p_chunk_tmem(const uint32_t (&sv)[32], int lim, uint64_t scale2, uint64_t neg_m2,
+                                             uint64_t& sum2, uint32_t t_p) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const uint64_t t = f2_fma(f2_pack(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), scale2, neg_m2);
+    float t0, t1;
+    f2_unpack(t, t0, t1);
+    float p0 = ex2(t0), p1 = ex2(t1);
+    if (MASKED) {
+      p0 = i < lim ? p0 : 0.f;
+      p1 = i + 1 < lim ? p1 : 0.f;
+    }
+    sum2 = f2_add(sum2, f2_pack(p0, p1));
+    pk[i >> 1] = cvt_half2(p0, p1);
+  }
+  tmem_st_32x32b_x16_async(t_p, pk);
+}
+
 template <bool PACKED>
-__global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 128 columns)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int32_t* __restrict__ valid_len,
                         const int32_t* __restrict__ offsets, __half* __restrict__ ctx, int B, int S, int NH,
-                        float score_scale_log2, int* __restrict__ status) {
+                        float score_scale_log2, const __grid_constant__ CUtensorMap tm_ctx,
+                        int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + kBars;
   const uint32_t qk_full = bar0, v_full = bar0 + 8, s_full = bar0 + 16, p_full = bar0 + 24, o_full = bar0 + 32,
-                 drain = bar0 + 40;
+                 o_free = bar0 + 40, v_free = bar0 + 48, drain = bar0 + 56;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Sequences are taken last to first: the QKV GEMM before this kernel writes
-  // the rows of the last sequences last, so those are the ones still in L2.
-  const int h = blockIdx.x, b = B - 1 - (int)blockIdx.y;
-  pdl_wait();                                          // Q/K/V (and offsets) of the previous kernels are visible
-  int n = valid_len[b];
-  n = n < 0 ? 0 : (n > S ? S : n);
-  if (PACKED && n == 0) return;                        // the sequence has no rows (uniform per CTA)
-  const int rows_exist = PACKED ? n : S;
   const int H = NH * kD;
-
-  // Tensor-map coordinates of row s of block t (0 = Q, 1 = K, 2 = V).
-  auto coord_x = [&](int t) { return PACKED ? t * H + h * kD : 0; };
-  auto coord_y = [&](int t, int s) { return PACKED ? offsets[b] + s : ((t * B + b) * NH + h) * S + s; };
-
+  const int items = B * NH;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar0 + 8 * i, bar0 + 8 * i == p_full ? kSoftmaxWarps : 1);
+    for (int i = 0; i < kNumBars; ++i) {
+      const uint32_t bar = bar0 + 8 * i;
+      mbar_init(bar, (bar == p_full || bar == o_free || bar == v_free) ? kSoftmaxWarps : 1);
+    }
     fence_barrier_init();
   }
   if (warp == kSoftmaxWarps) {
@@ -167,141 +188,198 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;                    // S in columns [0, 128); O in [0, 64) after softmax
+  const uint32_t tmem = *tmem_slot;                    // S [0, 128); P over [0, 64); O [64, 128)
+  pdl_wait();                                          // Q/K/V (and offsets) of the previous kernels are visible
   pdl_trigger();                                       // after taking TMEM
+
+  // Item i is (sequence B-1-i/nh, head i%nh): the sequences are taken last to
+  // first, since the QKV GEMM before this kernel writes the rows of the last
+  // sequences last, so those are the ones still in L2.
+  auto seq_of = [&](int item) { return B - 1 - item / NH; };
+  auto seq_len = [&](int item) {
+    const int n = valid_len[seq_of(item)];
+    return n < 0 ? 0 : (n > S ? S : n);
+  };
+  // Tensor-map coordinates of row 0 of block t (0 = Q, 1 = K, 2 = V).
+  auto coord_x = [&](int t, int h) { return PACKED ? t * H + h * kD : 0; };
+  auto coord_y = [&](int t, int b, int h) { return PACKED ? offsets[b] : ((t * B + b) * NH + h) * S; };
 
   bool ok = true;
   if (warp == kSoftmaxWarps) {
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       prefetch_tmap(&tm_qkv);
-      mbar_arrive_expect_tx(qk_full, 2 * kTileBytes);
-      tma_load_2d(&tm_qkv, sbase + kQ, qk_full, coord_x(0), coord_y(0, 0));
-      tma_load_2d(&tm_qkv, sbase + kK, qk_full, coord_x(1), coord_y(1, 0));
-      mbar_arrive_expect_tx(v_full, kTileBytes);
-      tma_load_2d(&tm_qkv, sbase + kV, v_full, coord_x(2), coord_y(2, 0));
+      prefetch_tmap(&tm_ctx);
       constexpr uint32_t idesc_s = idesc_f16_f32(kRows, kRows);
       constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kRows, kD);
-      if (mbar_wait(qk_full, 0, kWaitLimitNs)) {
+      const int G = static_cast<int>(gridDim.x);
+      auto next_loaded = [&](int item) {                // items with no valid key load nothing
+        while (item < items && seq_len(item) == 0) item += G;
+        return item;
+      };
+      auto load_qk = [&](int item) {
+        const int b = seq_of(item), h = item % NH;
+        mbar_arrive_expect_tx(qk_full, 2 * kTileBytes);
+        tma_load_2d(&tm_qkv, sbase + kQ, qk_full, coord_x(0, h), coord_y(0, b, h));
+        tma_load_2d(&tm_qkv, sbase + kK, qk_full, coord_x(1, h), coord_y(1, b, h));
+      };
+      auto load_v = [&](int item) {
+        const int b = seq_of(item), h = item % NH;
+        mbar_arrive_expect_tx(v_full, kTileBytes);
+        tma_load_2d(&tm_qkv, sbase + kV, v_full, coord_x(2, h), coord_y(2, b, h));
+      };
+      // Copies issued and not yet waited for, with the parity they complete.
+      int qk_pending = -1, v_pending = -1;
+      int cur = next_loaded(blockIdx.x);
+      if (cur < items) {
+        load_qk(cur);
+        load_v(cur);
+        qk_pending = v_pending = 0;
+      }
+      for (int it = 0; cur < items; ++it) {
+        const uint32_t ph = it & 1;
+        const int n = seq_len(cur);
+        const int nxt = next_loaded(cur + G);
+        if (!(ok = mbar_wait(qk_full, ph, kWaitLimitNs))) break;
+        qk_pending = -1;
+        // S goes into the columns that held the previous item's O.
+        if (it > 0 && !(ok = mbar_wait(o_free, ph ^ 1, kWaitLimitNs))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           mma_f16_ss(tmem, smem_desc_sw128(sbase + kQ + kk * 32), smem_desc_sw128(sbase + kK + kk * 32), idesc_s,
                      kk > 0 ? 1u : 0u);
         mma_commit(s_full);
-        // P written by the softmax warps (which have read all of S and zeroed
-        // the V rows of keys >= n).
-        if (mbar_wait(p_full, 0, kWaitLimitNs) && mbar_wait(v_full, 0, kWaitLimitNs)) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk)
-            mma_f16_ss(tmem, smem_desc_sw128(sbase + kP + (kk >> 2) * kTileBytes + (kk & 3) * 32),
-                       desc_mn_sw128(sbase + kV + kk * 16 * 128), idesc_o, kk > 0 ? 1u : 0u);
-          mma_commit(o_full);
-        } else {
-          ok = false;
+        if (it > 0) {                                    // the V tile held the previous item's output rows
+          if (!(ok = mbar_wait(v_free, ph ^ 1, kWaitLimitNs))) break;
+          load_v(cur);
+          v_pending = ph;
         }
-      } else {
-        ok = false;
+        if (nxt < items) {                               // the next Q and K, once S = Q K^T has read these
+          if (!(ok = mbar_wait(s_full, ph, kWaitLimitNs))) break;
+          load_qk(nxt);
+          qk_pending = ph ^ 1;
+        }
+        // P written to TMEM by the softmax warps (which have read all of S and
+        // zeroed the V rows of keys in [n, n rounded up to 16)).
+        if (!(ok = mbar_wait(p_full, ph, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait(v_full, ph, kWaitLimitNs))) break;
+        v_pending = -1;
+        tc_fence_after();
+        const int ksteps = (n + 15) >> 4;                // key groups of 16 holding valid keys
+        for (int kk = 0; kk < ksteps; ++kk)
+          mma_f16_ts(tmem + kOCol, tmem + 8 * kk, desc_mn_sw128(sbase + kV + kk * 16 * 128), idesc_o,
+                     kk > 0 ? 1u : 0u);
+        mma_commit(o_full);
+        cur = nxt;
       }
-      mma_commit(drain);                               // every MMA issued here has completed
+      mma_commit(drain);                                 // every MMA issued here has completed
       mbar_wait(drain, 0, kWaitLimitNs);
-      if (!ok) {                                       // let the copies land before the CTA exits
-        mbar_wait(qk_full, 0, kWaitLimitNs);
-        mbar_wait(v_full, 0, kWaitLimitNs);
-      }
+      // After a failed wait, let the copies in flight land before the CTA exits.
+      if (qk_pending >= 0) mbar_wait(qk_full, qk_pending, kWaitLimitNs);
+      if (v_pending >= 0) mbar_wait(v_full, v_pending, kWaitLimitNs);
     }
   } else {
-    const int r = warp * 32 + lane;                    // query row = TMEM lane
+    const int r = warp * 32 + lane;                      // query row = TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int nchunks = (n + 31) >> 5;                 // 32-key chunks holding valid keys
-    uint8_t* prow = smem + kP + r * 128;
-    uint32_t sa[32], sb[32];                           // two chunks: one in use, one loading
-    uint64_t sum2 = 0;                                 // two partial row sums (0.0f, 0.0f)
-    if (n > 0) {
-      ok = warp_wait(s_full, 0);
-      if (ok) {
-        tc_fence_after();
-        // Pass 1: row max over the valid keys.  The next chunk's TMEM load is
-        // in flight while the current one is scanned.
-        float mx = -INFINITY;
-        tmem_ld_32x32b_x32_async(t_row, sa);
-#pragma unroll
-        for (int c = 0; c < kRows / 32; ++c) {
-          if (c < nchunks) {
-            uint32_t(&cur)[32] = (c & 1) ? sb : sa;
-            uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
-            tmem_wait_ld(cur);
-            if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_row + 32 * (c + 1), nxt);
-            const int lim = n - 32 * c;
-            if (lim >= 32) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(cur[i]));
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (i < lim) mx = fmaxf(mx, __uint_as_float(cur[i]));
-            }
+    const int unit = lane & 7;                           // plain stores: 8 lanes per 128-byte row
+    uint32_t sa[32], sb[32];                             // two chunks: one in use, one loading
+    int it = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+      const int b = seq_of(item), h = item % NH;
+      const int n = seq_len(item);
+      if (n == 0) {                                      // no valid key: ctx = 0 (packed: no rows)
+        if (!PACKED) {
+          __half* out = ctx + (size_t)b * S * H + h * kD;
+#pragma unroll 1
+          for (int k = 0; k < 8; ++k) {
+            const int rr = warp * 32 + k * 4 + (lane >> 3);
+            if (rr < S) *reinterpret_cast<uint4*>(out + (size_t)rr * H + unit * 8) = make_uint4(0, 0, 0, 0);
           }
         }
-        const uint64_t scale2 = f2_pack(score_scale_log2, score_scale_log2);
-        const uint64_t neg_m2 = f2_pack(-mx * score_scale_log2, -mx * score_scale_log2);
-        // Pass 2: P, its row sum, FP16 P into the swizzled tile (over Q and K);
-        // chunks past n get P = 0.
-        tmem_ld_32x32b_x32_async(t_row, sa);
+        continue;
+      }
+      const uint32_t ph = it & 1;
+      ++it;
+      const int nchunks = (n + 31) >> 5;                 // 32-key chunks holding valid keys
+      uint64_t sum2 = 0;                                 // two partial row sums (0.0f, 0.0f)
+      if (!(ok = warp_wait(s_full, ph))) break;
+      tc_fence_after();
+      // Pass 1: row max over the valid keys.  The next chunk's TMEM load is
+      // in flight while the current one is scanned.
+      float mx = -INFINITY;
+      tmem_ld_32x32b_x32_async(t_row, sa);
 #pragma unroll
-        for (int c = 0; c < kRows / 32; ++c) {
-          if (c < nchunks) {
-            uint32_t(&cur)[32] = (c & 1) ? sb : sa;
-            uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
-            tmem_wait_ld(cur);
-            if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_row + 32 * (c + 1), nxt);
-            const int lim = n - 32 * c;
-            if (lim >= 32)
-              p_chunk<false>(cur, 32, scale2, neg_m2, sum2, prow, c, r);
-            else
-              p_chunk<true>(cur, lim, scale2, neg_m2, sum2, prow, c, r);
+      for (int c = 0; c < kRows / 32; ++c) {
+        if (c < nchunks) {
+          uint32_t(&cur)[32] = (c & 1) ? sb : sa;
+          uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
+          tmem_wait_ld(cur);
+          if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_row + 32 * (c + 1), nxt);
+          const int lim = n - 32 * c;
+          if (lim >= 32) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(cur[i]));
           } else {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) store_p_unit(prow, 4 * c + u, r, make_uint4(0, 0, 0, 0));
+            for (int i = 0; i < 32; ++i)
+              if (i < lim) mx = fmaxf(mx, __uint_as_float(cur[i]));
           }
         }
-        // V rows of keys >= n: their P is 0, but a row the TMA box brought in
-        // from outside the sequence may hold non-finite data (0 * NaN = NaN in
-        // the MMA), so zero them.  Row r of the tile is key r.
-        if (n < kRows) {
-          ok = warp_wait(v_full, 0);
-          if (ok && r >= n) {
-            uint4* vrow = reinterpret_cast<uint4*>(smem + kV + r * 128);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) vrow[u] = make_uint4(0, 0, 0, 0);
-          }
-        }
-        fence_proxy_async_smem();                      // P (and zeroed V rows) visible to the tensor core
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
-        if (ok) ok = warp_wait(o_full, 0);
       }
-    }
-    if (ok) {
-      // Row r of O, scaled by 1/sum, as FP16 into the V tile (free once P V has
-      // completed): 128 bytes per row, 16-byte units swizzled by r & 7.
+      const uint64_t scale2 = f2_pack(score_scale_log2, score_scale_log2);
+      const uint64_t neg_m2 = f2_pack(-mx * score_scale_log2, -mx * score_scale_log2);
+      // Pass 2: P and its row sum; FP16 P of chunk c goes to columns
+      // [16c, 16c + 16), which hold scores this thread has already read.
+      tmem_ld_32x32b_x32_async(t_row, sa);
+#pragma unroll
+      for (int c = 0; c < kRows / 32; ++c) {
+        if (c < nchunks) {
+          uint32_t(&cur)[32] = (c & 1) ? sb : sa;
+          uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
+          tmem_wait_ld(cur);
+          if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_row + 32 * (c + 1), nxt);
+          const int lim = n - 32 * c;
+          if (lim >= 32)
+            p_chunk_tmem<false>(cur, 32, scale2, neg_m2, sum2, t_row + 16 * c);
+          else
+            p_chunk_tmem<true>(cur, lim, scale2, neg_m2, sum2, t_row + 16 * c);
+        }
+      }
+      // P V reads the keys of the 16-key groups holding valid keys.  Keys in
+      // [n, n16) have P = 0, but a V row the TMA box brought in from outside the
+      // sequence may hold non-finite data (0 * NaN = NaN in the MMA), so they
+      // are zeroed; those rows all lie in warp n / 32.  Row r of the tile is key r.
+      const int n16 = (n + 15) & ~15;
+      if (n < n16 && warp == (n >> 5)) {
+        if (!(ok = warp_wait(v_full, ph))) break;
+        if (r >= n && r < n16) {
+          uint4* vrow = reinterpret_cast<uint4*>(smem + kV + r * 128);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) vrow[u] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();                        // zeroed V rows visible to the tensor core
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      if (!(ok = warp_wait(o_full, ph))) break;
       tc_fence_after();
+      tmem_ld_32x32b_x32_async(t_row + kOCol, sa);
+      tmem_ld_32x32b_x32_async(t_row + kOCol + 32, sb);
+      tmem_wait_ld(sa);
+      tmem_wait_ld(sb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);                // the next S may overwrite O
+      // Row r of O, scaled by 1/sum, as FP16 into the V tile (free once P V has
+      // completed): 128 bytes per row, 16-byte units swizzled by r & 7, the
+      // layout of a 128-byte-swizzled TMA box.
       float s0, s1;
       f2_unpack(sum2, s0, s1);
-      const float l = s0 + s1;
-      const float inv = l > 0.f ? 1.f / l : 0.f;       // n == 0: ctx = 0
+      const float inv = 1.f / (s0 + s1);                 // n > 0: the sum holds P = 1 at the row max
       const uint64_t inv2 = f2_pack(inv, inv);
       uint8_t* orow = smem + kV + r * 128;
-      if (n > 0) {
-        tmem_ld_32x32b_x32_async(t_row, sa);
-        tmem_ld_32x32b_x32_async(t_row + 32, sb);
-        tmem_wait_ld(sa);
-        tmem_wait_ld(sb);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sa[i] = sb[i] = 0u;
-      }
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         const uint32_t(&sv)[32] = c ? sb : sa;
@@ -316,24 +394,38 @@ __global__ void __launch_bounds__(kThreads, 4)   // four CTAs per SM (TMEM 4 x 1
                       o0, o1);
             w[j] = cvt_half2(o0, o1);
           }
-          const int unit = 4 * c + u;
-          *reinterpret_cast<uint4*>(orow + 16 * (unit ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+          const int un = 4 * c + u;
+          *reinterpret_cast<uint4*>(orow + 16 * (un ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();                          // the rows visible to the TMA store
+      __syncwarp();
+      // The warp's 32 rows: one TMA store when all of them exist; else the rows
+      // that do, stored coalesced (8 lanes per 128-byte row, 4 rows per
+      // instruction).  The V tile is released once the rows have been read.
+      const int rows_exist = PACKED ? n : S;
+      const int row0 = PACKED ? offsets[b] : b * S;
+      if (warp * 32 + 32 <= rows_exist) {
+        if (lane == 0) {
+          tma_store_2d(&tm_ctx, sbase + kV + warp * 32 * 128, h * kD, row0 + warp * 32);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();
+        }
+      } else {
+        __half* out = ctx + (size_t)row0 * H + h * kD;
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k) {
+          const int rr = warp * 32 + k * 4 + (lane >> 3);
+          if (rr < rows_exist) {
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + kV + rr * 128 + 16 * (unit ^ (rr & 7)));
+            *reinterpret_cast<uint4*>(out + (size_t)rr * H + unit * 8) = v;
+          }
         }
       }
       __syncwarp();
-      // The warp's 32 rows, stored coalesced: 8 lanes per 128-byte row, 4 rows
-      // per instruction.
-      const int unit = lane & 7;
-#pragma unroll 1
-      for (int it = 0; it < 8; ++it) {
-        const int rr = warp * 32 + it * 4 + (lane >> 3);
-        if (rr < rows_exist) {
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + kV + rr * 128 + 16 * (unit ^ (rr & 7)));
-          const size_t out_row = PACKED ? (size_t)offsets[b] + rr : (size_t)b * S + rr;
-          *reinterpret_cast<uint4*>(ctx + out_row * H + h * kD + unit * 8) = v;
-        }
-      }
+      if (lane == 0) mbar_arrive(v_free);
     }
+    if (lane == 0) bulk_wait_group_all();                // this warp's TMA stores have completed
   }
 
   if (!ok) atomicCAS(status, 0, kStatusWaitTimeout);
@@ -700,9 +792,23 @@ cudaError_t launch_tc(const __half* qkv, const int32_t* vl, const int32_t* offse
     return launch_kernel(attention_tc_long_kernel<PACKED>, grid, dim3(lng::kThreads), lng::kSmemTotal, stream,
                          nullptr, 0, map, vl, offsets, ctx, B, S, NH, scale_log2, status);
   }
-  const dim3 grid(NH, B);
+  // Persistent: four CTAs per SM, the footprint the kernel is built for
+  // (launch bounds, shared memory and TMEM above).  The occupancy calculator
+  // reports one CTA per SM for this kernel, so it is not asked.
+  static const int resident = kCtasPerSm * device_sm_count();
+  const long long items = (long long)B * NH;
+  const dim3 grid((unsigned)(items < resident ? items : resident));
+  // ctx [B*S, H] (the packed layout uses its first T rows), stored in boxes
+  // of 32 rows x 64 halves with the 128-byte swizzle of the staged rows.
+  const cuuint64_t cdims[2] = {H, (cuuint64_t)B * S};
+  const cuuint64_t cstrides[1] = {H * 2};
+  const cuuint32_t cbox[2] = {kD, 32};
+  CUtensorMap cmap;
+  if (fn(&cmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ctx, cdims, cstrides, cbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   return launch_kernel(attention_tc_kernel<PACKED>, grid, dim3(kThreads), kSmemTotal, stream, nullptr, 0, map, vl,
-                       offsets, ctx, B, S, NH, scale_log2, status);
+                       offsets, ctx, B, S, NH, scale_log2, cmap, status);
 }
 
 }  // namespace
@@ -713,6 +819,7 @@ cudaError_t launch_attention_tc(const __half* qkv, const int32_t* valid_len, con
                                 int batch, int seq, int head_num, int* status, cudaStream_t stream) {
   if (batch <= 0 || batch > 65535 || head_num <= 0 || head_num > 65535 || !attention_tc_supported(kD, seq))
     return cudaErrorInvalidValue;
+  if (3ll * batch * head_num * seq > 0x7fffffffll) return cudaErrorInvalidValue;   // int32 tensor-map rows
   if (offsets) return launch_tc<true>(qkv, valid_len, offsets, ctx, batch, seq, head_num, status, stream);
   return launch_tc<false>(qkv, valid_len, nullptr, ctx, batch, seq, head_num, status, stream);
 }
