@@ -326,7 +326,7 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
 // ("Faster Transformer 优化原理") runs add-bias + residual + LayerNorm as a
 // separate kernel after the GEMM; here the GEMM writes the normalised row.
 //   Pass 1: each epilogue warp forms z = acc + bias + residual for its 32 rows
-//     x 128 columns (residual by TMA, as in kBiasResidStore), writes z back
+//     x 128 columns (residual by TMA, two chunks ahead), writes z back
 //     into the accumulator's TMEM columns and keeps per-row (mean, M2) of its
 //     128 values, merged chunk by chunk with the pairwise update of Chan,
 //     Golub and LeVeque (1979), which has no E[z^2] - E[z]^2 cancellation.
@@ -337,6 +337,10 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
 //     memory and merges all 2P of them in a fixed order.
 //   Pass 2: out = (z - mean) * rsqrt(M2 / N + eps) * gamma + beta, from TMEM,
 //     stored as FP16 through the staging buffers and TMA stores.
+// The accumulator is released only after pass 2.  Releasing it after pass 1
+// (z kept as FP16 in registers) was measured slower: the next tile's MMAs
+// then run under the whole epilogue, and their operand traffic through
+// shared memory slows every epilogue phase more than the overlap gains.
 // The statistics are double-buffered by tile parity: a pair writes buffer b
 // again only two tiles later, after every other pair has signalled the tile in
 // between, i.e. after they have read buffer b.
@@ -382,13 +386,19 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
     *reinterpret_cast<float4*>(par_s + 256 + i) = t;
   }
   auto buf_of = [&](int j) { return ws.stage + ((ws.seq + j) & 1u) * kStageChunkBytes; };
-  auto issue_res = [&](int j) {                // lane 0: residual chunk j, once every store has read its buffer
-    sm100::bulk_wait_group_read<0>();
+  auto issue_res = [&](int j) {                // lane 0: residual chunk j into buffer (seq + j) & 1
     const uint32_t bar = ws.res_bar + 8u * ((ws.seq + j) & 1u);
     sm100::mbar_arrive_expect_tx(bar, kStageChunkBytes);
     sm100::tma_load_2d(ws.tm_r, sm100::smem_u32(buf_of(j)), bar, col_begin + 32 * j, row0);
   };
-  if (lane == 0) issue_res(0);
+  // Residual chunks 0 and 1 before the accumulator is awaited (once the
+  // previous tile's stores have read both buffers); chunk j + 2 once chunk j's
+  // residual has been read out of its buffer.
+  if (lane == 0) {
+    sm100::bulk_wait_group_read<0>();
+    issue_res(0);
+    issue_res(1);
+  }
   int got = 0;
   if (lane == 0) got = wait_full() ? 1 : 0;
   got = __shfl_sync(0xffffffffu, got, 0);      // also orders the parameter staging before its use
@@ -405,7 +415,6 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
     uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
     sm100::tmem_wait_ld(cur);
     if (j + 1 < CHUNKS) sm100::tmem_ld_32x32b_x32_async(t_cols + 32 * (j + 1), nxt);
-    if (lane == 0 && j + 1 < CHUNKS) issue_res(j + 1);
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {          // bias: one 16-byte broadcast read per 4 columns
@@ -435,6 +444,10 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
       q4[i & 3] = fmaf(d, d, q4[i & 3]);
     }
     chan_merge(n, mean, m2, 32.0f, mc, (q4[0] + q4[1]) + (q4[2] + q4[3]));
+    if (j + 2 < CHUNKS) {
+      __syncwarp();                            // every lane has used the residual it read from the buffer
+      if (lane == 0) issue_res(j + 2);
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) cur[i] = __float_as_uint(v[i]);
     sm100::tmem_st_32x32b_x32(t_cols + 32 * j, cur);     // z replaces the accumulator
