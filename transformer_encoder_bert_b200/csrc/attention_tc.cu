@@ -103,37 +103,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __shfl_sync(0xffffffffu, got, 0) != 0;
 }
 
-// Stores 16-byte unit `unit` (0..15) of a 128-key FP16 row r of P: keys
-// 64a .. 64a+63 form atom a (rows of 128 bytes), units swizzled by r & 7.
-__device__ __forceinline__ void store_p_unit(uint8_t* prow, int unit, int r, uint4 v) {
-  *reinterpret_cast<uint4*>(prow + (unit >> 3) * kTileBytes + 16 * ((unit & 7) ^ (r & 7))) = v;
-}
-
-// P of 32 keys (chunk c of the row) from 32 raw scores: p = 2^(s*c2 - m*c2)
-// for the first `lim` keys, 0 for the rest; adds to the pair sum and writes
-// the FP16 values as four 16-byte units of the row.
-template <bool MASKED>
-__device__ __forceinline__ void p_chunk(const uint32_t (&sv)[32], int lim, uint64_t scale2, uint64_t neg_m2,
-                                        uint64_t& sum2, uint8_t* prow, int c, int r) {
-  uint32_t pk[16];
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const uint64_t t = f2_fma(f2_pack(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), scale2, neg_m2);
-    float t0, t1;
-    f2_unpack(t, t0, t1);
-    float p0 = ex2(t0), p1 = ex2(t1);
-    if (MASKED) {
-      p0 = i < lim ? p0 : 0.f;
-      p1 = i + 1 < lim ? p1 : 0.f;
-    }
-    sum2 = f2_add(sum2, f2_pack(p0, p1));
-    pk[i >> 1] = cvt_half2(p0, p1);
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    store_p_unit(prow, 4 * c + u, r, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
-}
-
 // P of 32 keys (chunk c of the row) from 32 raw scores: p = 2^(s*c2 - m*c2)
 // for the first `lim` keys, 0 for the rest; adds to the pair sum and writes
 // the FP16 values into TMEM as 16 columns (two keys per column) of this lane.
@@ -439,52 +408,62 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // ---------------------------------------------------------------------------
 // Sequences longer than one key block (seq > 128): the same per-row softmax
-// over 128-key blocks with a running maximum (online softmax).  One CTA per
-// (sequence, head, 128 query rows), 160 threads, two CTAs per SM so that one
-// CTA's loads overlap the other's softmax:
+// over key blocks of 32 with a reference maximum (online softmax).  One CTA per
+// (sequence, head, 128 query rows), 160 threads, four CTAs per SM:
 //   warps 0..3  softmax: thread r owns query row r = TMEM lane r.  For key
 //               block j it reads its row of S_j = Q K_j^T from TMEM, writes
-//               P_j = exp(S_j/sqrt(d) - m) (FP16, swizzled K-major) and adds its
-//               row sum to l.  m is a reference maximum: it moves only when a
-//               block's maximum exceeds it by more than 2^8 in the exponent, and
-//               then O (in TMEM) and l are scaled by exp(m_old - m_new) before
-//               the next P V accumulates.  At the end it stores O / l.
-//   warp 4      one thread issues every TMA load (Q once; K blocks through a
-//               two-stage ring; V one block at a time) and every MMA:
-//               S_j into TMEM columns [0, 128), O += P_j V_j into [128, 192).
-// S_{j+1} is issued right after P_j V_j, so the next scores are ready when the
-// softmax warps finish block j.  Key blocks past n are never loaded; in the
-// last block, keys >= n get weight 0 and their V rows are zeroed.
+//               P_j = exp(S_j/sqrt(d) - m) as FP16 back into S_j's columns and
+//               adds its row sum to l.  m is a reference maximum: it moves only
+//               when a block's maximum exceeds it by more than 2^8 in the
+//               exponent, and then O (in TMEM) and l are scaled by
+//               exp(m_old - m_new) before the next P V accumulates.  At the end
+//               it stores O / l.
+//   warp 4      one thread issues every TMA load (Q once; K and V blocks
+//               through four-stage rings) and every MMA:
+//                 S_j = Q K_j^T   M=128, N=32, K=64 into S buffer j % 2
+//                 O += P_j V_j    M=128, N=64, K=16 per 16-key group (A = P_j
+//                                 read from TMEM; B = V_j MN-major from smem)
+// The two S buffers let S_{j+1} be computed while the softmax warps work on
+// S_j, and S_{j+2} goes into S_j's buffer as soon as P_j V_j has read P_j.
+// TMEM (128 columns): S buffers at [0, 32) and [32, 64), P_j (two halves per
+// column) over the first 16 columns of its buffer, O at [64, 128).  Key blocks
+// past n are never loaded; in the last block, keys >= n get weight 0 and the
+// V rows of keys in [n, n rounded up to 16) are zeroed.
 namespace lng {
 constexpr int kThreads = 32 * (kSoftmaxWarps + 1);
+constexpr int kBK = 32;                                     // keys per block
+constexpr int kStages = 4;                                  // K and V ring depth
+constexpr int kKVBytes = kBK * kD * 2;                      // 4 KB: 32 keys x 64 halves
 constexpr int kQ = 0;                                       // Q tile, later the output rows
-constexpr int kK = kTileBytes;                              // K of stage st (two stages)
-constexpr int kV = 3 * kTileBytes;                          // V of the current block
-constexpr int kP = 4 * kTileBytes;                          // P: two 64-key atoms
-constexpr int kBars = 6 * kTileBytes;
-// q_full, k_full[2], k_empty[2], v_full, v_empty, s_full, p_full, o_full, drain
-constexpr int kNumBars = 11;
+constexpr int kK = kTileBytes;                              // K stages
+constexpr int kV = kK + kStages * kKVBytes;                 // V stages
+constexpr int kBars = kV + kStages * kKVBytes;
+// q_full, k_full[4], v_full[4], s_full[2], p_full[2], o_done, drain
+constexpr int kNumBars = 15;
 constexpr int kSlot = kBars + kNumBars * 8;
 constexpr int kSmemTotal = 1024 + kSlot + 16;
-constexpr int kTmemCols = 256;
-constexpr int kOCol = 128;
+constexpr int kTmemCols = 128;
+constexpr int kOCol = 2 * kBK;
+constexpr int kCtasPerSm = 4;                               // TMEM 4 x 128 columns
 constexpr float kRescaleLog2 = 8.f;                         // P < 2^8 between rescales
-static_assert(2 * (kSmemTotal + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(kCtasPerSm * (kSmemTotal + 1024) <= 228 * 1024, "four CTAs per SM");
 }  // namespace lng
 
 template <bool PACKED>
-__global__ void __launch_bounds__(lng::kThreads, 2)
-    attention_tc_long_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int32_t* __restrict__ valid_len,
-                             const int32_t* __restrict__ offsets, __half* __restrict__ ctx, int B, int S, int NH,
-                             float score_scale_log2, int* __restrict__ status) {
+__global__ void __launch_bounds__(lng::kThreads, lng::kCtasPerSm)
+    attention_tc_long_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_kv,
+                             const int32_t* __restrict__ valid_len, const int32_t* __restrict__ offsets,
+                             __half* __restrict__ ctx, int B, int S, int NH, float score_scale_log2,
+                             int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + lng::kBars;
-  const uint32_t q_full = bar0, v_full = bar0 + 40, v_empty = bar0 + 48, s_full = bar0 + 56, p_full = bar0 + 64,
-                 o_full = bar0 + 72, drain = bar0 + 80;
+  const uint32_t q_full = bar0, o_done = bar0 + 104, drain = bar0 + 112;
   auto k_full = [&](int st) { return bar0 + 8 + 8 * st; };
-  auto k_empty = [&](int st) { return bar0 + 24 + 8 * st; };
+  auto v_full = [&](int st) { return bar0 + 40 + 8 * st; };
+  auto s_full = [&](int bf) { return bar0 + 72 + 8 * bf; };
+  auto p_full = [&](int bf) { return bar0 + 88 + 8 * bf; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lng::kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -503,13 +482,16 @@ __global__ void __launch_bounds__(lng::kThreads, 2)
       *reinterpret_cast<uint4*>(ctx + (row0 + q0 + (i >> 3)) * H + h * kD + (i & 7) * 8) = make_uint4(0, 0, 0, 0);
     return;
   }
-  const int nb = (n + kRows - 1) / kRows;              // key blocks holding valid keys
+  const int nb = (n + lng::kBK - 1) / lng::kBK;        // key blocks holding valid keys
 
   auto coord_x = [&](int t) { return PACKED ? t * H + h * kD : 0; };
   auto coord_y = [&](int t, int s) { return PACKED ? offsets[b] + s : ((t * B + b) * NH + h) * S + s; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < lng::kNumBars; ++i) mbar_init(bar0 + 8 * i, bar0 + 8 * i == p_full ? kSoftmaxWarps : 1);
+    for (int i = 0; i < lng::kNumBars; ++i) {
+      const uint32_t bar = bar0 + 8 * i;
+      mbar_init(bar, (bar == p_full(0) || bar == p_full(1)) ? kSoftmaxWarps : 1);
+    }
     fence_barrier_init();
   }
   if (warp == kSoftmaxWarps) {
@@ -526,107 +508,107 @@ __global__ void __launch_bounds__(lng::kThreads, 2)
   if (warp == kSoftmaxWarps) {
     if (lane == 0) {
       prefetch_tmap(&tm_qkv);
+      prefetch_tmap(&tm_kv);
+      // K_j and V_j go to stage j % kStages (one key block per box, same rows as the Q map).
       auto load_k = [&](int j) {
-        const int st = j & 1;
-        mbar_arrive_expect_tx(k_full(st), kTileBytes);
-        tma_load_2d(&tm_qkv, sbase + lng::kK + st * kTileBytes, k_full(st), coord_x(1), coord_y(1, j * kRows));
+        const int st = j % lng::kStages;
+        mbar_arrive_expect_tx(k_full(st), lng::kKVBytes);
+        tma_load_2d(&tm_kv, sbase + lng::kK + st * lng::kKVBytes, k_full(st), coord_x(1), coord_y(1, j * lng::kBK));
       };
       auto load_v = [&](int j) {
-        mbar_arrive_expect_tx(v_full, kTileBytes);
-        tma_load_2d(&tm_qkv, sbase + lng::kV, v_full, coord_x(2), coord_y(2, j * kRows));
+        const int st = j % lng::kStages;
+        mbar_arrive_expect_tx(v_full(st), lng::kKVBytes);
+        tma_load_2d(&tm_kv, sbase + lng::kV + st * lng::kKVBytes, v_full(st), coord_x(2), coord_y(2, j * lng::kBK));
       };
       mbar_arrive_expect_tx(q_full, kTileBytes);
       tma_load_2d(&tm_qkv, sbase + lng::kQ, q_full, coord_x(0), coord_y(0, q0));
-      load_k(0);
-      if (nb > 1) load_k(1);
-      load_v(0);
-      int k_loaded = nb > 1 ? 2 : 1, v_loaded = 1;
-      constexpr uint32_t idesc_s = idesc_f16_f32(kRows, kRows);
+      for (int j = 0; j < nb && j < lng::kStages; ++j) {
+        load_k(j);
+        load_v(j);
+      }
+      int loaded = nb < lng::kStages ? nb : lng::kStages;   // K and V blocks requested
+      constexpr uint32_t idesc_s = idesc_f16_f32(kRows, lng::kBK);
       constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kRows, kD);
-      auto issue_s = [&](int j) {                      // S = Q K_j^T, then K stage j & 1 is free
-        const int st = j & 1;
+      auto issue_s = [&](int j) {                      // S_j into buffer j % 2
+        const int st = j % lng::kStages;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          mma_f16_ss(tmem, smem_desc_sw128(sbase + lng::kQ + kk * 32),
-                     smem_desc_sw128(sbase + lng::kK + st * kTileBytes + kk * 32), idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        mma_commit(k_empty(st));
+          mma_f16_ss(tmem + (j & 1) * lng::kBK, smem_desc_sw128(sbase + lng::kQ + kk * 32),
+                     smem_desc_sw128(sbase + lng::kK + st * lng::kKVBytes + kk * 32), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(s_full(j & 1));
       };
-      ok = mbar_wait(q_full, 0, kWaitLimitNs) && mbar_wait(k_full(0), 0, kWaitLimitNs);
-      if (ok) {
+      ok = mbar_wait(q_full, 0, kWaitLimitNs);
+      for (int j = 0; j < 2 && j < nb && ok; ++j) {
+        if (!(ok = mbar_wait(k_full(j), 0, kWaitLimitNs))) break;
         tc_fence_after();
-        issue_s(0);
+        issue_s(j);
       }
       for (int j = 0; j < nb && ok; ++j) {
+        const int st = j % lng::kStages;
+        const uint32_t rph = (j / lng::kStages) & 1;
         // P_j is written (so S_j has been read and O rescaled) and V_j has landed.
-        if (!mbar_wait(p_full, j & 1, kWaitLimitNs) || !mbar_wait(v_full, j & 1, kWaitLimitNs)) { ok = false; break; }
+        if (!(ok = mbar_wait(p_full(j & 1), (j >> 1) & 1, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait(v_full(st), rph, kWaitLimitNs))) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)        // O += P_j V_j
-          mma_f16_ss(tmem + lng::kOCol, smem_desc_sw128(sbase + lng::kP + (kk >> 2) * kTileBytes + (kk & 3) * 32),
-                     desc_mn_sw128(sbase + lng::kV + kk * 16 * 128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(o_full);
-        mma_commit(v_empty);
-        if (j + 1 < nb) {
-          if (!mbar_wait(k_full((j + 1) & 1), ((j + 1) >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(j + 1);
-        }
-        if (j + 2 < nb) {                              // K_{j+2} into the stage S_j has finished with
-          if (!mbar_wait(k_empty(j & 1), (j >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
-          load_k(j + 2);
-          k_loaded = j + 3;
-        }
-        if (j + 1 < nb) {                              // V_{j+1} once P_j V_j has read V_j
-          if (!mbar_wait(v_empty, j & 1, kWaitLimitNs)) { ok = false; break; }
-          load_v(j + 1);
-          v_loaded = j + 2;
+        const int lim_blk = min(n - j * lng::kBK, lng::kBK);
+        const int ksteps = (lim_blk + 15) >> 4;
+        for (int kk = 0; kk < ksteps; ++kk)            // O += P_j V_j
+          mma_f16_ts(tmem + lng::kOCol, tmem + (j & 1) * lng::kBK + 8 * kk,
+                     desc_mn_sw128(sbase + lng::kV + st * lng::kKVBytes + kk * 16 * 128), idesc_o,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(o_done);
+        if (j + 2 < nb) {
+          // P_j V_j has read P_j (S_j's buffer is free) and V_j (its stage is free);
+          // S_j, long complete, has read K_j.
+          if (!(ok = mbar_wait(o_done, j & 1, kWaitLimitNs))) break;
+          if (j + lng::kStages < nb) {
+            load_k(j + lng::kStages);
+            load_v(j + lng::kStages);
+            loaded = j + lng::kStages + 1;
+          }
+          if (j + 2 < nb) {
+            const int st2 = (j + 2) % lng::kStages;
+            if (!(ok = mbar_wait(k_full(st2), ((j + 2) / lng::kStages) & 1, kWaitLimitNs))) break;
+            tc_fence_after();
+            issue_s(j + 2);
+          }
         }
       }
       mma_commit(drain);                               // every MMA issued here has completed
       mbar_wait(drain, 0, kWaitLimitNs);
       if (!ok) {                                       // let the copies land before the CTA exits
         mbar_wait(q_full, 0, kWaitLimitNs);
-        for (int j = k_loaded > 2 ? k_loaded - 2 : 0; j < k_loaded; ++j)
-          mbar_wait(k_full(j & 1), (j >> 1) & 1, kWaitLimitNs);
-        mbar_wait(v_full, (v_loaded - 1) & 1, kWaitLimitNs);
+        for (int j = loaded > lng::kStages ? loaded - lng::kStages : 0; j < loaded; ++j) {
+          mbar_wait(k_full(j % lng::kStages), (j / lng::kStages) & 1, kWaitLimitNs);
+          mbar_wait(v_full(j % lng::kStages), (j / lng::kStages) & 1, kWaitLimitNs);
+        }
       }
     }
   } else {
     const int r = warp * 32 + lane;                    // query row = TMEM lane
-    const uint32_t t_s = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t t_o = t_s + lng::kOCol;
-    uint8_t* prow = smem + lng::kP + r * 128;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t t_o = t_lane + lng::kOCol;
     const uint64_t scale2 = f2_pack(score_scale_log2, score_scale_log2);
     uint32_t sa[32], sb[32];
     uint64_t sum2 = 0;                                 // two partial row sums (0.0f, 0.0f)
     float m_ref = 0.f;                                 // the max that P, O and l are taken against
     for (int j = 0; j < nb && ok; ++j) {
-      ok = warp_wait(s_full, j & 1);
-      if (!ok) break;
+      const uint32_t t_s = t_lane + (j & 1) * lng::kBK;
+      if (!(ok = warp_wait(s_full(j & 1), (j >> 1) & 1))) break;
       tc_fence_after();
-      const int lim_blk = min(n - j * kRows, kRows);   // valid keys in this block (>= 1)
-      const int nchunks = (lim_blk + 31) >> 5;
-      // Pass 1: block max over the valid keys.
+      const int lim_blk = min(n - j * lng::kBK, lng::kBK);   // valid keys in this block (>= 1)
+      // The block's 32 scores of this row in registers.
+      tmem_ld_32x32b_x32(t_s, sa);
       float bmax = -INFINITY;
-      tmem_ld_32x32b_x32_async(t_s, sa);
+      if (lim_blk >= lng::kBK) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kRows / 32; ++c) {
-        if (c < nchunks) {
-          uint32_t(&cur)[32] = (c & 1) ? sb : sa;
-          uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
-          tmem_wait_ld(cur);
-          if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_s + 32 * (c + 1), nxt);
-          const int lim = lim_blk - 32 * c;
-          if (lim >= 32) {
+        for (int i = 0; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sa[i]));
+        bmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, __uint_as_float(cur[i]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (i < lim) bmax = fmaxf(bmax, __uint_as_float(cur[i]));
-          }
-        }
+        for (int i = 0; i < 32; ++i)
+          if (i < lim_blk) bmax = fmaxf(bmax, __uint_as_float(sa[i]));
       }
       // Every P, and every term of O and l, is taken against the same reference
       // m, so O / l is the softmax-weighted sum whatever m is; m moves (and O and
@@ -640,58 +622,48 @@ __global__ void __launch_bounds__(lng::kThreads, 2)
         m_ref = bmax;
         moved = true;
       }
-      if (j > 0) {                                     // P_{j-1} V_{j-1} is done: P may be rewritten
-        ok = warp_wait(o_full, (j - 1) & 1);
-        if (!ok) break;
+      if (__any_sync(0xffffffffu, moved)) {            // O *= alpha (alpha = 1 on rows that keep theirs)
+        if (!(ok = warp_wait(o_done, (j - 1) & 1))) break;   // P_{j-1} V_{j-1} has completed
         tc_fence_after();
-        if (__any_sync(0xffffffffu, moved)) {          // O *= alpha (alpha = 1 on rows that keep theirs)
+        uint32_t oa[32];
 #pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            tmem_ld_32x32b_x32(t_o + 32 * half, sa);
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld_32x32b_x32(t_o + 32 * half, oa);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sa[i] = __float_as_uint(__uint_as_float(sa[i]) * alpha);
-            tmem_st_32x32b_x32(t_o + 32 * half, sa);
-          }
+          for (int i = 0; i < 32; ++i) oa[i] = __float_as_uint(__uint_as_float(oa[i]) * alpha);
+          tmem_st_32x32b_x32(t_o + 32 * half, oa);
         }
-        sum2 = f2_mul(sum2, f2_pack(alpha, alpha));
       }
+      sum2 = f2_mul(sum2, f2_pack(alpha, alpha));
       const uint64_t neg_m2 = f2_pack(-m_ref * score_scale_log2, -m_ref * score_scale_log2);
-      // Pass 2: P_j, its row sum, FP16 P into the swizzled tile.
-      tmem_ld_32x32b_x32_async(t_s, sa);
+      // P_j and its row sum; FP16 P goes to the first 16 columns of S_j's
+      // buffer, which hold scores this thread has already read.
+      if (lim_blk >= lng::kBK) {
+        p_chunk_tmem<false>(sa, 32, scale2, neg_m2, sum2, t_s);
+      } else {
+        p_chunk_tmem<true>(sa, lim_blk, scale2, neg_m2, sum2, t_s);
+        // V rows of keys in [lim_blk, lim_blk rounded up to 16) are read by
+        // P V; a row the TMA box brought in from outside the sequence may hold
+        // non-finite data (0 * NaN = NaN in the MMA), so zero them.  Those rows
+        // of the 32-row V tile are rows of warp 0.
+        const int n16 = (lim_blk + 15) & ~15;
+        if (lim_blk < n16 && warp == 0) {
+          if (!(ok = warp_wait(v_full(j % lng::kStages), (j / lng::kStages) & 1))) break;
+          if (r >= lim_blk && r < n16) {
+            uint4* vrow = reinterpret_cast<uint4*>(smem + lng::kV + (j % lng::kStages) * lng::kKVBytes + r * 128);
 #pragma unroll
-      for (int c = 0; c < kRows / 32; ++c) {
-        if (c < nchunks) {
-          uint32_t(&cur)[32] = (c & 1) ? sb : sa;
-          uint32_t(&nxt)[32] = (c & 1) ? sa : sb;
-          tmem_wait_ld(cur);
-          if (c + 1 < nchunks) tmem_ld_32x32b_x32_async(t_s + 32 * (c + 1), nxt);
-          const int lim = lim_blk - 32 * c;
-          if (lim >= 32)
-            p_chunk<false>(cur, 32, scale2, neg_m2, sum2, prow, c, r);
-          else
-            p_chunk<true>(cur, lim, scale2, neg_m2, sum2, prow, c, r);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) store_p_unit(prow, 4 * c + u, r, make_uint4(0, 0, 0, 0));
+            for (int u = 0; u < 8; ++u) vrow[u] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();                    // zeroed V rows visible to the tensor core
         }
       }
-      // Last, partial block: V rows of keys >= n may hold non-finite data from
-      // outside the sequence (0 * NaN = NaN in the MMA), so zero them.
-      if (lim_blk < kRows) {
-        ok = warp_wait(v_full, j & 1);
-        if (ok && r >= lim_blk) {
-          uint4* vrow = reinterpret_cast<uint4*>(smem + lng::kV + r * 128);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) vrow[u] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      fence_proxy_async_smem();                        // P (and zeroed V rows) visible to the tensor core
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full(j & 1));
     }
     if (ok) {
-      ok = warp_wait(o_full, (nb - 1) & 1);
+      ok = warp_wait(o_done, (nb - 1) & 1);
       if (ok) {
         tc_fence_after();
         tmem_ld_32x32b_x32_async(t_o, sa);
@@ -702,11 +674,10 @@ __global__ void __launch_bounds__(lng::kThreads, 2)
     }
     if (ok) {
       // Row r of O / l as FP16 into the Q tile (its last reader, the MMA of
-      // S_{nb-1}, has completed), then coalesced stores.
+      // the last S, has completed), then coalesced stores.
       float s0, s1;
       f2_unpack(sum2, s0, s1);
-      const float l = s0 + s1;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = 1.f / (s0 + s1);               // n >= 1: the sum holds P = 1 at the first block's max
       uint8_t* orow = smem + lng::kQ + r * 128;
 #pragma unroll
       for (int unit = 0; unit < 8; ++unit) {
@@ -788,9 +759,17 @@ cudaError_t launch_tc(const __half* qkv, const int32_t* vl, const int32_t* offse
     return cudaErrorInvalidValue;
   const float scale_log2 = kLog2e / sqrtf((float)kD);
   if (S > kRows) {
+    // K and V blocks through a second map over the same rows, with boxes of
+    // one key block.
+    const cuuint32_t kvbox[2] = {kD, lng::kBK};
+    CUtensorMap kvmap;
+    if (fn(&kvmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(qkv), dims, strides, kvbox, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((S + kRows - 1) / kRows), NH, B);
     return launch_kernel(attention_tc_long_kernel<PACKED>, grid, dim3(lng::kThreads), lng::kSmemTotal, stream,
-                         nullptr, 0, map, vl, offsets, ctx, B, S, NH, scale_log2, status);
+                         nullptr, 0, map, kvmap, vl, offsets, ctx, B, S, NH, scale_log2, status);
   }
   // Persistent: four CTAs per SM, the footprint the kernel is built for
   // (launch bounds, shared memory and TMEM above).  The occupancy calculator
