@@ -346,6 +346,24 @@ def test_packed_forward_matches_oracle_and_zeroes_padding(seq, lo, hi, L):
     assert enc.device_status() == 0
 
 
+@pytest.mark.parametrize("seq", [128, 100], ids=str)
+def test_packed_forward_many_attention_items(seq):
+    """Padding removal with more (sequence, head) items than the persistent
+    tcgen05 attention keeps resident (64 x 12 = 768): empty sequences (no rows
+    in the packed layout) among ragged ones; one layer against the oracle, and
+    the padded rows zero."""
+    sh = EI.EncoderShape(12, 64, 3072, 1)
+    inp = EI.make_inputs(EI.Workload("packed-items", sh, 64, seq, "fp16", 0, seq, seed=seq))
+    inp.valid_len[::9] = 0
+    enc = encoder_from_inputs(inp)
+    enc.set_packing(True)
+    got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+    m = valid_mask(inp.valid_len, seq)
+    assert np.all(got[~m] == 0)
+    _check(got, _oracle(inp), inp.valid_len, seq, FP16_LAYER_REL_L2)
+    assert enc.device_status() == 0
+
+
 PACKED_FULL_SIZE = [
     ("bert-base-s32", 512, None, 4),
     ("bert-base", 256, 128, 3),

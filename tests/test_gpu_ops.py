@@ -302,6 +302,36 @@ def test_attention_mma_sync_path_for_long_sequences(batch, seq):
     assert rel_l2(got, ref) < ATTN_REL_L2
 
 
+@pytest.mark.parametrize("seq", [128, 96, 80], ids=str)
+def test_attention_tc_items_beyond_the_resident_grid(seq):
+    """64 < seq <= 128: the persistent tcgen05 kernel runs about four CTAs per
+    SM, each taking (sequence, head) items in turn and loading the next item's
+    Q, K and V while it computes the current one.  64 sequences x 12 heads =
+    768 items, more than one round; lengths 0 (zero rows), 1, multiples of 16
+    and their neighbours, and seq itself.  Every row of every item against the
+    oracle; a second call gives the same bits."""
+    shape = (12, 64, 3072)
+    nh, d, _ = shape
+    batch = 64
+    wl, inp, enc, x64, vl, lw = _setup(shape, batch, seq)
+    qkv = EI.random_array((3, batch, nh, seq, d), "fp16", seed=seq)
+    base = [0, 1, 15, 16, 17, 31, 32, 33, 47, 63, 64, 65, seq - 1, seq]
+    vlen = np.array([base[i % len(base)] if i % 3 else (i * 37) % (seq + 1) for i in range(batch)], np.int32)
+    ctx = empty_dev((batch * seq, nh * d), "fp16")
+    enc.op_attention(to_dev(qkv), to_dev(vlen), ctx, batch, seq)
+    got = to_host(ctx).reshape(batch, seq, nh * d)
+    ref = O.attention(qkv.astype(np.float64), vlen)
+    assert np.all(np.isfinite(got))
+    for b in np.nonzero(vlen == 0)[0]:
+        assert np.all(got[b] == 0)
+    assert rel_l2(got, ref) < ATTN_REL_L2
+    assert max_abs(got, ref) < 4 * _ulp_bound(ref)
+    ctx2 = empty_dev((batch * seq, nh * d), "fp16")
+    enc.op_attention(to_dev(qkv), to_dev(vlen), ctx2, batch, seq)
+    assert np.array_equal(to_host(ctx2).reshape(batch, seq, nh * d), got)
+    assert enc.device_status() == 0
+
+
 @pytest.mark.parametrize("batch,seq,lens", [
     (3, 300, [300, 129, 1]),          # 3 query blocks: the second CTA's upper block lies past seq
     (2, 256, [256, 128]),             # key blocks exactly full; one block only
