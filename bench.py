@@ -625,7 +625,7 @@ def run_decoder(args, rank: int, world: int, local_rank: int):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "tgt_seq": wl.tgt_seq, "mem_seq": wl.mem_seq,
                        "layers": sh.num_layers, "l2": "flushed before every timed step (256 MiB write)",
-                       "launch": "enc_decoder_forward per step (12 launches per layer)"},
+                       "launch": "enc_decoder_forward per step (9 to 12 launches per layer)"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                          "traffic": None, "kernel": "whole decoder forward",
                          "peak_source": f"{peak_src} burst bf16 matmul"},

@@ -370,8 +370,10 @@ ENC_API enc_status enc_decoder_create(int head_num, int size_per_head, int ffn_d
  *   mem_len:  device int32 [batch], clamped to [0, mem_seq] on device;
  *   out:      device [batch, tgt_seq, H]; must not overlap y.
  * 16-byte-aligned buffers; the workspace grows like enc_forward's.  12 kernel
- * launches per layer.  Asynchronous; host checks fail before anything is
- * enqueued. */
+ * launches per layer, 9 where the three bias + residual + LayerNorm steps run
+ * in their GEMMs' epilogues (the encoder's rule and options: 2-CTA tiles,
+ * hidden size <= 768 by default).  Asynchronous; host checks fail before
+ * anything is enqueued. */
 ENC_API enc_status enc_decoder_forward(enc_t h, const void* y, const int32_t* tgt_len, const void* mem,
                                        const int32_t* mem_len, void* out, int batch, int tgt_seq, int mem_seq,
                                        enc_stream_t stream);

@@ -52,6 +52,37 @@ def test_decoder_matches_oracle(nh, d, F, L, B, T, S):
     assert dec.device_status() == 0
 
 
+def test_decoder_fused_layernorm_gemms_at_size():
+    """Enough target tokens (32 x 128) for the 2-CTA tiles: the three bias +
+    residual + LayerNorm steps run in their GEMMs' epilogues (row statistics
+    exchanged across the cluster), 9 launches per layer; sampled sequences
+    against the oracle, and against the same decoder with both fusions off."""
+    sh = EI.EncoderShape(12, 64, 3072, 1)
+    B, T, S = 32, 128, 96
+    wl = EI.DecoderWorkload("dec-fused", sh, B, T, S, "fp16", T // 2, T, S // 2, S, ln_affine_random=True, seed=7)
+    inp = EI.make_decoder_inputs(wl)
+    dec = _decoder(inp)
+    n0 = dec.launch_count()
+    got = _run(dec, inp)
+    assert dec.launch_count() - n0 == 9
+    pick = [0, 1, B - 1]
+    sub = EI.make_decoder_inputs(wl)
+    sub.y, sub.mem = inp.y[pick], inp.mem[pick]
+    sub.tgt_len, sub.mem_len = inp.tgt_len[pick], inp.mem_len[pick]
+    ref = _oracle(sub)
+    m = valid_mask(sub.tgt_len, T)
+    assert rel_l2(got[pick], ref, m) < FP16_LAYER_REL_L2
+    assert max_abs(got[pick], ref, m) < FP16_LAYER_MAX_ABS
+    dec.set_option("ln_fuse_out_proj", 0)
+    dec.set_option("ln_fuse_ffn2", 0)
+    n0 = dec.launch_count()
+    unfused = _run(dec, inp)
+    assert dec.launch_count() - n0 == 12
+    mall = valid_mask(inp.tgt_len, T)
+    assert rel_l2(got, unfused, mall) < FP16_LAYER_REL_L2
+    assert dec.device_status() == 0
+
+
 def test_decoder_empty_target_and_memory_and_tanh_gelu():
     sh = EI.EncoderShape(12, 64, 3072, 2)
     wl = EI.DecoderWorkload("dec-empty", sh, 4, 40, 50, "fp16", 1, 40, 1, 50, seed=3)

@@ -343,6 +343,13 @@ class Decoder:
     def set_gelu(self, form: str):
         _check(self.lib.enc_set_gelu(self.handle, {"erf": 0, "tanh": 1}[form]))
 
+    def set_option(self, name: str, value):
+        """One kernel-path switch (OPTION_CODES, enc_option in include/enc.h)."""
+        _check(self.lib.enc_set_option(self.handle, OPTION_CODES[name], int(value)))
+
+    def launch_count(self) -> int:
+        return int(self.lib.enc_launch_count(self.handle))
+
     def forward(self, y, tgt_len, mem, mem_len, out=None, stream=None):
         """y: CUDA [B, T, H] FP16; mem: CUDA [B, S, H] FP16; lengths: CUDA int32 [B]."""
         import torch

@@ -95,7 +95,8 @@ struct LayerDev {
 struct DecLayerDev {
   void *w_qkv, *w_o, *w_q2, *w_kv2, *w_o2, *w_ff1, *w_ff2;
   float *b_qkv, *b_o, *b_q2, *b_kv2, *b_o2, *b_ff1, *b_ff2;
-  __half *ln_g[3], *ln_b[3];
+  __half *ln_g[3], *ln_b[3];                 // FP16 (LayerNorm kernel)
+  float *ln_gf[3], *ln_bf[3];                // FP32 (LayerNorm fused into a GEMM epilogue)
   CUtensorMap tm_qkv[2], tm_o[2], tm_q2[2], tm_kv2[2], tm_o2[2], tm_ff1[2], tm_ff2[2];
 };
 
@@ -1493,10 +1494,18 @@ enc_status dec_layer(enc_handle* h, int l, const void* yin, void* yout, const in
   const __half* qkv = static_cast<const __half*>(w.qkv);
   if ((s = dec_attention(h, qkv, qkv + hd * T, qkv + 2 * hd * T, tgt_len, w.ctx, B, T, T, true, st)) != ENC_OK)
     return s;
-  if ((s = run_gemm(h, w.ctx, Mt, H, L.w_o, L.tm_o, H, enc::Epi::kBiasResidStore, L.b_o, w.z, {}, st, nullptr,
-                    yin)) != ENC_OK)
-    return s;
-  if ((s = dec_ln(h, w.z, L.ln_g[0], L.ln_b[0], w.h1, Mt, st)) != ENC_OK) return s;
+  // GEMM + bias + residual + LayerNorm i: in the GEMM epilogue where the
+  // encoder fuses it (2-CTA tiles, the same options), else through z and the
+  // LayerNorm kernel.
+  auto resid_ln = [&](const void* A, int K, void* W, const CUtensorMap* tm, const float* b, const void* resid, int i,
+                      int which, void* out) -> enc_status {
+    if (ln_fused(h, Mt, which))
+      return run_gemm(h, A, Mt, K, W, tm, H, enc::Epi::kBiasResidLN, b, out, {}, st, nullptr, resid, L.ln_gf[i],
+                      L.ln_bf[i]);
+    enc_status r = run_gemm(h, A, Mt, K, W, tm, H, enc::Epi::kBiasResidStore, b, w.z, {}, st, nullptr, resid);
+    return r != ENC_OK ? r : dec_ln(h, w.z, L.ln_g[i], L.ln_b[i], out, Mt, st);
+  };
+  if ((s = resid_ln(w.ctx, H, L.w_o, L.tm_o, L.b_o, yin, 0, 1, w.h1)) != ENC_OK) return s;
   if ((s = run_gemm(h, w.h1, Mt, H, L.w_q2, L.tm_q2, H, enc::Epi::kBiasQkvSplit, L.b_q2, w.q2, spt, st)) != ENC_OK)
     return s;
   if ((s = run_gemm(h, mem, Ms, H, L.w_kv2, L.tm_kv2, 2 * H, enc::Epi::kBiasQkvSplit, L.b_kv2, w.kv2, sps, st)) !=
@@ -1504,16 +1513,10 @@ enc_status dec_layer(enc_handle* h, int l, const void* yin, void* yout, const in
     return s;
   const __half* kv2 = static_cast<const __half*>(w.kv2);
   if ((s = dec_attention(h, w.q2, kv2, kv2 + hd * S, mem_len, w.ctx, B, T, S, false, st)) != ENC_OK) return s;
-  if ((s = run_gemm(h, w.ctx, Mt, H, L.w_o2, L.tm_o2, H, enc::Epi::kBiasResidStore, L.b_o2, w.z, {}, st, nullptr,
-                    w.h1)) != ENC_OK)
-    return s;
-  if ((s = dec_ln(h, w.z, L.ln_g[1], L.ln_b[1], w.h2, Mt, st)) != ENC_OK) return s;
+  if ((s = resid_ln(w.ctx, H, L.w_o2, L.tm_o2, L.b_o2, w.h1, 1, 1, w.h2)) != ENC_OK) return s;
   const enc::Epi gelu = h->gelu == ENC_GELU_TANH ? enc::Epi::kBiasGeluTanh : enc::Epi::kBiasGelu;
   if ((s = run_gemm(h, w.h2, Mt, H, L.w_ff1, L.tm_ff1, h->F, gelu, L.b_ff1, w.u, {}, st)) != ENC_OK) return s;
-  if ((s = run_gemm(h, w.u, Mt, h->F, L.w_ff2, L.tm_ff2, H, enc::Epi::kBiasResidStore, L.b_ff2, w.z, {}, st, nullptr,
-                    w.h2)) != ENC_OK)
-    return s;
-  return dec_ln(h, w.z, L.ln_g[2], L.ln_b[2], yout, Mt, st);
+  return resid_ln(w.u, h->F, L.w_ff2, L.tm_ff2, L.b_ff2, w.h2, 2, 2, yout);
 }
 
 }  // namespace
@@ -1566,7 +1569,7 @@ enc_status enc_decoder_create(int head_num, int size_per_head, int ffn_dim, int 
   const size_t mrows[7] = {(size_t)H, (size_t)H, (size_t)H, (size_t)H, (size_t)H, (size_t)H, F};
   const size_t mcols[7] = {3 * (size_t)H, (size_t)H, (size_t)H, 2 * (size_t)H, (size_t)H, F, (size_t)H};
   const size_t vlen[7] = {3 * (size_t)H, (size_t)H, (size_t)H, 2 * (size_t)H, (size_t)H, F, (size_t)H};
-  size_t per_layer = 6 * align_up((size_t)H * 2, 256), staging = 0;
+  size_t per_layer = 6 * (align_up((size_t)H * 2, 256) + align_up((size_t)H * 4, 256)), staging = 0;
   for (int i = 0; i < 7; ++i) {
     per_layer += align_up(mrows[i] * mcols[i] * 2, 256) + align_up(vlen[i] * 4, 256);
     staging = std::max(staging, align_up(mrows[i] * mcols[i] * 2, 256));
@@ -1622,6 +1625,13 @@ enc_status enc_decoder_create(int head_num, int size_per_head, int ffn_dim, int 
       if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder LayerNorm upload"); }
       if (i % 2 == 0) L.ln_g[i / 2] = dst; else L.ln_b[i / 2] = dst;
       p += align_up((size_t)H * 2, 256);
+      float* dstf = reinterpret_cast<float*>(p);
+      widen_to_f32_kernel<__half><<<(unsigned)((H + 255) / 256), 256>>>(dst, dstf, H);
+      e = cudaDeviceSynchronize();
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) { free_handle(h); return cuda_fail(e, "decoder LayerNorm widen"); }
+      if (i % 2 == 0) L.ln_gf[i / 2] = dstf; else L.ln_bf[i / 2] = dstf;
+      p += align_up((size_t)H * 4, 256);
     }
   }
   *out = h;
