@@ -346,7 +346,7 @@ __device__ __forceinline__ bool epilogue_warp_tile(uint32_t t_cols, int row0, in
 // between, i.e. after they have read buffer b.
 // ---------------------------------------------------------------------------
 struct LnCtx {
-  float2* stats;          // [2 buffers][2 halves][128 rows] (mean, M2)
+  float2* stats;          // [2 buffers][column slices][128 rows] (mean, M2)
   uint32_t local_bar;     // 8 epilogue warps of this CTA, one phase per tile
   uint32_t ready_bar0;    // + 8 * buffer: one arrival from each other pair
   int pairs;              // P
@@ -371,19 +371,22 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
                                                  EpiWarpState& ws, const LnCtx& ln, int slice, int rloc,
                                                  bool signaller, uint32_t local, WaitFull wait_full,
                                                  Release release) {
-  constexpr int CHUNKS = 4;                    // 128 columns per warp
+  constexpr int kCols = 256 / kEpiSlices;      // columns per warp (128 with 8 epilogue warps)
+  constexpr int CHUNKS = kCols / 32;
   const int lane = threadIdx.x & 31;
   {
-    const int i = lane * 4;                    // bias, gamma, beta of the warp's 128 columns
+    const int i = lane * 4;                    // bias, gamma, beta of the warp's columns
     float4 b = make_float4(0.f, 0.f, 0.f, 0.f), g = b, t = b;
-    if (col_begin + i < N) {
+    if (i < kCols && col_begin + i < N) {
       b = __ldg(reinterpret_cast<const float4*>(bias + col_begin + i));
       g = __ldg(reinterpret_cast<const float4*>(gamma + col_begin + i));
       t = __ldg(reinterpret_cast<const float4*>(beta + col_begin + i));
     }
-    *reinterpret_cast<float4*>(par_s + i) = b;
-    *reinterpret_cast<float4*>(par_s + 128 + i) = g;
-    *reinterpret_cast<float4*>(par_s + 256 + i) = t;
+    if (i < kCols) {
+      *reinterpret_cast<float4*>(par_s + i) = b;
+      *reinterpret_cast<float4*>(par_s + kCols + i) = g;
+      *reinterpret_cast<float4*>(par_s + 2 * kCols + i) = t;
+    }
   }
   auto buf_of = [&](int j) { return ws.stage + ((ws.seq + j) & 1u) * kStageChunkBytes; };
   auto issue_res = [&](int j) {                // lane 0: residual chunk j into buffer (seq + j) & 1
@@ -455,7 +458,7 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
 
   // Exchange.
   const uint32_t b = local & 1u;
-  ln.stats[(b * 2 + slice) * 128 + rloc] = make_float2(mean, m2);
+  ln.stats[(b * kEpiSlices + slice) * 128 + rloc] = make_float2(mean, m2);
   __syncwarp();
   int ok = 1;
   if (lane == 0) {
@@ -471,14 +474,14 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok) return false;
   float tn = 0.f, tmean = 0.f, tm2 = 0.f;
-  const uint32_t st0 = sm100::smem_u32(ln.stats + (b * 2) * 128 + rloc);
+  const uint32_t st0 = sm100::smem_u32(ln.stats + (b * kEpiSlices) * 128 + rloc);
   for (int p = 0; p < ln.pairs; ++p) {
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
+    for (int hf = 0; hf < kEpiSlices; ++hf) {
       const uint32_t addr = st0 + hf * 128 * 8;
-      const float2 h = p == ln.pair ? ln.stats[(b * 2 + hf) * 128 + rloc]
+      const float2 h = p == ln.pair ? ln.stats[(b * kEpiSlices + hf) * 128 + rloc]
                                     : ld_cluster_f2(mapa_shared(addr, 2 * p + ln.rir));
-      chan_merge(tn, tmean, tm2, 128.0f, h.x, h.y);
+      chan_merge(tn, tmean, tm2, (float)kCols, h.x, h.y);
     }
   }
   const float rstd = rsqrtf(tm2 / (float)N + kLnEps);
@@ -499,8 +502,8 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {          // gamma, beta: 16-byte broadcast reads
-      const float4 g4 = *reinterpret_cast<const float4*>(par_s + 128 + 32 * j + i);
-      const float4 t4 = *reinterpret_cast<const float4*>(par_s + 256 + 32 * j + i);
+      const float4 g4 = *reinterpret_cast<const float4*>(par_s + kCols + 32 * j + i);
+      const float4 t4 = *reinterpret_cast<const float4*>(par_s + 2 * kCols + 32 * j + i);
       const float o0 = fmaf((__uint_as_float(cur[i]) - tmean) * rstd, g4.x, t4.x);
       const float o1 = fmaf((__uint_as_float(cur[i + 1]) - tmean) * rstd, g4.y, t4.y);
       const float o2 = fmaf((__uint_as_float(cur[i + 2]) - tmean) * rstd, g4.z, t4.z);
@@ -713,7 +716,7 @@ struct PairCfgT {
   // Per epilogue warp: bias (and, for the fused LayerNorm, gamma and beta) of its columns.
   static constexpr int kParamFloats = 3 * (256 / kEpiSlices);
   static constexpr int kStatsOffset = (kBiasOffset + kEpiWarps * kParamFloats * 4 + 15) / 16 * 16;
-  static constexpr int kStatsBytes = 2 * 2 * 128 * 8;       // LayerNorm statistics, [2][2][128] float2
+  static constexpr int kStatsBytes = 2 * kEpiSlices * 128 * 8;   // LayerNorm statistics, [2][slices][128] float2
   static constexpr int kStoreOffset = (kStatsOffset + kStatsBytes + 1023) / 1024 * 1024;
   static constexpr int kSmem = 1024 + kStoreOffset + kEpiWarps * kStoreBufs * (32 * 32 * 2);
   static_assert(kSmem <= 227 * 1024, "dynamic shared memory of one CTA");
