@@ -1158,11 +1158,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();                             // every CTA's partial is in its shared memory
 
   if (warp >= 2) {
-    // Rows [row0, row1) of the tile, 8 rows per pass, one float4 column unit per lane.
+    // Rows [row0, row1) of the tile, 8 rows per pass, one float4 column unit per
+    // lane.  The tile's rows that exist (fewer than 128 in the last row block,
+    // e.g. 32 at batch 1) are shared evenly by the cluster's CTAs: the cluster
+    // waits for its slowest reducer at the barrier below.
     const int t = threadIdx.x - 64;
     const int u = t & 31;
-    const int row0 = ks * kBM / splits;
-    const int row1 = (ks + 1) * kBM / splits;
+    const int valid = min(M - m_blk * kBM, kBM);
+    const int row0 = ks * valid / splits;
+    const int row1 = (ks + 1) * valid / splits;
     const int col = n_blk * G::kBN + 4 * u;
     if (col < N) {
       for (int r = row0 + (t >> 5); r < row1; r += 8) {
