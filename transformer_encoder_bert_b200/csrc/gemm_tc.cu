@@ -581,13 +581,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_kb = (K + kBK - 1) / kBK;
+  // The weights do not depend on the previous kernel: with a fixed row count
+  // (the grid's first tiles all exist) the producer requests the first stages'
+  // weight tiles of its first tile before waiting for it.
+  int pre = 0;
+  if (!m_dev && warp == 0 && lane == 0) {
+    pre = min(G::kStages, num_kb);
+    const int n_blk = (int)blockIdx.x % num_n;
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(full_bar(i), G::kStageBytes);
+      tma_load_2d(&tm_b, smem_u32(sB + i * G::kBBytes), full_bar(i), i * kBK, n_blk * BN);
+    }
+  }
   pdl_wait();                                  // the previous kernel's writes (A, m_dev) are visible
   pdl_trigger();
   const int M = m_dev ? min(*m_dev, M_max) : M_max;
   const int num_m = (M + kBM - 1) / kBM;
-  const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
-  const int num_kb = (K + kBK - 1) / kBK;
 
   bool ok = true;
   if (warp == 0) {
@@ -599,6 +611,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % G::kStages;
           const uint32_t ph = (it / G::kStages) & 1u;
+          if ((int)it < pre) {                   // the weight tile is already on its way
+            tma_load_2d(&tm_a, smem_u32(sA + s * G::kABytes), full_bar(s), kb * kBK, m_blk * kBM);
+            continue;
+          }
           if (!mbar_wait<kSleepNs>(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(s), G::kStageBytes);
           tma_load_2d(&tm_a, smem_u32(sA + s * G::kABytes), full_bar(s), kb * kBK, m_blk * kBM);
@@ -791,12 +807,25 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();                               // barriers of both CTAs are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_kb = (K + kBK - 1) / kBK;
+  // The weights do not depend on the previous kernel: with a fixed row count
+  // (the grid's first work items all exist) each CTA's producer requests the
+  // first stages' weight halves of its first work item before waiting for it.
+  int pre = 0;
+  if (!m_dev && warp == 0 && lane == 0) {
+    pre = min(G::kStages, num_kb);
+    const int n_blk = kLn ? pic : cluster % num_n;
+    for (int i = 0; i < pre; ++i) {
+      const uint32_t leader_full = mapa_shared(full_bar(i), lead);
+      mbar_arrive_expect_tx_cluster(leader_full, G::kStageBytes);
+      tma_load_2d_pair(&tm_b, smem_u32(sB + i * G::kBBytes), leader_full, i * kBK, n_blk * BN + (int)rir * 128);
+    }
+  }
   pdl_wait();                                   // the previous kernel's writes (A, m_dev) are visible
   pdl_trigger();
   const int M = m_dev ? min(*m_dev, M_max) : M_max;
   const int num_m = (M + 255) / 256;
-  const int num_n = (N + BN - 1) / BN;
-  const int num_kb = (K + kBK - 1) / kBK;
   // Work items walked by each cluster: 256x256 tiles, or (fused LayerNorm)
   // 256-row blocks whose column block is the pair's index in the cluster.
   const int num_work = kLn ? num_m : num_m * num_n;
@@ -822,6 +851,10 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_kb; ++kb, ++issued) {
           const int s = issued % G::kStages;
           const uint32_t ph = (issued / G::kStages) & 1u;
+          if ((int)issued < pre) {               // the weight half is already on its way
+            tma_load_2d_pair(&tm_a, smem_u32(sA + s * G::kABytes), mapa_shared(full_bar(s), lead), kb * kBK, a_row);
+            continue;
+          }
           if (!mbar_wait<kSleepNs>(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
           const uint32_t leader_full = mapa_shared(full_bar(s), lead);
           mbar_arrive_expect_tx_cluster(leader_full, G::kStageBytes);
@@ -1081,6 +1114,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The weights do not depend on the previous kernel: with a fixed row count
+  // (no device count, so no tile of this grid can turn out empty) the producer
+  // requests the first stages' weight tiles before waiting for it, so that
+  // their latency overlaps its tail.
+  int pre = 0;
+  if (!m_dev && warp == 0 && lane == 0) {
+    pre = min(G::kStages, kb1 - kb0);
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(full_bar(i), G::kStageBytes);
+      tma_load_2d(&tm_b, sbase + i * G::kStageBytes + G::kABytes, full_bar(i), (kb0 + i) * kBK, n_blk * G::kBN);
+    }
+  }
   pdl_wait();                                 // the previous kernel's writes (A, m_dev) are visible
   pdl_trigger();
   const int M = m_dev ? min(*m_dev, M_max) : M_max;
@@ -1101,6 +1146,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % G::kStages;
         const uint32_t ph = (it / G::kStages) & 1u;
+        if ((int)it < pre) {                  // the weight tile is already on its way
+          tma_load_2d(&tm_a, sbase + s * G::kStageBytes, full_bar(s), kb * kBK, m_blk * kBM);
+          continue;
+        }
         if (!mbar_wait<kSleepNs>(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { ok = false; break; }
         mbar_arrive_expect_tx(full_bar(s), G::kStageBytes);
         tma_load_2d(&tm_a, sbase + s * G::kStageBytes, full_bar(s), kb * kBK, m_blk * kBM);
