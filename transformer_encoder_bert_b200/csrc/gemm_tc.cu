@@ -1188,7 +1188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int got = 0;
     if (lane == 0) got = mbar_wait<kSleepNs>(tfull_bar, 0, kWaitLimitNs) ? 1 : 0;
     got = __shfl_sync(0xffffffffu, got, 0);
-    if (got) {
+    // Only rows that exist are reduced: a quadrant past them copies nothing.
+    if (got && quad * 32 < M - m_blk * kBM) {
       tc_fence_after();
       uint32_t v[32];
 #pragma unroll 1
@@ -1199,7 +1200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(smem + part_offset(r, slice * 16 + 8 * j + q)) =
               make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       }
-    } else {
+    } else if (!got) {
       ok = false;
     }
   }

@@ -111,7 +111,7 @@ __device__ __forceinline__ void normalise_row(const typename Vec<T>::Raw (&zr)[V
     const int c = lane + 32 * v;
     if (c < nvec) {
       float o[E], gg[E], tt[E];
-      param(c, gg, tt);
+      param(v, c, gg, tt);
 #pragma unroll
       for (int e = 0; e < E; ++e) o[e] = fmaf((z[v][e] - mean) * rstd, gg[e], tt[e]);
       Vec<T>::store(orow + c * E, o);
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kLnWarps * 32)
       if (c < nvec) x[v] = *reinterpret_cast<const Raw*>(zin + (size_t)r * H + c * E);
     }
   };
-  auto param = [&](int c, float (&gg)[E], float (&tt)[E]) {
+  auto param = [&](int, int c, float (&gg)[E], float (&tt)[E]) {
     Vec<T>::unpack(*reinterpret_cast<const Raw*>(sg + c * E), gg);
     Vec<T>::unpack(*reinterpret_cast<const Raw*>(st + c * E), tt);
   };
@@ -184,22 +184,33 @@ __global__ void __launch_bounds__(128)
                              const __half* __restrict__ beta, __half* __restrict__ out, int rows, int H,
                              const int* __restrict__ rows_dev) {
   constexpr int E = 8;
-  pdl_wait();                                   // the rows of the previous kernels are visible
-  pdl_trigger();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  const int nvec = H / E;
+  // gamma and beta do not depend on the previous kernel: requested before
+  // waiting for it.
+  uint4 gv[VPT], bv[VPT];
+#pragma unroll
+  for (int v = 0; v < VPT; ++v) {
+    const int c = lane + 32 * v;
+    if (c < nvec) {
+      gv[v] = __ldg(reinterpret_cast<const uint4*>(gamma + c * E));
+      bv[v] = __ldg(reinterpret_cast<const uint4*>(beta + c * E));
+    }
+  }
+  pdl_wait();                                   // the rows of the previous kernels are visible
+  pdl_trigger();
   if (rows_dev) rows = min(rows, *rows_dev);   // packed tokens: the row count lives on the device
   if (row >= rows) return;
-  const int nvec = H / E;
   uint4 za[VPT];
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
     const int c = lane + 32 * v;
     if (c < nvec) za[v] = __ldg(reinterpret_cast<const uint4*>(zin + (size_t)row * H + c * E));
   }
-  normalise_row<__half, VPT>(za, lane, nvec, H, out + (size_t)row * H, [&](int c, float (&gg)[E], float (&tt)[E]) {
-    Vec<__half>::unpack(__ldg(reinterpret_cast<const uint4*>(gamma + c * E)), gg);
-    Vec<__half>::unpack(__ldg(reinterpret_cast<const uint4*>(beta + c * E)), tt);
+  normalise_row<__half, VPT>(za, lane, nvec, H, out + (size_t)row * H, [&](int v, int, float (&gg)[E], float (&tt)[E]) {
+    Vec<__half>::unpack(gv[v], gg);
+    Vec<__half>::unpack(bv[v], tt);
   });
 }
 
