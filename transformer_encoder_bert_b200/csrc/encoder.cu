@@ -297,7 +297,7 @@ enc_status step_qkv(enc_handle* h, int l, const void* x, void* qkv, int batch, i
 // Attention kernel choice: the tensor-core kernels for size_per_head 64 and
 // sequences longer than the short kernel's 64-row tiles (one 128-key block up to
 // 128, key blocks with a running maximum beyond); mma.sync otherwise (and for
-// every length under ENC_ATTN_NO_TC=1).
+// every length with the tc_attention option off).
 bool use_tc_attention(const enc_handle* h, int seq) {
   return enc::attention_tc_supported(h->d, seq) && h->tc_attn;
 }
@@ -333,9 +333,11 @@ enc_status step_out_proj(enc_handle* h, int l, const void* ctx, const void* resi
 // kernel.  Needs the 2-CTA tiles to be the ones chosen for the shape (large M)
 // and H a multiple of 256.  Measured on BERT-Base shapes, the fused epilogue
 // (two passes over the accumulator and a row-statistics exchange per tile)
-// pays off behind FFN2's long K = F main loop with clusters of at most 6 CTAs
-// (H <= 768), and not behind the output projection's K = H main loop, nor with
-// 8-CTA clusters (H = 1024): those keep the separate LayerNorm kernel.
+// hides behind FFN2's long K = F main loop, and even behind the output
+// projection's short K = H one it beats the GEMM plus LayerNorm kernel, with
+// clusters of at most 6 CTAs (H <= 768).  With 8-CTA clusters (H = 1024) it
+// measured slower: those shapes keep the separate LayerNorm kernel unless the
+// option asks for fusion wherever supported (2).
 bool ln_fused(const enc_handle* h, int tokens, int which) {
   if (h->dtype != ENC_FP16 || !h->tma_store || !enc::gemm_ln_supported(tokens, h->H) ||
       choose_bn(h, tokens, h->H) != enc::kPairTile)
