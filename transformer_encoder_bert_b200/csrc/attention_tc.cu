@@ -2,7 +2,7 @@
 // (tcgen05 + TMEM + TMA) for size_per_head 64 and seq > 64.  Two kernels:
 // attention_tc_kernel for seq <= 128, where one block of 128 keys covers every
 // key of a sequence (described here), and attention_tc_long_kernel for longer
-// sequences (described above it).
+// sequences (described where it is defined).
 //
 // The source page ("Faster Transformer 优化原理") runs attention as two batched
 // GEMMs around a SoftMax kernel.  Here both products run on tcgen05 and the
@@ -27,10 +27,10 @@
 // P in TMEM frees the Q and K tiles as soon as S = Q K^T has completed, so the
 // next item's Q and K load while this item's softmax, P V and output run; its
 // V loads once the output rows staged in the V tile have been read by their
-// TMA stores.  TMEM:
-// S in columns [0, 128), P (two halves per column) over [0, 64), O in
-// [64, 128); the next S waits until O has been read.  Footprint per CTA: 48 KB
-// of tiles and 128 TMEM columns.  Every mbarrier wait is bounded in time.
+// TMA stores.  TMEM: S in columns [0, 128), P (two halves per column) over
+// [0, 64), O in [64, 128); the next S waits until O has been read.  Footprint
+// per CTA: 48 KB of tiles and 128 TMEM columns.  Every mbarrier wait is
+// bounded in time.
 //
 // Q, K and V are read through one 2-D tensor map with rows of 64 halves:
 // the split layout [3, B, nh, S, 64] (rows = ((t*B + b)*nh + h)*S + s) or the
