@@ -355,7 +355,22 @@ def time_forward(enc, x, vl, out, wl, args, flush, stream, barrier):
             per_kernel[names[j]].append(evs[j].elapsed_time(evs[j + 1]))
         traced.append(evs[0].elapsed_time(evs[nk]))
     return {"ms": sum(step_ms) / len(step_ms), "per_kernel": per_kernel, "launches": launches,
-            "traced_ms": sum(traced) / len(traced), "nk": nk}
+            "traced_ms": sum(traced) / len(traced), "nk": nk, "step_ms": step_ms}
+
+
+def step_stats(step_ms, device=None):
+    """Median, 10th and 90th percentile of the per-step device times (ms), each
+    the max over ranks."""
+    q = sorted(step_ms)
+
+    def pct(p):
+        i = p / 100.0 * (len(q) - 1)
+        lo = int(math.floor(i))
+        hi = min(lo + 1, len(q) - 1)
+        return q[lo] + (q[hi] - q[lo]) * (i - lo)
+
+    med, p10, p90 = max_over_ranks([pct(50), pct(10), pct(90)], device=device)
+    return {"median": med, "p10": p10, "p90": p90}
 
 
 def kernel_table(wl, inp, per_kernel, peaks, packed: bool, graph_ms=None, forwards=None):
@@ -507,6 +522,7 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     clk = clocks.stop()
 
     ms, e2e_step = max_over_ranks([ms, e2e_step], device=dev)
+    main_stats = step_stats(main_t["step_ms"], device=dev)
     if rank != 0:
         return 0
 
@@ -520,7 +536,8 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
     value = job_throughput(wl.batch, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "step_ms": main_stats, "higher_is_better": True,
+        "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16" if wl.dtype == "fp16" else "fp32", "data": "synthetic",
         "config": dict(workload_config(wl, world, l2="flushed before every timed step (256 MiB write)"),
                        launch="one recorded CUDA graph per step" if args.graph else "enc_forward per step",
@@ -549,6 +566,7 @@ def run_ours(args, wl: EI.Workload, rank: int, world: int, local_rank: int):
         tc_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         line["secondary"] = {
             "workload": sw.name, "value": sw.batch / (st["ms"] * 1e-3), "unit": UNIT, "ms_per_step": st["ms"],
+            "step_ms": step_stats(st["step_ms"]),
             "traced_ms_per_forward": st["traced_ms"], "gpu_launches": int(st["launches"]),
             "roofline": roofline_of(skern, swork, sdom, peaks, peak_src,
                                     measured_traffic(sdom, sw.name)),
@@ -604,7 +622,11 @@ def run_decoder(args, rank: int, world: int, local_rank: int):
     for _ in range(args.warmup):
         dec.forward(y, tl, mem, ml, out)
     torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
     ts = []
+    launches0 = dec.launch_count()
     for _ in range(args.steps):
         flush.zero_()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -613,15 +635,38 @@ def run_decoder(args, rank: int, world: int, local_rank: int):
         e.record()
         e.synchronize()
         ts.append(s.elapsed_time(e))
+    launches = dec.launch_count() - launches0
+    # e2e: each step copies its inputs from pinned host memory, runs the
+    # decoder and copies the output back to pinned host memory.
+    hy, hmem = torch.from_numpy(inp.y).pin_memory(), torch.from_numpy(inp.mem).pin_memory()
+    htl, hml = torch.from_numpy(inp.tgt_len).pin_memory(), torch.from_numpy(inp.mem_len).pin_memory()
+    hout = torch.empty_like(hy).pin_memory()
+    e2e_ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        y.copy_(hy, non_blocking=True)
+        mem.copy_(hmem, non_blocking=True)
+        tl.copy_(htl, non_blocking=True)
+        ml.copy_(hml, non_blocking=True)
+        dec.forward(y, tl, mem, ml, out)
+        hout.copy_(out, non_blocking=True)
+        e.record()
+        e.synchronize()
+        e2e_ts.append(s.elapsed_time(e))
+    clk = clocks.stop()
     status = dec.device_status()
-    ms = max_over_ranks([sum(ts) / len(ts)], device=dev)[0]
+    ms, e2e_ms = max_over_ranks([sum(ts) / len(ts), sum(e2e_ts) / len(e2e_ts)], device=dev)
+    stats = step_stats(ts, device=dev)
     if rank != 0:
         return 0
+    h2d = sum(t.numel() * t.element_size() for t in (hy, hmem, htl, hml))
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     tf = decoder_flops(wl) / (ms * 1e-3) / 1e12
     line = {"metric": "decoder fwd sequences/s", "value": job_throughput(wl.batch, world, ms), "unit": UNIT,
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "step_ms": stats,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "tgt_seq": wl.tgt_seq, "mem_seq": wl.mem_seq,
                        "layers": sh.num_layers, "l2": "flushed before every timed step (256 MiB write)",
@@ -629,6 +674,9 @@ def run_decoder(args, rank: int, world: int, local_rank: int):
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                          "traffic": None, "kernel": "whole decoder forward",
                          "peak_source": f"{peak_src} burst bf16 matmul"},
+            "e2e": {"value": job_throughput(wl.batch, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+            "gpu_launches": int(launches), "clocks": clk,
             "device_status": status}
     print(json.dumps(line), flush=True)
     return 0

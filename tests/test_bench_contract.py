@@ -7,6 +7,7 @@
 - The DRAM traffic figure is taken from profiles/traffic.md only while the
   kernel's sources are the ones it was measured on.
 - Named workloads have the shapes of the configurations they stand for.
+- The per-step statistics are the median and the 10th / 90th percentiles.
 """
 import os
 import sys
@@ -43,6 +44,13 @@ def test_kernel_work_fp32_counts_four_byte_elements():
     wl = bench.parse_workload("tiny-fp32:1")
     M, H = 32, 128
     assert bench.kernel_work(wl)["ln1"] == (0.0, 4 * 2 * M * H)
+
+
+def test_step_stats_are_median_and_deciles():
+    st = bench.step_stats([float(v) for v in (11, 1, 5, 3, 9, 7, 2, 4, 6, 8, 10)])
+    assert st == {"median": 6.0, "p10": 2.0, "p90": 10.0}
+    st = bench.step_stats([2.0, 1.0])                 # linear interpolation between ranks
+    assert st["median"] == pytest.approx(1.5) and st["p10"] == pytest.approx(1.1)
 
 
 def test_job_throughput_counts_every_rank():

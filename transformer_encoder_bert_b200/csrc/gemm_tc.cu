@@ -369,8 +369,8 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
                                                  const float* __restrict__ bias, const float* __restrict__ gamma,
                                                  const float* __restrict__ beta, float* par_s, const CUtensorMap* tm_c,
                                                  EpiWarpState& ws, const LnCtx& ln, int slice, int rloc,
-                                                 bool signaller, uint32_t local, WaitFull wait_full,
-                                                 Release release) {
+                                                 bool signaller, uint32_t local, bool prefetch, int next_row0,
+                                                 WaitFull wait_full, Release release) {
   constexpr int kCols = 256 / kEpiSlices;      // columns per warp (128 with 8 epilogue warps)
   constexpr int CHUNKS = kCols / 32;
   const int lane = threadIdx.x & 31;
@@ -397,10 +397,17 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
   // Residual chunks 0 and 1 before the accumulator is awaited (once the
   // previous tile's stores have read both buffers); chunk j + 2 once chunk j's
   // residual has been read out of its buffer.
+  // With `prefetch`, the rest of this tile's residual (first tile) and the next
+  // tile's (at row next_row0, if any) are requested into L2 now, so that the
+  // loads of pass 1 find them there.
   if (lane == 0) {
     sm100::bulk_wait_group_read<0>();
     issue_res(0);
     issue_res(1);
+    if (prefetch && local == 0)
+      for (int j = 2; j < CHUNKS; ++j) sm100::tma_prefetch_2d_l2(ws.tm_r, col_begin + 32 * j, row0);
+    if (prefetch && next_row0 >= 0)
+      for (int j = 0; j < CHUNKS; ++j) sm100::tma_prefetch_2d_l2(ws.tm_r, col_begin + 32 * j, next_row0);
   }
   int got = 0;
   if (lane == 0) got = wait_full() ? 1 : 0;
@@ -932,12 +939,18 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kThreads, 1)
       auto wait_full = [&] { return mbar_wait<kSleepNs>(tfull_bar(acc), aph, kWaitLimitNs); };
       auto release = [&] { mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0); };
       bool got;
-      if constexpr (kLn)
+      if constexpr (kLn) {
+        // Residual prefetch into L2 where the epilogue outlasts the main loop
+        // (K <= 1024, the output projection); with FFN2's K = F it measured slower.
+        const bool prefetch = K <= 1024;
+        const int next_row0 = w + num_clusters < num_work ? row0 + num_clusters * 256 : -1;
         got = epilogue_ln_tile(t_cols, row0, n_blk * BN + slice * kCols, N, bias, ln_gamma, ln_beta, par_s, tmc,
-                               ws, ln, slice, quad * 32 + lane, warp == 2, local, wait_full, release);
-      else
+                               ws, ln, slice, quad * 32 + lane, warp == 2, local, prefetch, next_row0, wait_full,
+                               release);
+      } else {
         got = epilogue_warp_tile<EPI, kChunks, G::kStoreBufs>(t_cols, row0, n_blk * BN + slice * kCols, M, N, bias,
                                                               bias_s, C, sp, tmc, ws, resid, wait_full, release);
+      }
       if (!got) { ok = false; break; }
     }
     if (lane == 0) bulk_wait_group_all();      // every TMA store of this warp has completed

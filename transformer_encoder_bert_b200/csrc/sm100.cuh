@@ -98,6 +98,14 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* m, uint32_t dst, 
       : "memory");
 }
 
+// 2-D tiled prefetch global -> L2 of one box of the map (no shared memory,
+// no barrier; a box partly outside the tensor fetches only its inside).
+__device__ __forceinline__ void tma_prefetch_2d_l2(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // 2-D / 5-D tiled store shared (this CTA) -> global, tracked by bulk groups.
 // Elements of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t x, int32_t y) {
