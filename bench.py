@@ -52,6 +52,9 @@ KERNEL_NAMES = ["qkv_gemm", "attention", "out_proj_gemm", "ln1", "ffn1_gemm", "f
 # when the output-projection and FFN2 GEMMs write the LayerNorm of their rows
 KERNEL_NAMES_FUSED = ["qkv_gemm", "attention", "out_proj_ln_gemm", "ffn1_gemm", "ffn2_ln_gemm"]
 KERNEL_NAMES_FFN2_LN = ["qkv_gemm", "attention", "out_proj_gemm", "ln1", "ffn1_gemm", "ffn2_ln_gemm"]
+# Six kernels per layer with the output projection fused and FFN2 not: only
+# when the options ask for it (ln_fuse_out_proj=2, ln_fuse_ffn2=0).
+KERNEL_NAMES_OPROJ_LN = ["qkv_gemm", "attention", "out_proj_ln_gemm", "ffn1_gemm", "ffn2_gemm", "ln2"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -293,12 +296,14 @@ def workload_config(wl: EI.Workload, world: int, l2: str):
 
 
 # ------------------------------------------------------------------ our arm
-def kernel_names(nk: int, num_layers: int, packed: bool):
-    """Names of the nk kernels of one forward, in launch order."""
+def kernel_names(nk: int, num_layers: int, packed: bool, ffn2_ln_off: bool = False):
+    """Names of the nk kernels of one forward, in launch order (`ffn2_ln_off`:
+    the options turned the FFN2 LayerNorm fusion off)."""
     if nk == 1:
         return ["persistent"]                 # the single-launch forward of the whole stack
     per_layer = (nk - (3 if packed else 0)) // num_layers
-    layer_names = {5: KERNEL_NAMES_FUSED, 6: KERNEL_NAMES_FFN2_LN}.get(per_layer, KERNEL_NAMES)
+    six = KERNEL_NAMES_OPROJ_LN if ffn2_ln_off else KERNEL_NAMES_FFN2_LN
+    layer_names = {5: KERNEL_NAMES_FUSED, 6: six}.get(per_layer, KERNEL_NAMES)
     if packed:
         return ["offsets", "pack"] + layer_names * num_layers + ["unpack"]
     return layer_names * num_layers
@@ -347,7 +352,8 @@ def time_forward(enc, x, vl, out, wl, args, flush, stream, barrier):
         graph.close()
     enc.set_trace_events(None)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    names = kernel_names(nk, wl.shape.num_layers, args.packed)
+    ffn2_ln_off = any(o.replace(" ", "") in ("ln_fuse_ffn2=0", "ln_fuse_ffn2=False") for o in args.option)
+    names = kernel_names(nk, wl.shape.num_layers, args.packed, ffn2_ln_off)
     per_kernel = {k: [] for k in names}
     traced = []
     for evs in ev_sets:
@@ -614,6 +620,9 @@ def run_decoder(args, rank: int, world: int, local_rank: int):
     inp = EI.make_decoder_inputs(wl)
     sh = wl.shape
     dec = Decoder(sh.head_num, sh.size_per_head, sh.ffn_dim, inp.layers)
+    options = dict(o.split("=", 1) for o in args.option)
+    for name, v in options.items():
+        dec.set_option(name, int(v))
     dev = torch.device("cuda", local_rank)
     y, mem = torch.from_numpy(inp.y).to(dev), torch.from_numpy(inp.mem).to(dev)
     tl, ml = torch.from_numpy(inp.tgt_len).to(dev), torch.from_numpy(inp.mem_len).to(dev)
@@ -670,7 +679,8 @@ def run_decoder(args, rank: int, world: int, local_rank: int):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "tgt_seq": wl.tgt_seq, "mem_seq": wl.mem_seq,
                        "layers": sh.num_layers, "l2": "flushed before every timed step (256 MiB write)",
-                       "launch": "enc_decoder_forward per step (9 to 12 launches per layer)"},
+                       "launch": "enc_decoder_forward per step (9 to 12 launches per layer)",
+                       **({"options": options} if options else {})},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                          "traffic": None, "kernel": "whole decoder forward",
                          "peak_source": f"{peak_src} burst bf16 matmul"},

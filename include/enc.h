@@ -130,10 +130,13 @@ typedef enum {
    * statistics exchanged across the thread-block cluster that covers a row;
    * needs the 2-CTA tiles and a hidden size that is a multiple of 256, at most
    * 1024): 0 never (a separate LayerNorm kernel), 1 (default) where it measured
-   * faster (hidden size <= 768, clusters of at most 6 CTAs), 2 wherever
-   * supported. */
+   * faster (hidden size <= 768, clusters of at most 6 CTAs, and a token count
+   * whose row blocks fill the clusters' waves about as well as the unfused
+   * GEMM's tiles fill its waves), 2 wherever supported. */
   ENC_OPT_LN_FUSE_FFN2 = 4,
-  /* The same for the output-projection GEMM and LayerNorm 1 (0, 1 = default, 2). */
+  /* The same for the output-projection GEMM and LayerNorm 1 (0, 1 = default, 2);
+   * its default asks for clearly better-filled waves than FFN2's, since its
+   * short K = hidden main loop does not hide the fused epilogue. */
   ENC_OPT_LN_FUSE_OUT_PROJ = 5,
   /* 1 (default): kernels are launched with programmatic dependent launch, so
    * each one's set-up overlaps its predecessor's tail; 0: plain stream order. */

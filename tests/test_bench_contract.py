@@ -108,6 +108,8 @@ def test_source_digest_depends_on_every_listed_file():
 def test_kernel_names_follow_launch_order():
     assert bench.kernel_names(7 * 2, 2, False) == bench.KERNEL_NAMES * 2
     assert bench.kernel_names(6 * 12, 12, False) == bench.KERNEL_NAMES_FFN2_LN * 12
+    assert bench.kernel_names(6 * 12, 12, False, ffn2_ln_off=True) == bench.KERNEL_NAMES_OPROJ_LN * 12
+    assert bench.kernel_names(5 * 12, 12, False) == bench.KERNEL_NAMES_FUSED * 12
     names = bench.kernel_names(6 * 12 + 3, 12, True)
     assert names[:2] == ["offsets", "pack"] and names[-1] == "unpack" and len(names) == 75
 

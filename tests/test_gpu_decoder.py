@@ -53,15 +53,18 @@ def test_decoder_matches_oracle(nh, d, F, L, B, T, S):
 
 
 def test_decoder_fused_layernorm_gemms_at_size():
-    """Enough target tokens (32 x 128) for the 2-CTA tiles: the three bias +
-    residual + LayerNorm steps run in their GEMMs' epilogues (row statistics
-    exchanged across the cluster), 9 launches per layer; sampled sequences
-    against the oracle, and against the same decoder with both fusions off."""
+    """Enough target tokens (32 x 128) for the 2-CTA tiles: with both fusions
+    asked for wherever supported, the three bias + residual + LayerNorm steps
+    run in their GEMMs' epilogues (row statistics exchanged across the
+    cluster), 9 launches per layer; sampled sequences against the oracle, and
+    against the same decoder with both fusions off."""
     sh = EI.EncoderShape(12, 64, 3072, 1)
     B, T, S = 32, 128, 96
     wl = EI.DecoderWorkload("dec-fused", sh, B, T, S, "fp16", T // 2, T, S // 2, S, ln_affine_random=True, seed=7)
     inp = EI.make_decoder_inputs(wl)
     dec = _decoder(inp)
+    dec.set_option("ln_fuse_out_proj", 2)
+    dec.set_option("ln_fuse_ffn2", 2)
     n0 = dec.launch_count()
     got = _run(dec, inp)
     assert dec.launch_count() - n0 == 9

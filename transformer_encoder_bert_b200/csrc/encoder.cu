@@ -331,19 +331,28 @@ enc_status step_out_proj(enc_handle* h, int l, const void* ctx, const void* resi
 // Whether GEMM `which` (1: output projection, 2: FFN2) writes the LayerNorm of
 // its rows (kBiasResidLN) instead of z = acc + bias + residual for a LayerNorm
 // kernel.  Needs the 2-CTA tiles to be the ones chosen for the shape (large M)
-// and H a multiple of 256.  Measured on BERT-Base shapes, the fused epilogue
-// (two passes over the accumulator and a row-statistics exchange per tile)
-// hides behind FFN2's long K = F main loop, and even behind the output
-// projection's short K = H one it beats the GEMM plus LayerNorm kernel, with
-// clusters of at most 6 CTAs (H <= 768).  With 8-CTA clusters (H = 1024) it
-// measured slower: those shapes keep the separate LayerNorm kernel unless the
-// option asks for fusion wherever supported (2).
+// and H a multiple of 256.  The fused kernel runs one cluster of H/128 CTAs per
+// 256 rows (22 six-CTA clusters fit at once for H = 768), the unfused one a CTA
+// pair per 256x256 tile (74 pairs), so the two fill their last wave
+// differently.  Measured on BERT-Base shapes (forwards of 6144 to 32768
+// tokens): FFN2's fused epilogue hides behind its long K = F main loop and pays
+// off unless its last wave is far emptier than the unfused kernel's (24
+// clusters' worth of rows on 22 slots: 13 % slower); the output projection's
+// short K = H main loop cannot hide it, and fusing pays off only where the
+// fused kernel fills its waves clearly better (64 and 128 row blocks: 1-3 %
+// faster; 24, 32, 48 and 96: 0.3-5 % slower).  With 8-CTA clusters (H = 1024)
+// fusion measured slower: those shapes keep the separate LayerNorm kernel
+// unless the option asks for fusion wherever supported (2).
 bool ln_fused(const enc_handle* h, int tokens, int which) {
   if (h->dtype != ENC_FP16 || !h->tma_store || !enc::gemm_ln_supported(tokens, h->H) ||
       choose_bn(h, tokens, h->H) != enc::kPairTile)
     return false;
   const int mode = which == 2 ? h->ln_fuse_ffn2 : h->ln_fuse_oproj;
-  return mode == 2 || (mode == 1 && h->H <= 768);
+  if (mode == 2) return true;
+  if (mode != 1 || h->H > 768) return false;
+  float fused = 0.f, unfused = 0.f;
+  if (!enc::gemm_ln_wave_efficiency(tokens, h->H, fused, unfused)) return false;
+  return which == 2 ? fused >= unfused - 0.3f : fused >= unfused + 0.1f;
 }
 
 // The single-launch forward (persistent.cu): FP16, padding kept, few enough

@@ -1402,6 +1402,28 @@ bool encode_output_map_split(CUtensorMap* map, void* base, const SplitShape& sp)
 
 bool gemm_ln_supported(int M, int N) { return M >= 256 && N % 256 == 0 && N <= 1024; }
 
+bool gemm_ln_wave_efficiency(int M, int N, float& fused, float& unfused) {
+  cudaError_t e_ln = cudaSuccess, e_pair = cudaSuccess;
+  int ln_slots = 0;
+  switch (N) {
+    case 256: ln_slots = pair_max_clusters<Epi::kBiasResidLN, 2>(e_ln); break;
+    case 512: ln_slots = pair_max_clusters<Epi::kBiasResidLN, 4>(e_ln); break;
+    case 768: ln_slots = pair_max_clusters<Epi::kBiasResidLN, 6>(e_ln); break;
+    case 1024: ln_slots = pair_max_clusters<Epi::kBiasResidLN, 8>(e_ln); break;
+    default: return false;
+  }
+  const int pair_slots = pair_max_clusters<Epi::kBiasResidStore, 2>(e_pair);
+  if (e_ln != cudaSuccess || e_pair != cudaSuccess || ln_slots <= 0 || pair_slots <= 0 || M <= 0) return false;
+  auto eff = [](int work, int slots) {
+    const int waves = (work + slots - 1) / slots;
+    return static_cast<float>(work) / static_cast<float>(waves * slots);
+  };
+  const int num_m = (M + 255) / 256;
+  fused = eff(num_m, ln_slots);
+  unfused = eff(num_m * (N / 256), pair_slots);
+  return true;
+}
+
 int choose_gemm_splits(int tiles, int num_kb, int num_sms) {
   if (tiles <= 0) return 1;
   for (int s = std::min(SplitCfg::kMaxSplits, num_kb); s >= 2; --s)

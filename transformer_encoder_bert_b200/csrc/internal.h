@@ -105,6 +105,12 @@ int choose_gemm_splits(int tiles, int num_kb, int num_sms);
 // Whether kBiasResidLN can run for an [M, N] GEMM: the row of N columns is
 // covered by one cluster of N/128 CTAs (N a multiple of 256, N <= 1024), M >= 256.
 bool gemm_ln_supported(int M, int N);
+// Wave efficiency (work items / (waves x resident slots)) of an [M, N] GEMM with
+// 2-CTA tiles: `fused` for the LayerNorm-fused kernel (one cluster of N/128 CTAs
+// per 256 rows), `unfused` for the plain bias + residual kernel (one CTA pair
+// per 256x256 tile).  False when N is not a LayerNorm width or the occupancy
+// query fails.
+bool gemm_ln_wave_efficiency(int M, int N, float& fused, float& unfused);
 cudaError_t launch_gemm_tc(const TcGemmArgs& a, cudaStream_t stream);
 
 // Encode a 2-D K-major FP16 tensor map over [rows, cols=K] with a {64, box_rows} box.
