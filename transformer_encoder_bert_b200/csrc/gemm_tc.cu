@@ -364,6 +364,8 @@ __device__ __forceinline__ void chan_merge(float& n, float& mean, float& m2, flo
   n = nn;
 }
 
+constexpr int kMaxLnPairs = 4;                 // clusters of up to 8 CTAs (N <= 1024)
+
 template <typename WaitFull, typename Release>
 __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int col_begin, int N,
                                                  const float* __restrict__ bias, const float* __restrict__ gamma,
@@ -480,15 +482,25 @@ __device__ __forceinline__ bool epilogue_ln_tile(uint32_t t_cols, int row0, int 
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok) return false;
+  // Every pair's statistics of the row are requested before the first merge
+  // (one remote-load latency); merged in pair order.
   float tn = 0.f, tmean = 0.f, tm2 = 0.f;
   const uint32_t st0 = sm100::smem_u32(ln.stats + (b * kEpiSlices) * 128 + rloc);
-  for (int p = 0; p < ln.pairs; ++p) {
+  float2 hs[kMaxLnPairs][kEpiSlices];
 #pragma unroll
-    for (int hf = 0; hf < kEpiSlices; ++hf) {
-      const uint32_t addr = st0 + hf * 128 * 8;
-      const float2 h = p == ln.pair ? ln.stats[(b * kEpiSlices + hf) * 128 + rloc]
-                                    : ld_cluster_f2(mapa_shared(addr, 2 * p + ln.rir));
-      chan_merge(tn, tmean, tm2, (float)kCols, h.x, h.y);
+  for (int p = 0; p < kMaxLnPairs; ++p) {
+    if (p < ln.pairs) {
+#pragma unroll
+      for (int hf = 0; hf < kEpiSlices; ++hf)
+        hs[p][hf] = p == ln.pair ? ln.stats[(b * kEpiSlices + hf) * 128 + rloc]
+                                 : ld_cluster_f2(mapa_shared(st0 + hf * 128 * 8, 2 * p + ln.rir));
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < kMaxLnPairs; ++p) {
+    if (p < ln.pairs) {
+#pragma unroll
+      for (int hf = 0; hf < kEpiSlices; ++hf) chan_merge(tn, tmean, tm2, (float)kCols, hs[p][hf].x, hs[p][hf].y);
     }
   }
   const float rstd = rsqrtf(tm2 / (float)N + kLnEps);
@@ -1052,17 +1064,15 @@ __device__ __forceinline__ uint32_t part_offset(int r, int u) {
   return SplitCfg::kPartOffset + r * 512 + 16 * (u ^ (r & 31));
 }
 
-// Bias, residual and the epilogue's element-wise function on 4 consecutive
-// columns of row `row`.
+// Bias `b`, residual `u` (4 halves) and the epilogue's element-wise function
+// on 4 consecutive columns of a row; both operands were loaded by the caller
+// ahead of the partial sums they are added to.
 template <Epi EPI>
-__device__ __forceinline__ void epilogue4(float (&v)[4], const float* __restrict__ bias,
-                                          const __half* __restrict__ resid, int row, int N, int col) {
+__device__ __forceinline__ void epilogue4(float (&v)[4], const float4& b, const uint2& u) {
   if constexpr (EPI != Epi::kStore) {
-    const float4 b = __ldg(reinterpret_cast<const float4*>(bias + col));
     v[0] += b.x; v[1] += b.y; v[2] += b.z; v[3] += b.w;
   }
   if constexpr (EPI == Epi::kBiasResidStore) {
-    const uint2 u = *reinterpret_cast<const uint2*>(resid + (size_t)row * N + col);
     const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
     const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
     v[0] += lo.x; v[1] += lo.y; v[2] += hi.x; v[3] += hi.y;
@@ -1153,6 +1163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   bool ok = true;
+  float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
@@ -1194,6 +1205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait<kSleepNs>(drain_bar, 0, kWaitLimitNs);
     }
   } else {
+    // The bias of this thread's reduction columns, before the accumulator is awaited.
+    const int col = n_blk * G::kBN + 4 * lane;
+    if constexpr (EPI != Epi::kStore)
+      if (col < N) b4 = __ldg(reinterpret_cast<const float4*>(bias + col));
     // TMEM lanes of quadrant warp % 4; columns [64 * slice, 64 * slice + 64).
     const int quad = warp & 3;
     const int slice = (warp - 2) >> 2;
@@ -1235,13 +1250,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = row0 + (t >> 5); r < row1; r += 8) {
         const int grow = m_blk * kBM + r;
         if (grow >= M) break;
+        // The residual and every CTA's partial are requested before any is
+        // used, so the row costs one remote-load latency, not one per split.
+        uint2 ru = make_uint2(0u, 0u);
+        if constexpr (EPI == Epi::kBiasResidStore) ru = *reinterpret_cast<const uint2*>(resid + (size_t)grow * N + col);
         const uint32_t off = sbase + part_offset(r, u);
+        float4 p[G::kMaxSplits];
+#pragma unroll
+        for (int s = 0; s < G::kMaxSplits; ++s)
+          if (s < splits) p[s] = ld_cluster_f4(mapa_shared(off, (uint32_t)s));
         float a[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = 0; s < splits; ++s) {      // rank order: the same sum on every run
-          const float4 p = ld_cluster_f4(mapa_shared(off, (uint32_t)s));
-          a[0] += p.x; a[1] += p.y; a[2] += p.z; a[3] += p.w;
+#pragma unroll
+        for (int s = 0; s < G::kMaxSplits; ++s) {   // rank order: the same sum on every run
+          if (s < splits) {
+            a[0] += p[s].x; a[1] += p[s].y; a[2] += p[s].z; a[3] += p[s].w;
+          }
         }
-        epilogue4<EPI>(a, bias, resid, grow, N, col);
+        epilogue4<EPI>(a, b4, ru);
         __half* dst = C + row_offset<EPI>(grow, N, sp) + col_offset<EPI>(col, sp);
         *reinterpret_cast<uint2*>(dst) = make_uint2(pack_half2(a[0], a[1]), pack_half2(a[2], a[3]));
       }
