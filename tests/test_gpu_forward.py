@@ -364,6 +364,36 @@ def test_packed_forward_many_attention_items(seq):
     assert enc.device_status() == 0
 
 
+@pytest.mark.parametrize("batch,seq,per_layer", [
+    (64, 96, 7),      # 24 row blocks on 22 fused-cluster slots: neither LayerNorm fused
+    (64, 128, 6),     # 32 row blocks: FFN2 only
+    (128, 96, 6),     # 48: FFN2 only
+    (128, 128, 5),    # 64: both
+    (256, 96, 6),     # 96: FFN2 only
+    (512, 32, 5),     # 64: both
+    (256, 128, 5),    # 128: both
+], ids=str)
+def test_layernorm_fusion_follows_wave_fill(batch, seq, per_layer):
+    """The default LayerNorm fusion compares how full the last wave of the
+    fused kernel (one 6-CTA cluster per 256 rows) and of the unfused GEMM (a CTA
+    pair per 256x256 tile) would be: the kernels per layer at BERT-Base token
+    counts from 6144 to 32768, and one layer at the first of them against the
+    same encoder with both fusions forced on."""
+    sh = EI.EncoderShape(12, 64, 3072, 1)
+    inp = EI.make_inputs(EI.Workload("wave-fill", sh, batch, seq, "fp16", 1, seq, seed=batch + seq))
+    enc = encoder_from_inputs(inp)
+    assert enc.kernels_per_forward(batch, seq) == per_layer
+    if (batch, seq) == (64, 96):
+        got = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+        enc.set_option("ln_fuse_out_proj", 2)
+        enc.set_option("ln_fuse_ffn2", 2)
+        assert enc.kernels_per_forward(batch, seq) == 5
+        fused = to_host(enc.forward(to_dev(inp.x), to_dev(inp.valid_len)))
+        m = valid_mask(inp.valid_len, seq)
+        assert rel_l2(got, fused, m) < FP16_LAYER_REL_L2
+        assert enc.device_status() == 0
+
+
 PACKED_FULL_SIZE = [
     ("bert-base-s32", 512, None, 4),
     ("bert-base", 256, 128, 3),
