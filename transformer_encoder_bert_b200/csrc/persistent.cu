@@ -166,10 +166,6 @@ struct Ctx {
   uint32_t a_phase;       // A-chunk loads so far (parity of the staging barrier)
 };
 
-__device__ __forceinline__ const __half* weight_of(const PersistLayer& L, int p) {
-  return p == kQkv ? L.w_qkv : p == kOproj ? L.w_o : p == kFfn1 ? L.w_ff1 : L.w_ff2;
-}
-
 // Warp 0: the weight tile of this CTA's k-th unit of the forward into slot
 // k & 1: rows n0 .. n0 + 31 of the [N, K] weight, columns k0 .. k0 + KU - 1,
 // as KU / 64 TMA boxes (one per lane, 128-byte swizzle).
