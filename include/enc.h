@@ -300,8 +300,9 @@ ENC_API enc_status enc_graph_destroy(enc_graph_t graph);
  * issues: 1 when the single-launch forward runs (ENC_OPT_PERSISTENT);
  * otherwise per layer 7, less one for each of the output-projection and FFN2
  * GEMMs that writes the LayerNorm of its rows itself (FP16, enough tokens for
- * the 2-CTA tiles; by default FFN2 with hidden size 256, 512 or 768); plus 3
- * with padding removal.  0 for invalid arguments. */
+ * the 2-CTA tiles, hidden size 256, 512 or 768 by default; which of the two
+ * follows ENC_OPT_LN_FUSE_FFN2 and ENC_OPT_LN_FUSE_OUT_PROJ); plus 3 with
+ * padding removal.  0 for invalid arguments. */
 ENC_API int enc_kernels_per_forward(enc_t h, int batch, int seq);
 
 /* enc_launch_count - kernel launches this handle has issued since enc_create
