@@ -307,7 +307,7 @@ def test_attention_tc_items_beyond_the_resident_grid(seq):
     """64 < seq <= 128: the persistent tcgen05 kernel runs about four CTAs per
     SM, each taking (sequence, head) items in turn and loading the next item's
     Q, K and V while it computes the current one.  64 sequences x 12 heads =
-    768 items, more than one item per CTA; lengths 0 (zero rows), 1, multiples of 16
+    768 items, more than the resident CTAs; lengths 0 (zero rows), 1, multiples of 16
     and their neighbours, and seq itself.  Every row of every item against the
     oracle; a second call gives the same bits."""
     shape = (12, 64, 3072)
